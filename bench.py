@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark: expert-FFN HBM GB/s at batch-1 decode (MXFP4 DeepSeek-V4-Flash
+MoE layer: 256 experts, top-6, hidden 4096, intermediate 2048, 1 token).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+A step is one pass of the hot path over one decode token of one layer:
+router (softmax top-6) + routed-expert FFN (gate/up, SwiGLU, down, weighted
+combine).  Steps rotate over `--layers` distinct resident layers (16 x 3.42 GB
+by default), so each step's six experts are cold in L2 (inputs larger than L2).
+The timed region replays pre-captured CUDA graphs (one router graph, one FFN
+graph per layer); CUDA events bracket every FFN call for the roofline.
+
+`value` = algorithmic bytes (the six selected experts' packed bytes, read
+once) x steps / device time, summed over ranks (one independent replica per
+GPU, weak scaling).  `e2e` repeats the measurement through the C ABI with
+pinned host buffers and the host<->device copies inside the timed region.
+`--impl reference` times the CPU oracle on the same workload and metric.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "expert-FFN HBM GB/s (% of peak) at bs=1 decode; prefill tokens/s per MoE layer"
+WORKLOAD = "decode_mx"
+WORKLOAD_DESC = ("decode MoE layer: 256 experts, top-6, hidden 4096, intermediate 2048, "
+                 "batch 1, MXFP4 gate/up/down (e8m0 exponents 2^-9..2^0), bf16 N(0,1) "
+                 "activations, softmax top-6 router")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=16)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-sample-s", type=float, default=15.0)
+    ap.add_argument("--reference-budget-s", type=float, default=150.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, dev_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            p = torch.cuda.get_device_properties(dev_index)
+            try:
+                bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _reasons(self):
+        try:
+            return self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _one(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        r = self._reasons()
+        for bit, name in self.REASONS.items():
+            if r & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._one()
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._one()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._one()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    from block_quantized_expert_mxfp4_b200 import build as b
+    h = hashlib.sha256()
+    for p in sorted(b.sources()) + [os.path.join(b.CSRC, n) for n in sorted(os.listdir(b.CSRC))
+                                    if n.endswith((".cuh", ".h"))]:
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """dram bytes per FFN call from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_mx_traffic.json")) as f:
+            d = json.load(f)
+        if d.get("kernel_source_hash") == kernel_source_hash():
+            return d["dram_bytes_per_forward"]
+    except Exception:
+        pass
+    return None
+
+
+# -------------------------------------------------------------- CPU oracle --
+def oracle_sample(seconds: float, max_steps: int = 1 << 30):
+    """Time the CPU oracle on (token, expert) pairs of the decode workload.
+    Returns (bytes, seconds, steps, threads)."""
+    import numpy as np
+    import oracle
+    from block_quantized_expert_mxfp4_b200 import synth
+
+    oracle.build()
+    wl = synth.WORKLOADS[WORKLOAD]
+    lg = synth.router_logits(7, 64, wl.E, stream=99)
+    x = synth.activations(7, 64, wl.H, stream=99)
+    ids, _ = oracle.route_topk(lg, wl.k)
+    per_pair = 3 * (wl.I * wl.H // 2 + wl.I * wl.H // 32)
+    done, t_used, steps = 0, 0.0, 0
+    cache = {}
+    while t_used < seconds and steps < max_steps:
+        t, s = divmod(steps, wl.k)
+        t %= 4  # the experts of 4 tokens (24 pairs) are generated once, then reused
+        e = int(ids[t, s])
+        if e not in cache:
+            ws = []
+            for pi, (rows, cols) in enumerate(((wl.I, wl.H), (wl.I, wl.H), (wl.H, wl.I))):
+                q, sc = synth.mx_expert_bytes(0, 0, pi, rows, cols, wl.code_lo, wl.code_hi, [e],
+                                              wl.E)
+                ws.append(oracle.Weight(oracle.MXFP4, q, sc))
+            cache[e] = oracle.Layer(*ws)
+        L = cache[e]
+        t0 = time.perf_counter()
+        oracle.route_topk(lg[t:t + 1], wl.k)
+        oracle.expert_ffn(L, 0, x[t])
+        t_used += time.perf_counter() - t0
+        done += per_pair
+        steps += 1
+    return done, t_used, steps, oracle.get_threads()
+
+
+# ------------------------------------------------------------------ ours --
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import block_quantized_expert_mxfp4_b200 as qk
+    from block_quantized_expert_mxfp4_b200 import build as qk_build, synth, workload
+
+    qk_build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = synth.WORKLOADS[WORKLOAD]
+    T, k = wl.T, wl.k
+    L = args.layers
+    layers = [workload.make_layer(wl, seed=rank, layer=l) for l in range(L)]
+    expert_bytes = layers[0].expert_bytes()
+    bytes_per_step = k * T * expert_bytes if T == 1 else None  # T=1: k distinct experts
+
+    # per-slot inputs and outputs (distinct token per slot)
+    xs = [synth.activations(rank, T, wl.H, stream=l).to(dev) for l in range(L)]
+    lgs = [synth.router_logits(rank, T, wl.E, stream=l).to(dev) for l in range(L)]
+    ids = [torch.empty((T, k), dtype=torch.int32, device=dev) for _ in range(L)]
+    ws_ = [torch.empty((T, k), dtype=torch.float32, device=dev) for _ in range(L)]
+    ys = [torch.empty((T, wl.H), dtype=torch.float32, device=dev) for _ in range(L)]
+    lays = [lay.c() for lay in layers]
+    wsp = torch.empty(qk.moe_expert_workspace_size(lays[0], T, k), dtype=torch.uint8, device=dev)
+
+    def route(l, stream=None):
+        qk.moe_route_topk(lgs[l], k, ids[l], ws_[l], stream)
+
+    def ffn(l, stream=None):
+        qk.moe_expert_forward(lays[l], xs[l], ids[l], ws_[l], ys[l], wsp, stream=stream)
+
+    # warm-up eagerly (sets kernel attributes), then capture graphs
+    for l in range(L):
+        route(l)
+        ffn(l)
+    torch.cuda.synchronize()
+    if qk.qk_last_device_status() != qk.QK_OK:
+        raise RuntimeError("device status after warm-up")
+    s = torch.cuda.Stream(device=dev)
+    # G_all: L steps back to back (the throughput region); g_step[l]: one step;
+    # G_ev: L steps with external event nodes bracketing every FFN call.
+    ev_a = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(L)]
+    ev_b = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(L)]
+    G_all, G_ev, g_step = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), []
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(G_all, stream=s):
+            for l in range(L):
+                route(l)
+                ffn(l)
+        with torch.cuda.graph(G_ev, stream=s):
+            for l in range(L):
+                route(l)
+                ev_a[l].record(s)
+                ffn(l)
+                ev_b[l].record(s)
+        for l in range(L):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                route(l)
+                ffn(l)
+            g_step.append(g)
+    torch.cuda.synchronize()
+
+    K, W = args.steps, max(3, args.warmup)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    with torch.cuda.stream(s):
+        for i in range(W):
+            g_step[i % L].replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        torch.cuda._sleep(20_000_000)  # lets the host queue ahead of the GPU (untimed)
+        ev0.record(s)
+        for _ in range(K // L):
+            G_all.replay()
+        for i in range(K % L):
+            g_step[i].replay()
+        ev1.record(s)
+        torch.cuda.synchronize()
+        clocks.stop()
+        # roofline region: per-call device time of the FFN (events inside the graph)
+        ffn_ms = []
+        for _ in range(max(1, min(K, 2048) // L)):
+            G_ev.replay()
+            torch.cuda.synchronize()
+            ffn_ms += [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+    if world > 1:
+        dist.barrier()
+    st = qk.qk_last_device_status()
+    if st != qk.QK_OK:
+        raise RuntimeError(f"device status {qk.status_string(st)}")
+    elapsed = ev0.elapsed_time(ev1) / 1e3
+    ffn_s = statistics.fmean(ffn_ms) / 1e3
+    t_max = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    elapsed_max = float(t_max.item())
+    total_bytes = bytes_per_step * K * world
+    value = total_bytes / elapsed_max / 1e9
+
+    # ---- e2e through the C ABI with pinned host buffers
+    E2 = min(args.e2e_steps, K)
+    xh = [synth.activations(rank, T, wl.H, stream=1000 + i % 64).pin_memory() for i in range(64)]
+    lh = [synth.router_logits(rank, T, wl.E, stream=1000 + i % 64).pin_memory() for i in range(64)]
+    yh = torch.empty((T, wl.H), dtype=torch.float32).pin_memory()
+    xd, ld = xs[0].clone(), lgs[0].clone()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        for i in range(3):
+            xd.copy_(xh[i], non_blocking=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(s)
+        for i in range(E2):
+            l = i % L
+            xd.copy_(xh[i % 64], non_blocking=True)
+            ld.copy_(lh[i % 64], non_blocking=True)
+            qk.moe_route_topk(ld, k, ids[l], ws_[l], s)
+            qk.moe_expert_forward(lays[l], xd, ids[l], ws_[l], ys[l], wsp, stream=s)
+            yh.copy_(ys[l], non_blocking=True)
+        e1.record(s)
+        torch.cuda.synchronize()
+    e2e_t = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = bytes_per_step * E2 * world / float(e2e_t.item()) / 1e9
+
+    peak, peak_kind = peaks()
+    achieved = bytes_per_step / ffn_s / 1e9
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(elapsed_max / K * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e2m1/e8m0 weights -> f16 MMA, f32 accumulate",
+        "data": "synthetic (seeded; random-init MXFP4 weights of the DeepSeek-V4-Flash expert shape)",
+        "config": {"workload": WORKLOAD_DESC, "layers_resident": L,
+                   "resident_weight_GB": round(L * wl.E * expert_bytes / 1e9, 2),
+                   "bytes_per_step": bytes_per_step,
+                   "l2": "inputs larger than L2: steps rotate over the resident layers",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "moe_expert_forward (k_gateup -> k_down, PDL-chained)",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "ffn_us": round(ffn_s * 1e6, 3), "ffn_calls_timed": len(ffn_ms),
+                     "traffic": recorded_traffic()},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": T * wl.H * 2 + T * wl.E * 4,
+                "d2h_bytes_per_step": T * wl.H * 4, "steps": E2},
+        "gpu_launches": 3 * K,
+        "clocks": clocks.summary(),
+    }
+    return out
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from block_quantized_expert_mxfp4_b200 import synth
+        wl = synth.WORKLOADS[WORKLOAD]
+        nbytes, secs, steps, thr = oracle_sample(args.reference_budget_s, args.steps + args.warmup)
+        v = nbytes / secs / 1e9
+        line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+                "n_gpus": 1, "steps": steps, "warmup": 0,
+                "ms_per_step": round(secs / max(steps, 1) * 1e3, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 dequantized weights)",
+                "data": "synthetic (seeded)",
+                "config": {"workload": WORKLOAD_DESC, "parallelism": "host cores"},
+                "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": thr,
+                                 "kind": "oracle",
+                                 "sample": f"{steps} (token, expert) pairs of the decode layer "
+                                           f"(13.37 MB of MXFP4 weights each), bounded by "
+                                           f"{args.reference_budget_s:.0f} s"},
+                "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nbytes, secs, steps, thr = oracle_sample(args.cpu_sample_s)
+        out["cpu_baseline"] = {
+            "value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": thr, "kind": "oracle",
+            "sample": f"{steps} (token, expert) pairs of the decode layer, {secs:.1f} s of CPU time"}
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

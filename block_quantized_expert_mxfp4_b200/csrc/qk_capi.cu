@@ -1,0 +1,154 @@
+// qk_capi.cu -- the extern "C" entry points of libqk.so declared in qk.h:
+// argument validation, workspace carving, dispatch, and the device status word.
+#include <cuda_runtime.h>
+
+#include "qk_device.cuh"
+#include "qk_internal.h"
+
+namespace qk {
+__device__ int g_status = 0;
+__device__ unsigned long long g_wait_limit_ns = 1000000000ull;
+}  // namespace qk
+
+using namespace qk;
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool weight_ok(const qk_weight& w, int rows, int cols, int E) {
+  if (w.fmt != QK_FMT_MXFP4 && w.fmt != QK_FMT_NVFP4) return false;
+  if (!w.q || !w.scales || !aligned16(w.q) || !aligned16(w.scales)) return false;
+  if (w.fmt == QK_FMT_NVFP4 && !w.scale_2) return false;
+  return w.rows == rows && w.cols == cols && w.n_experts == E;
+}
+
+static qk_status layer_ok(const qk_moe_layer* L) {
+  if (!L) return QK_ERR_INVALID_ARG;
+  const int H = L->hidden, I = L->inter, E = L->gate.n_experts;
+  if (H < 64 || I < 64 || H % 64 || I % 64 || E <= 0 || E > 32767) return QK_ERR_INVALID_ARG;
+  if (!weight_ok(L->gate, I, H, E) || !weight_ok(L->up, I, H, E) || !weight_ok(L->down, H, I, E))
+    return QK_ERR_INVALID_ARG;
+  return QK_OK;
+}
+
+extern "C" {
+
+size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_t top_k) {
+  if (layer_ok(L) != QK_OK || n_tokens < 0 || top_k < 1 || top_k > 8) return 0;
+  return decode_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
+}
+
+qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t n_tokens,
+                             const int32_t* topk_ids, const float* topk_w, int32_t top_k,
+                             void* y, int32_t y_is_bf16, int32_t act_quant, void* workspace,
+                             size_t workspace_bytes, qk_stream_t stream) {
+  const qk_status lrc = layer_ok(L);
+  if (lrc != QK_OK) return lrc;
+  if (n_tokens < 0 || top_k < 1 || top_k > 8) return QK_ERR_INVALID_ARG;
+  if (act_quant != QK_ACT_NONE) return QK_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return QK_OK;
+  if (!x_bf16 || !topk_ids || !topk_w || !y || !aligned16(x_bf16)) return QK_ERR_INVALID_ARG;
+  const size_t need = moe_expert_workspace_size(L, n_tokens, top_k);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return QK_ERR_WORKSPACE;
+  if ((int64_t)n_tokens * top_k > kMaxPairs) return QK_ERR_UNSUPPORTED;
+  DecodeArgs a = {};
+  a.gate = L->gate;
+  a.up = L->up;
+  a.down = L->down;
+  a.x = static_cast<const uint16_t*>(x_bf16);
+  a.ids = topk_ids;
+  a.w = topk_w;
+  a.y = y;
+  a.T = n_tokens;
+  a.k = top_k;
+  a.E = L->gate.n_experts;
+  a.H = L->hidden;
+  a.I = L->inter;
+  a.P = n_tokens * top_k;
+  a.y_bf16 = y_is_bf16 ? 1 : 0;
+  decode_carve(a, workspace);
+  return decode_forward(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qk_status moe_route_topk(const float* logits, int32_t n_tokens, int32_t n_experts, int32_t top_k,
+                         int32_t* ids, float* w, qk_stream_t stream) {
+  if (n_tokens < 0 || n_experts < 1 || n_experts > 2048 || top_k < 1 || top_k > 32 ||
+      top_k > n_experts)
+    return QK_ERR_INVALID_ARG;
+  if (n_tokens == 0) return QK_OK;
+  if (!logits || !ids || !w) return QK_ERR_INVALID_ARG;
+  return route_topk_launch(logits, n_tokens, n_experts, top_k, ids, w,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+qk_status quant_convert_mxfp4_to_nvfp4(const uint8_t* e8m0, int32_t n_experts, int32_t rows,
+                                       int32_t cols, uint8_t* e4m3, float* scale_2,
+                                       unsigned long long* n_inexact, qk_stream_t stream) {
+  if (n_experts < 0 || rows < 0 || cols <= 0 || cols % 32) return QK_ERR_INVALID_ARG;
+  if (!e8m0 || !e4m3 || !scale_2 || !n_inexact) return QK_ERR_INVALID_ARG;
+  return convert_launch(e8m0, n_experts, rows, cols, e4m3, scale_2, n_inexact,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+qk_status fp8_block_linear(const void* x_bf16, int32_t M, int32_t K, const uint8_t* w,
+                           const uint8_t* w_scale, int32_t N, void* y, int32_t y_is_bf16,
+                           qk_stream_t stream) {
+  if (M < 1 || K < 128 || K % 128 || N < 16 || N % 16) return QK_ERR_INVALID_ARG;
+  if (!x_bf16 || !w || !w_scale || !y || !aligned16(x_bf16) || !aligned16(w))
+    return QK_ERR_INVALID_ARG;
+  return fp8_linear_launch(x_bf16, M, K, w, w_scale, N, y, y_is_bf16 ? 1 : 0,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fp8_shared_expert_workspace_size(int32_t M, int32_t hidden, int32_t inter) {
+  if (M < 1 || hidden < 128 || inter < 128 || hidden % 128 || inter % 128) return 0;
+  return fp8_ffn_workspace_bytes(M, hidden, inter);
+}
+
+qk_status fp8_shared_expert_forward(const void* x_bf16, int32_t M, int32_t hidden, int32_t inter,
+                                    const uint8_t* w_gate, const uint8_t* s_gate,
+                                    const uint8_t* w_up, const uint8_t* s_up,
+                                    const uint8_t* w_down, const uint8_t* s_down, float* y,
+                                    void* workspace, size_t workspace_bytes, qk_stream_t stream) {
+  if (M < 1 || hidden < 128 || inter < 128 || hidden % 128 || inter % 128) return QK_ERR_INVALID_ARG;
+  if (!x_bf16 || !w_gate || !s_gate || !w_up || !s_up || !w_down || !s_down || !y)
+    return QK_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down))
+    return QK_ERR_INVALID_ARG;
+  const size_t need = fp8_shared_expert_workspace_size(M, hidden, inter);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return QK_ERR_WORKSPACE;
+  return fp8_ffn_launch(x_bf16, M, hidden, inter, w_gate, s_gate, w_up, s_up, w_down, s_down, y,
+                        workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qk_status qk_last_device_status(qk_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return QK_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return QK_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return QK_ERR_CUDA;
+  return v;
+}
+
+const char* qk_status_string(qk_status s) {
+  switch (s) {
+    case QK_OK: return "ok";
+    case QK_ERR_INVALID_ARG: return "invalid argument";
+    case QK_ERR_UNSUPPORTED: return "unsupported";
+    case QK_ERR_WORKSPACE: return "workspace missing or too small";
+    case QK_ERR_NAN_SCALE: return "NaN scale code";
+    case QK_ERR_CUDA: return "CUDA runtime error";
+    case QK_ERR_TIMEOUT: return "bounded device wait ran out";
+    default: return "unknown status";
+  }
+}
+
+qk_status qk_debug_set_wait_limit_ns(unsigned long long limit_ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &limit_ns, sizeof(limit_ns)) == cudaSuccess
+             ? QK_OK
+             : QK_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,203 @@
+// qk_device.cuh -- device helpers shared by the libqk kernels (sm_100a only).
+//
+// Thin wrappers over PTX instructions documented in the PTX ISA (mbarrier,
+// cp.async.bulk, ldmatrix, mma.sync, cvt with e2m1x2 / e4m3x2 / ue8m0x2
+// sources, griddepcontrol), the per-device status word, and bounded waits.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qk.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libqk targets sm_100a (B200) only"
+#endif
+
+namespace qk {
+
+// ---------------------------------------------------------------- status --
+// First device-side error wins; read and cleared by qk_last_device_status().
+extern __device__ int g_status;
+// Limit of every bounded wait, in ns (qk_debug_set_wait_limit_ns).
+extern __device__ unsigned long long g_wait_limit_ns;
+// Limit used when draining copies after a wait ran out (never 0).
+constexpr unsigned long long kDrainLimitNs = 1000000000ull;
+
+__device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// -------------------------------------------------------------- mbarrier --
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` for at most `limit_ns`; false if it ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 >= limit_ns) return false;
+  }
+}
+
+// 1-D bulk copy global -> shared, completing `bytes` on `bar`.  dst, src and
+// bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Same with an L2 eviction hint: weights are streamed once per call.
+__device__ __forceinline__ void bulk_g2s_evict_first(void* dst, const void* src, uint32_t bytes,
+                                                     uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
+      "%2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// ------------------------------------------------------ PDL (griddepcontrol)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;");
+}
+
+// ------------------------------------------------------------- ldmatrix --
+// Four 8x8 b16 matrices: lane l supplies the row address for matrix l/8, row
+// l%8; register j of lane (g = l/4, t = l%4) receives bytes [4t, 4t+4) of row
+// g of matrix j.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                            const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(row_addr)));
+}
+
+// Two matrices (lanes 0..15 supply the row addresses).
+__device__ __forceinline__ void ldmatrix_x2(uint32_t& r0, uint32_t& r1, const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(smem_u32(row_addr)));
+}
+
+// ------------------------------------------------------------------ mma --
+// D = A(16x16 f16, row) * B(16x8 f16, col) + C, fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ------------------------------------------------------------- converts --
+// Byte I of `w` (two e2m1 codes) -> f16x2, low nibble -> low half.
+template <int I>
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t w);
+#define QK_E2M1X2(IDX)                                                              \
+  template <>                                                                       \
+  __device__ __forceinline__ uint32_t e2m1x2_to_f16x2<IDX>(uint32_t w) {            \
+    uint32_t out;                                                                   \
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %1;\n"            \
+        " cvt.rn.f16x2.e2m1x2 %0, b" #IDX ";\n}\n"                                   \
+        : "=r"(out)                                                                 \
+        : "r"(w));                                                                  \
+    return out;                                                                     \
+  }
+QK_E2M1X2(0)
+QK_E2M1X2(1)
+QK_E2M1X2(2)
+QK_E2M1X2(3)
+#undef QK_E2M1X2
+
+// Low (I=0) or high (I=1) 16 bits of `w` (two e4m3 codes) -> f16x2.
+template <int I>
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w);
+#define QK_E4M3X2(IDX)                                                              \
+  template <>                                                                       \
+  __device__ __forceinline__ uint32_t e4m3x2_to_f16x2<IDX>(uint32_t w) {            \
+    uint32_t out;                                                                   \
+    asm("{\n .reg .b16 h0, h1;\n mov.b32 {h0, h1}, %1;\n"                           \
+        " cvt.rn.f16x2.e4m3x2 %0, h" #IDX ";\n}\n"                                   \
+        : "=r"(out)                                                                 \
+        : "r"(w));                                                                  \
+    return out;                                                                     \
+  }
+QK_E4M3X2(0)
+QK_E4M3X2(1)
+#undef QK_E4M3X2
+
+// e8m0 code -> fp32 2^(c-127) (c = 0 gives the subnormal 2^-127; c = 255 is
+// reported by the caller).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t c) {
+  return __uint_as_float(c ? (c << 23) : 0x00400000u);
+}
+
+// e4m3 (E4M3FN) code -> fp32, via the hardware e4m3x2 -> f16x2 conversion.
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  const uint32_t h = e4m3x2_to_f16x2<0>(c & 0xFFu);
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xFFFFu)));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// Power-of-two exponent s such that amax * 2^-s lies in [2^14, 2^15): the
+// largest magnitude keeps full f16 precision with headroom below 65504.
+__device__ __forceinline__ int f16_shift_for(float amax) {
+  if (!(amax > 0.f) || !isfinite(amax)) return 0;
+  return ilogbf(amax) - 14;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+}  // namespace qk

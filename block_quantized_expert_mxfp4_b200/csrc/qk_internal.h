@@ -1,0 +1,51 @@
+// qk_internal.h -- host-side declarations shared by the libqk translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "qk.h"
+
+namespace qk {
+
+constexpr int kMaxPairs = 128;  // decode path: tokens * top_k
+constexpr int kMaxStages = 6;   // deepest bulk-copy ring
+
+inline size_t align256(size_t n) { return (n + 255) / 256 * 256; }
+
+// Arguments of the decode kernels (passed by value as a kernel parameter).
+struct DecodeArgs {
+  qk_weight gate, up, down;
+  const uint16_t* x;  // bf16 [T][H]
+  const int32_t* ids; // [T][k]
+  const float* w;     // [T][k]
+  void* y;
+  int T, k, E, H, I, P;
+  int y_bf16;
+  int stages;
+  int rows_act;       // activation rows staged per tile (<= 8)
+  // workspace
+  float* h;           // [P][I] fp32
+  float* hmax;        // [P][I/8] per-tile absmax of h
+  float* part;        // [P][H] fp32 per-pair expert outputs
+  int* counters;      // [H/16]
+  int n_counters;
+};
+
+qk_status decode_forward(DecodeArgs args, cudaStream_t st);
+size_t decode_workspace_bytes(int T, int k, int H, int I);
+void decode_carve(DecodeArgs& a, void* ws);
+
+qk_status route_topk_launch(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                            cudaStream_t st);
+qk_status convert_launch(const uint8_t* e8m0, int E, int N, int K, uint8_t* e4m3, float* scale_2,
+                         unsigned long long* n_inexact, cudaStream_t st);
+qk_status fp8_linear_launch(const void* x, int M, int K, const uint8_t* w, const uint8_t* ws, int N,
+                            void* y, int y_bf16, cudaStream_t st);
+size_t fp8_ffn_workspace_bytes(int M, int H, int I);
+qk_status fp8_ffn_launch(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
+                         const uint8_t* wu, const uint8_t* su, const uint8_t* wd, const uint8_t* sd,
+                         float* y, void* ws, cudaStream_t st);
+
+}  // namespace qk

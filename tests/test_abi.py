@@ -1,0 +1,90 @@
+"""The C-ABI library loads on a CPU-only host and exports every symbol the
+header declares; host-side argument validation returns its status codes
+without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_quantized_expert_mxfp4_b200 as qk
+from block_quantized_expert_mxfp4_b200 import _lib
+from conftest import ROOT
+
+
+def _declared():
+    hdr = open(os.path.join(ROOT, "include", "qk.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_0-9]+)\s*\(", hdr, re.M)
+
+
+def test_library_exports_every_declared_symbol():
+    L = qk.load()
+    names = _declared()
+    assert len(names) == 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(_lib.SYMBOLS)
+
+
+def test_status_strings():
+    for code in range(7):
+        assert qk.status_string(code) not in ("", "unknown status")
+    assert qk.status_string(99) == "unknown status"
+
+
+def _fake_layer(H=4096, I=2048, E=256, fmts=(1, 1, 1)):
+    base = 1 << 20  # fake 16-aligned addresses: never dereferenced on these paths
+    ws = []
+    for i, ((r, c), f) in enumerate(zip(((I, H), (I, H), (H, I)), fmts)):
+        ws.append(_lib.qk_weight(f, base * (3 * i + 1), base * (3 * i + 2),
+                                 base * (3 * i + 3) if f == 2 else None, E, r, c))
+    return _lib.make_layer(*ws)
+
+
+def test_workspace_query_and_shape_validation():
+    L = qk.load()
+    lay = _fake_layer()
+    n1 = L.moe_expert_workspace_size(ctypes.byref(lay), 1, 6)
+    n16 = L.moe_expert_workspace_size(ctypes.byref(lay), 16, 6)
+    assert 0 < n1 < n16
+    assert L.moe_expert_workspace_size(ctypes.byref(lay), 1, 9) == 0        # top_k > 8
+    assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(H=4032 + 16)), 1, 6) == 0
+    assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(fmts=(1, 3, 1))), 1, 6) == 0
+    bad = _fake_layer()
+    bad.down.rows = 2048
+    assert L.moe_expert_workspace_size(ctypes.byref(bad), 1, 6) == 0
+    nv = _fake_layer(fmts=(2, 2, 2))
+    nv.up.scale_2 = None
+    assert L.moe_expert_workspace_size(ctypes.byref(nv), 1, 6) == 0
+
+
+def test_forward_argument_errors_are_synchronous():
+    L = qk.load()
+    lay = _fake_layer()
+    vp = ctypes.c_void_p
+    f = L.moe_expert_forward
+    p = vp(1 << 24)
+    ws = L.moe_expert_workspace_size(ctypes.byref(lay), 1, 6)
+    assert f(ctypes.byref(lay), p, 0, p, p, 6, p, 0, 0, p, ws, None) == qk.QK_OK  # T = 0
+    assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 1, p, ws, None) == qk.QK_ERR_UNSUPPORTED
+    assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 0, p, ws - 1, None) == qk.QK_ERR_WORKSPACE
+    assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 0, None, ws, None) == qk.QK_ERR_WORKSPACE
+    assert f(ctypes.byref(lay), None, 1, p, p, 6, p, 0, 0, p, ws, None) == qk.QK_ERR_INVALID_ARG
+    assert f(ctypes.byref(lay), vp((1 << 24) + 8), 1, p, p, 6, p, 0, 0, p, ws, None) == \
+        qk.QK_ERR_INVALID_ARG                                               # x not 16-B aligned
+    assert f(None, p, 1, p, p, 6, p, 0, 0, p, ws, None) == qk.QK_ERR_INVALID_ARG
+    assert L.moe_route_topk(p, 4, 8, 9, p, p, None) == qk.QK_ERR_INVALID_ARG  # k > E
+    assert L.moe_route_topk(p, 0, 8, 2, p, p, None) == qk.QK_OK
+    assert L.quant_convert_mxfp4_to_nvfp4(p, 2, 4, 48, p, p, p, None) == qk.QK_ERR_INVALID_ARG
+    assert L.fp8_block_linear(p, 1, 100, p, p, 16, p, 0, None) == qk.QK_ERR_INVALID_ARG
+    assert L.fp8_shared_expert_workspace_size(8, 4096, 2048) > 0
+    assert L.fp8_shared_expert_forward(p, 8, 4096, 2048, p, p, p, p, p, p, p, p, 0, None) == \
+        qk.QK_ERR_WORKSPACE
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        _lib.load()

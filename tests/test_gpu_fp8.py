@@ -1,0 +1,50 @@
+"""GPU parity: FP8 E4M3 block-128 linear and the fused shared-expert FFN."""
+import numpy as np
+import pytest
+import torch
+
+import block_quantized_expert_mxfp4_b200 as qk
+import oracle
+from block_quantized_expert_mxfp4_b200 import synth, workload
+from helpers import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("M,K,N", [(8, 4096, 2048), (3, 2048, 4096), (20, 512, 256),
+                                   (1, 128, 16), (8, 384, 144)])
+def test_fp8_block_linear(M, K, N):
+    w = synth.fp8_codes(3, M + K, N * K, "cuda").view(N, K)
+    s = synth.scale_codes(3, N + K, ((N + 127) // 128) * (K // 128), 118, 127, "cuda").view(
+        (N + 127) // 128, K // 128)
+    x = synth.activations(M, M, K)
+    y = torch.empty((M, N), device="cuda")
+    qk.fp8_block_linear(x.cuda(), w, s, y)
+    assert qk.qk_last_device_status() == qk.QK_OK
+    yo = oracle.fp8_block_linear(x, w.cpu(), s.cpu(), 128)
+    assert_parity(y.cpu().numpy(), yo, what=f"fp8 linear {M}x{K}x{N}")
+
+
+def test_fp8_block_linear_bf16_out():
+    M, K, N = 8, 1024, 512
+    w = synth.fp8_codes(4, 1, N * K, "cuda").view(N, K)
+    s = synth.scale_codes(4, 2, (N // 128) * (K // 128), 118, 127, "cuda").view(N // 128, K // 128)
+    x = synth.activations(4, M, K)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    qk.fp8_block_linear(x.cuda(), w, s, y)
+    assert_parity(y.float().cpu().numpy(), oracle.fp8_block_linear(x, w.cpu(), s.cpu()),
+                  what="fp8 bf16")
+
+
+@pytest.mark.parametrize("M", [8, 1, 13])
+def test_fp8_shared_expert_accumulates(M):
+    H, I = 4096, 2048
+    sh = workload.make_fp8_shared(0, 0, H, I)
+    x = synth.activations(11, M, H)
+    y0 = torch.from_numpy(np.random.default_rng(M).standard_normal((M, H)).astype(np.float32))
+    y = y0.cuda().clone()
+    ws = torch.empty(qk.fp8_shared_expert_workspace_size(M, H, I), dtype=torch.uint8, device="cuda")
+    qk.fp8_shared_expert_forward(x.cuda(), sh.wg, sh.sg, sh.wu, sh.su, sh.wd, sh.sd, y, ws)
+    assert qk.qk_last_device_status() == qk.QK_OK
+    so = oracle.fp8_swiglu_ffn(x, *(t.cpu() for t in (sh.wg, sh.sg, sh.wu, sh.su, sh.wd, sh.sd)))
+    assert_parity((y.cpu() - y0).numpy(), so, what=f"shared expert M={M}")
