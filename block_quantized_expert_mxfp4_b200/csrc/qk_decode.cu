@@ -188,8 +188,8 @@ __host__ __device__ inline Geo make_geo(int K, int fa, int fb) {
 // Fixed shared-memory header (routing, barriers, reduction buffers).
 struct SmemHead {
   Route R;
-  uint64_t full[kMaxStages];
-  float red[kWarps * 32 * 4];
+  alignas(8) uint64_t full[kMaxStages];
+  alignas(16) float red[kWarps * 32 * 4];  // read and written as float4
   float mx_red[kWarps * kTileN];
   float mx_out[kTileN];
   int shift[kTileN];

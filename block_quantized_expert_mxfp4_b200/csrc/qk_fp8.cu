@@ -36,8 +36,8 @@ struct Fp8Args {
 };
 
 struct Fp8Head {
-  uint64_t full[kMaxStages];
-  float red[kWarps * 32 * 4];
+  alignas(8) uint64_t full[kMaxStages];
+  alignas(16) float red[kWarps * 32 * 4];  // read and written as float4
   float mx_red[kWarps * kTileN];
   float mx_out[kTileN];
   int shift[kTileN];

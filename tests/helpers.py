@@ -1,5 +1,8 @@
 """Shared test helpers: oracle sub-layers regenerated on the host from the
 seeded generators, and the parity metrics."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -52,6 +55,10 @@ def cosine(got, ref):
 
 def assert_parity(got, ref, tol=TOL_REL, cos=TOL_COS, what=""):
     e, c = rel_err(got, ref), cosine(got, ref)
+    log = os.environ.get("QK_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"case": what, "max_rel": e, "cosine": c, "tol": tol}) + "\n")
     assert np.all(np.isfinite(np.asarray(got, dtype=np.float64))), what
     assert e <= tol and c >= cos, f"{what}: max-rel {e:.3e} (tol {tol}), cosine {c:.7f}"
     return e, c
