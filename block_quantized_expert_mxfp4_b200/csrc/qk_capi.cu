@@ -24,7 +24,7 @@ static bool weight_ok(const qk_weight& w, int rows, int cols, int E) {
 static qk_status layer_ok(const qk_moe_layer* L) {
   if (!L) return QK_ERR_INVALID_ARG;
   const int H = L->hidden, I = L->inter, E = L->gate.n_experts;
-  if (H < 64 || I < 64 || H % 64 || I % 64 || E <= 0 || E > 32767) return QK_ERR_INVALID_ARG;
+  if (H < 128 || I < 128 || H % 128 || I % 128 || E <= 0 || E > 32767) return QK_ERR_INVALID_ARG;
   if (!weight_ok(L->gate, I, H, E) || !weight_ok(L->up, I, H, E) || !weight_ok(L->down, H, I, E))
     return QK_ERR_INVALID_ARG;
   return QK_OK;

@@ -1,4 +1,4 @@
-// qk_decode.cu -- decode path of moe_expert_forward (a few tokens per call).
+// qk_decode.cu -- decode path of moe_expert_forward (up to 16 tokens per call).
 //
 // The routed-expert FFN of a DeepSeek-V4-Flash-style MoE layer
 // ("DeepSeek-V4-Flash-W4A16-FP8", base-model table: hidden 4096, 256 routed
@@ -7,46 +7,125 @@
 // conversion"; gate+up carry ~2/3 of the expert bytes, "Why this mix?").
 //
 // Two kernels, chained with programmatic dependent launch:
-//   k_gateup  h[p][n]  = silu(g) * u, g/u = gate/up row n of expert e(p) . x[t(p)]
-//   k_down    part[p][m] = down row m of expert e(p) . h[p];  y[t] = sum_s w * part
-// Work unit: k_gateup = 8 output rows (8 gate + 8 up weight rows = one 16-row
-// MMA tile), k_down = 16 output rows, both over the full reduction length.
-// The unit's packed rows are copied by the bulk-copy (TMA) engine into padded
-// shared-memory rows, a ring of stages deep.  Eight warps split the reduction
-// dimension; each forms m16n8k16 A fragments with ldmatrix and the hardware
-// e2m1x2 -> f16x2 conversion (exact), multiplies with f16 activations on the
-// tensor cores (fp32 accumulate) and applies the block scale in fp32:
-//   MXFP4: once per 32-block on the fp32 partial (2^(c-127), exact)
-//   NVFP4: the e4m3 scale is folded into the f16 A fragment (e2m1*e4m3 is
-//          exact in f16), scale_2 at the end.
-// Activations enter the MMA as f16 scaled by a power of two per token (x) or
-// per pair (h) so that the largest magnitude sits in [2^14, 2^15).
+//   k_gateup  h[p][n] = silu(gate_n . x_t) * (up_n . x_t)       for pair p = (t, s)
+//   k_down    y[t][m] = sum_s w[t][s] * (down_m . h_p)          (fixed slot order)
 //
-// Token columns: the N=8 side of the MMA holds up to 8 tokens routed to the
-// unit's expert; more tokens are processed in further 8-column tiles.
+// Work decomposition.  A "virtual expert" is an expert together with up to 8
+// of its routed pairs (one m16n8k16 N-tile); experts with more pairs become
+// several virtual experts.  A unit is one 16-row MMA tile of a virtual expert
+// (k_gateup: 8 gate rows + the same 8 up rows; k_down: 16 down rows) over the
+// full reduction length, cut into chunks of Kc.  All chunks of the call are
+// split evenly and contiguously over the CTAs, and each CTA's range evenly over
+// its warps, so every warp streams about the same number of bytes.  A unit cut
+// by a range boundary is finished by the last of its owners (a per-unit
+// counter; partial sums added in chunk order, so results are deterministic for
+// a given grid).
+//
+// Data path.  Each warp streams its chunks through its own ring of shared-
+// memory stages with cp.async (16 bytes per lane, one instruction per 512-byte
+// packed row, asynchronous issue), rows padded by 16 bytes so ldmatrix reads
+// them without bank conflicts.  A thread forms m16n8k16 A fragments with
+// ldmatrix and the hardware e2m1x2 -> f16x2 conversion (exact) and multiplies
+// on the tensor cores with f16 activations (fp32 accumulate):
+//   MXFP4: the fp32 partial of each 32-block is scaled by 2^(c-127) (exact);
+//   NVFP4: the e4m3 scale is folded into the f16 fragment (e2m1 * e4m3 is exact
+//          in f16) and scale_2 is applied at the end.
+// Activations are staged once per CTA segment as f16 rows scaled by a power of
+// two per row, chosen so the row's largest magnitude sits in [2^14, 2^15); their
+// loads are issued ahead of the weight stream.
 #include <algorithm>
 
 #include "qk_common.cuh"
 
 namespace qk {
 
+constexpr int kDW = 8;    // warps per CTA
+constexpr int kXCap = 8;  // activation rows staged per segment
+constexpr int kMaxD = 4;  // deepest ring per warp
 
 // --------------------------------------------------------------- routing --
-// Per-CTA routing tables built in shared memory from the ids (P <= kMaxPairs
-// <= blockDim, one pair per thread).  Active experts ascend by id; the pairs
-// of one expert ascend by pair index (= token-major order).
 struct Route {
-  int n_active;
-  int16_t act_expert[kMaxPairs];    // active experts, ascending id
-  int16_t act_cnt[kMaxPairs];       // pairs per active expert
-  int16_t act_off[kMaxPairs + 1];   // pair-list offsets per active expert
-  int16_t pair_list[kMaxPairs];     // pair indices, grouped by expert
+  int n_v;                         // virtual experts
+  int16_t v_expert[kMaxPairs];
+  int16_t v_p0[kMaxPairs];         // first entry in pair_list
+  int8_t v_n[kMaxPairs];           // pairs (1..8)
+  int16_t pair_list[kMaxPairs];    // pairs grouped by expert, ascending pair index
+  int16_t pair_v[kMaxPairs];       // virtual expert of pair p (-1: invalid id)
+  int8_t pair_j[kMaxPairs];        // column of pair p in its virtual expert
   int16_t tmp_e[kMaxPairs];
   int8_t tmp_first[kMaxPairs];
+  int16_t act_cnt[kMaxPairs];
+  int16_t act_off[kMaxPairs + 1];
+  int16_t act_v0[kMaxPairs + 1];
 };
 
+__device__ __forceinline__ void place_pair(Route& R, int p, int e, int slot, int rank, int total) {
+  const int pos = R.act_off[slot] + rank;
+  R.pair_list[pos] = (int16_t)p;
+  const int v = R.act_v0[slot] + rank / kTileN;
+  R.pair_v[p] = (int16_t)v;
+  R.pair_j[p] = (int8_t)(rank % kTileN);
+  if (rank % kTileN == 0) {
+    R.v_expert[v] = (int16_t)e;
+    R.v_p0[v] = (int16_t)pos;
+    R.v_n[v] = (int8_t)min(kTileN, total - rank);
+  }
+}
+
+// Routing tables from the ids.  Active experts ascend by id; the pairs of one
+// expert ascend by pair index.  P <= 32: one warp with match/ballot; larger P:
+// one pair per thread (P <= kMaxPairs <= blockDim).
 __device__ void build_route(const int32_t* __restrict__ ids, int P, int E, Route& R) {
-  const int p = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (P <= 32) {
+    if (tid < 32) {
+      int e = -1;
+      if (lane < P) {
+        e = ids[lane];
+        if (e < 0 || e >= E) {
+          set_status(QK_ERR_INVALID_ARG);
+          e = -1;
+        }
+        R.pair_v[lane] = -1;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const bool valid = e >= 0;
+      const bool first = valid && (__ffs(peers) - 1 == lane);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int total = __popc(peers);
+      const unsigned firsts = __ballot_sync(0xffffffffu, first);
+      int slot = 0;
+      for (int i = 0; i < 32; ++i) {
+        const int ei = __shfl_sync(0xffffffffu, e, i);
+        slot += ((firsts >> i) & 1u) && ei < e;
+      }
+      const int n_active = __popc(firsts);
+      if (first) R.act_cnt[slot] = (int16_t)total;
+      __syncwarp();
+      const int cnt = lane < n_active ? R.act_cnt[lane] : 0;
+      const int vcnt = (cnt + kTileN - 1) / kTileN;
+      int off = cnt, v0 = vcnt;  // inclusive scans over active slots
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, off, o), b = __shfl_up_sync(0xffffffffu, v0, o);
+        if (lane >= o) {
+          off += a;
+          v0 += b;
+        }
+      }
+      if (lane <= n_active) {
+        R.act_off[lane] = (int16_t)(off - cnt);
+        R.act_v0[lane] = (int16_t)(v0 - vcnt);
+      }
+      const int n_v = __shfl_sync(0xffffffffu, v0, 31);
+      if (lane == 0) R.n_v = n_v;
+      __syncwarp();
+      if (valid) place_pair(R, lane, e, slot, rank, total);
+    }
+    __syncthreads();
+    return;
+  }
+  const int p = tid;
   int e = -1;
   if (p < P) {
     e = ids[p];
@@ -55,6 +134,7 @@ __device__ void build_route(const int32_t* __restrict__ ids, int P, int E, Route
       e = -1;
     }
     R.tmp_e[p] = (int16_t)e;
+    R.pair_v[p] = -1;
   }
   __syncthreads();
   int first = (e >= 0);
@@ -69,72 +149,159 @@ __device__ void build_route(const int32_t* __restrict__ ids, int P, int E, Route
       rank += (q < p && eq == e);
       total += (eq == e);
     }
-    if (first) {
-      R.act_expert[slot] = (int16_t)e;
-      R.act_cnt[slot] = (int16_t)total;
-    }
+    if (first) R.act_cnt[slot] = (int16_t)total;
   }
-  if (p == 0) R.n_active = n_active;
   __syncthreads();
   if (p <= n_active) {
-    int off = 0;
-    for (int a = 0; a < p; ++a) off += R.act_cnt[a];
+    int off = 0, v0 = 0;
+    for (int a = 0; a < p; ++a) {
+      off += R.act_cnt[a];
+      v0 += (R.act_cnt[a] + kTileN - 1) / kTileN;
+    }
     R.act_off[p] = (int16_t)off;
+    R.act_v0[p] = (int16_t)v0;
   }
   __syncthreads();
-  if (e >= 0) R.pair_list[R.act_off[slot] + rank] = (int16_t)p;
+  if (e >= 0) place_pair(R, p, e, slot, rank, total);
+  if (p == 0) R.n_v = R.act_v0[n_active];
   __syncthreads();
 }
 
-// Decoded scale for the fragment rows of one 32-block.
-//  MX: fp32 2^(c-127), applied to the fp32 partial.
-//  NV: f16x2 broadcast of the e4m3 scale of this thread's 16-half, applied to A.
-template <int FMT>
-struct BlockScale;
-
-template <>
-struct BlockScale<QK_FMT_MXFP4> {
-  float f;
-  __device__ __forceinline__ void load(const uint8_t* row_scales, int blk, int /*t*/, bool& bad) {
-    const uint32_t c = row_scales[blk];
-    bad |= (c == 255u);
-    f = e8m0_to_f32(c);
-  }
+// ------------------------------------------------------------- geometry --
+// Shared by host and device: one warp's stage holds a chunk's 16 packed rows
+// (stride Kc/2 + 16 bytes) followed by its 16 scale-row slices.
+struct DGeo {
+  int K, Kc;        // reduction length, chunk length
+  int nk;           // chunks per unit
+  int nbc;          // 32-blocks per chunk
+  int nib;          // padded bytes per packed smem row (Kc/2 + 16)
+  int sc_off;       // offset of the scale rows in a stage
+  int sca, scb;     // scale bytes per chunk row, rows 0..7 / 8..15
+  int sca_g, scb_g; // scale bytes per global row (full K)
+  int sc_vec;       // bytes per scale cp.async (16 or 4)
+  int stage;        // bytes per stage (128-multiple)
+  int act_stride;   // halves per staged activation row
+  int xcap;         // staged activation rows
+  int D;            // stages per warp
+  int smem;         // total dynamic shared memory
 };
 
-template <>
-struct BlockScale<QK_FMT_NVFP4> {
-  uint32_t h2;
-  __device__ __forceinline__ void load(const uint8_t* row_scales, int blk, int t, bool& bad) {
-    const uint32_t c = row_scales[2 * blk + (t >> 1)];
-    bad |= ((c & 0x7Fu) == 0x7Fu);
-    const uint32_t h = e4m3x2_to_f16x2<0>(c) & 0xFFFFu;
-    h2 = h | (h << 16);
-  }
+__host__ __device__ inline int sc_row_bytes(int fmt, int K) {
+  return fmt == QK_FMT_MXFP4 ? K / 32 : K / 16;
+}
+
+struct DHead {
+  Route R;
+  int seg_v0, seg_v1, seg_rows;
+  int16_t row_key[kXCap];               // staged row -> token (k_gateup) or pair (k_down)
+  int8_t col_row[kMaxPairs * kTileN];   // (v - seg_v0, column) -> staged row
+  int shift[kXCap];
+  float red8[kDW][kXCap];
+};
+constexpr int kDHead = (int)((sizeof(DHead) + 127) / 128 * 128);
+
+__host__ __device__ inline DGeo make_dgeo(int K, int Kc, int fa, int fb, int xcap, int D) {
+  DGeo g;
+  g.K = K;
+  g.Kc = Kc;
+  g.nk = K / Kc;
+  g.nbc = Kc / 32;
+  g.nib = Kc / 2 + 16;
+  g.sca_g = sc_row_bytes(fa, K);
+  g.scb_g = sc_row_bytes(fb, K);
+  g.sca = sc_row_bytes(fa, Kc);
+  g.scb = sc_row_bytes(fb, Kc);
+  g.sc_vec = (g.sca % 16 || g.scb % 16 || g.sca_g % 16 || g.scb_g % 16) ? 4 : 16;
+  g.sc_off = 16 * g.nib;
+  g.stage = (g.sc_off + 8 * g.sca + 8 * g.scb + 127) / 128 * 128;
+  g.act_stride = K + 32;  // 2K+64 bytes: conflict-free 16-byte fragment loads
+  g.xcap = xcap;
+  g.D = D;
+  g.smem = kDHead + xcap * g.act_stride * 2 + kDW * D * g.stage;
+  return g;
+}
+
+struct DArgs {
+  DecodeArgs a;
+  DGeo G;
+  int RT;          // units (row tiles) per virtual expert
+  int64_t C_max;   // upper bound of chunks (grid sizing only)
 };
 
+// ---------------------------------------------------------- fragments --
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
-// One 32-block of a 16-row tile against one 8-column activation tile.
-// wa: A word of rows g (rows 0..7 of the tile), wb: rows g+8.  xb: the
-// thread's 8 f16 activations (4 regs).  acc rows g -> acc[0..1], g+8 -> acc[2..3].
+// Four e8m0 codes -> fp32 2^(c-127) (code 0 -> the subnormal 2^-127 exactly).
+__device__ __forceinline__ void ue8m0x4(uint32_t c4, float (&f)[4]) {
+  uint32_t lo, hi;
+  asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.bf16x2.ue8m0x2 %0, a;\n"
+      " cvt.rn.bf16x2.ue8m0x2 %1, b;\n}\n"
+      : "=r"(lo), "=r"(hi)
+      : "r"(c4));
+  f[0] = __uint_as_float(lo << 16);
+  f[1] = __uint_as_float(lo & 0xFFFF0000u);
+  f[2] = __uint_as_float(hi << 16);
+  f[3] = __uint_as_float(hi & 0xFFFF0000u);
+}
+
+__device__ __forceinline__ bool has_ff_byte(uint32_t c4) {
+  const uint32_t v = ~c4;
+  return ((v - 0x01010101u) & c4 & 0x80808080u) != 0u;
+}
+
+// Scales of 4 consecutive 32-blocks for one fragment row.
+template <int FMT>
+struct Scale4;
+
+template <>
+struct Scale4<QK_FMT_MXFP4> {
+  float f[4];
+  __device__ __forceinline__ void load(const uint8_t* row, int b, int /*t*/, bool& bad) {
+    const uint32_t c4 = *reinterpret_cast<const uint32_t*>(row + b);
+    bad |= has_ff_byte(c4);
+    ue8m0x4(c4, f);
+  }
+};
+
+template <>
+struct Scale4<QK_FMT_NVFP4> {
+  uint32_t h2[4];  // f16x2 broadcast of this thread's 16-half scale, per block
+  __device__ __forceinline__ void load(const uint8_t* row, int b, int t, bool& bad) {
+    const uint2 c = *reinterpret_cast<const uint2*>(row + 2 * b);
+    bad |= has_ff_byte(c.x | 0x80808080u) | has_ff_byte(c.y | 0x80808080u);
+    // thread t holds elements 8t..8t+7 of each 32-block: 16-half number t>>1
+    const uint32_t sel = (t >> 1) ? 0x3232u : 0x1010u;
+    const uint32_t w[2] = {c.x, c.y};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t h = (i & 1) ? e4m3x2_to_f16x2<1>(w[i >> 1]) : e4m3x2_to_f16x2<0>(w[i >> 1]);
+      h2[i] = __byte_perm(h, h, sel);
+    }
+  }
+};
+
+// One 32-block of the 16-row tile against one 8-column activation tile.
+// wa: A word of rows g (tile rows 0..7), wb: rows g+8.  xb: the thread's
+// 8 f16 activations of this block.  acc rows g -> acc[0..1], g+8 -> acc[2..3].
 template <int FA, int FB>
 __device__ __forceinline__ void block_mma(float (&acc)[4], uint32_t wa, uint32_t wb,
-                                          const uint4& xb, const BlockScale<FA>& sa,
-                                          const BlockScale<FB>& sb) {
+                                          const uint4& xb, const Scale4<FA>& sa,
+                                          const Scale4<FB>& sb, int i) {
   uint32_t a0 = e2m1x2_to_f16x2<0>(wa), a1 = e2m1x2_to_f16x2<0>(wb);
   uint32_t a2 = e2m1x2_to_f16x2<1>(wa), a3 = e2m1x2_to_f16x2<1>(wb);
   uint32_t c0 = e2m1x2_to_f16x2<2>(wa), c1 = e2m1x2_to_f16x2<2>(wb);
   uint32_t c2 = e2m1x2_to_f16x2<3>(wa), c3 = e2m1x2_to_f16x2<3>(wb);
   if constexpr (FA == QK_FMT_NVFP4) {
-    a0 = hmul2(a0, sa.h2); a2 = hmul2(a2, sa.h2); c0 = hmul2(c0, sa.h2); c2 = hmul2(c2, sa.h2);
+    a0 = hmul2(a0, sa.h2[i]); a2 = hmul2(a2, sa.h2[i]);
+    c0 = hmul2(c0, sa.h2[i]); c2 = hmul2(c2, sa.h2[i]);
   }
   if constexpr (FB == QK_FMT_NVFP4) {
-    a1 = hmul2(a1, sb.h2); a3 = hmul2(a3, sb.h2); c1 = hmul2(c1, sb.h2); c3 = hmul2(c3, sb.h2);
+    a1 = hmul2(a1, sb.h2[i]); a3 = hmul2(a3, sb.h2[i]);
+    c1 = hmul2(c1, sb.h2[i]); c3 = hmul2(c3, sb.h2[i]);
   }
   if constexpr (FA == QK_FMT_NVFP4 && FB == QK_FMT_NVFP4) {
     mma_f16_16816(acc, a0, a1, a2, a3, xb.x, xb.y);
@@ -144,15 +311,15 @@ __device__ __forceinline__ void block_mma(float (&acc)[4], uint32_t wa, uint32_t
     mma_f16_16816(d, a0, a1, a2, a3, xb.x, xb.y);
     mma_f16_16816(d, c0, c1, c2, c3, xb.z, xb.w);
     if constexpr (FA == QK_FMT_MXFP4) {
-      acc[0] = fmaf(d[0], sa.f, acc[0]);
-      acc[1] = fmaf(d[1], sa.f, acc[1]);
+      acc[0] = fmaf(d[0], sa.f[i], acc[0]);
+      acc[1] = fmaf(d[1], sa.f[i], acc[1]);
     } else {
       acc[0] += d[0];
       acc[1] += d[1];
     }
     if constexpr (FB == QK_FMT_MXFP4) {
-      acc[2] = fmaf(d[2], sb.f, acc[2]);
-      acc[3] = fmaf(d[3], sb.f, acc[3]);
+      acc[2] = fmaf(d[2], sb.f[i], acc[2]);
+      acc[3] = fmaf(d[3], sb.f[i], acc[3]);
     } else {
       acc[2] += d[2];
       acc[3] += d[3];
@@ -160,395 +327,562 @@ __device__ __forceinline__ void block_mma(float (&acc)[4], uint32_t wa, uint32_t
   }
 }
 
-template <int FMT>
-__host__ __device__ constexpr int scale_bytes_per_row(int K) {
-  return FMT == QK_FMT_MXFP4 ? K / 32 : K / 16;
-}
-
-// Shared-memory geometry of one kernel instantiation (host and device agree).
-struct Geo {
-  int K;           // reduction length (bytes of a packed row = K/2)
-  int nib_row;     // padded bytes per smem nibble row
-  int sca, scb;    // scale bytes per row, rows 0..7 and 8..15
-  int stage;       // bytes per stage
-  int act_stride;  // halves per activation row in smem
-};
-
-__host__ __device__ inline Geo make_geo(int K, int fa, int fb) {
-  Geo g;
-  g.K = K;
-  g.nib_row = K / 2 + 16;
-  g.sca = fa == QK_FMT_MXFP4 ? K / 32 : K / 16;
-  g.scb = fb == QK_FMT_MXFP4 ? K / 32 : K / 16;
-  g.stage = (16 * g.nib_row + 8 * g.sca + 8 * g.scb + 127) / 128 * 128;
-  g.act_stride = K + 32;  // 2K+64 bytes: conflict-free 16-B fragment loads
-  return g;
-}
-
-// Fixed shared-memory header (routing, barriers, reduction buffers).
-struct SmemHead {
-  Route R;
-  alignas(8) uint64_t full[kMaxStages];
-  alignas(16) float red[kWarps * 32 * 4];  // read and written as float4
-  float mx_red[kWarps * kTileN];
-  float mx_out[kTileN];
-  int shift[kTileN];
-  int rows[kTileN];
-  int flag;
-};
-
-constexpr int kHeadBytes = (int)((sizeof(SmemHead) + 127) / 128 * 128);
-
-// Issue the bulk copies of one unit: 16 nibble rows + the two scale slabs.
-// rows 0..7 come from (qa, sa) rows ra0.., rows 8..15 from (qb, sb) rows rb0..
-__device__ __forceinline__ void issue_unit(uint8_t* stage, uint64_t* bar, const Geo& G,
-                                           const uint8_t* qa, const uint8_t* sa, int64_t ra0,
-                                           const uint8_t* qb, const uint8_t* sb, int64_t rb0,
-                                           uint64_t pol) {
-  const int rb = G.K / 2;
-  mbar_arrive_expect_tx(bar, 16u * rb + 8u * G.sca + 8u * G.scb);
-#pragma unroll 1
-  for (int i = 0; i < 8; ++i) {
-    bulk_g2s_evict_first(stage + i * G.nib_row, qa + (ra0 + i) * rb, rb, bar, pol);
-    bulk_g2s_evict_first(stage + (8 + i) * G.nib_row, qb + (rb0 + i) * rb, rb, bar, pol);
-  }
-  uint8_t* sc = stage + 16 * G.nib_row;
-  bulk_g2s_evict_first(sc, sa + ra0 * G.sca, 8 * G.sca, bar, pol);
-  bulk_g2s_evict_first(sc + 8 * G.sca, sb + rb0 * G.scb, 8 * G.scb, bar, pol);
-}
-
-// Warp's share of one unit: 16 tile rows x its block range, one token tile.
+// One chunk of one unit (warp): 16 rows x Kc against one token tile.
+// st: the stage (packed rows, then scale rows); xrow: this thread's activation
+// row at the chunk's first block.
 template <int FA, int FB>
-__device__ __forceinline__ void unit_mma(float (&acc)[4], const uint8_t* stage, const Geo& G,
-                                         const __half* act, int rows_act, int warp, int lane,
-                                         bool& bad) {
+__device__ __forceinline__ void chunk_mma(float (&acc)[4], const uint8_t* st, const DGeo& G,
+                                          const __half* xrow, int lane, bool& bad) {
   const int g = lane >> 2, t = lane & 3;
-  const int nb = G.K / 32;
-  const int b0 = warp * nb / kWarps, b1 = (warp + 1) * nb / kWarps;
-  const uint8_t* sc_a = stage + 16 * G.nib_row + g * G.sca;
-  const uint8_t* sc_b = stage + 16 * G.nib_row + 8 * G.sca + g * G.scb;
-  // token columns past the staged rows read a staged row (their results are unused)
-  const __half* xrow = act + min(g, rows_act - 1) * G.act_stride + 8 * t;
-  // ldmatrix row address: matrix j = lane>>3 (0: rows 0-7 blk b, 1: rows 8-15
-  // blk b, 2: rows 0-7 blk b+1, 3: rows 8-15 blk b+1), row lane&7.
   const int mj = lane >> 3, mr = lane & 7;
-  const uint8_t* lrow = stage + ((mj & 1) * 8 + mr) * G.nib_row + (mj >> 1) * 16;
-  int b = b0;
-  for (; b + 1 < b1; b += 2) {
-    uint32_t wa0, wb0, wa1, wb1;
-    ldmatrix_x4(wa0, wb0, wa1, wb1, lrow + b * 16);
-    BlockScale<FA> sa0, sa1;
-    BlockScale<FB> sb0, sb1;
-    sa0.load(sc_a, b, t, bad);
-    sb0.load(sc_b, b, t, bad);
-    sa1.load(sc_a, b + 1, t, bad);
-    sb1.load(sc_b, b + 1, t, bad);
-    const uint4 x0 = *reinterpret_cast<const uint4*>(xrow + b * 32);
+  // ldmatrix row address: matrix mj (0: rows 0-7 blk b, 1: rows 8-15 blk b,
+  // 2: rows 0-7 blk b+1, 3: rows 8-15 blk b+1), row mr
+  const uint8_t* lrow = st + ((mj & 1) * 8 + mr) * G.nib + (mj >> 1) * 16;
+  const uint8_t* sa = st + G.sc_off + g * G.sca;
+  const uint8_t* sb = st + G.sc_off + 8 * G.sca + g * G.scb;
+#pragma unroll 2
+  for (int b = 0; b < G.nbc; b += 4) {
+    uint32_t w[8];
+    ldmatrix_x4(w[0], w[1], w[2], w[3], lrow + b * 16);
+    ldmatrix_x4(w[4], w[5], w[6], w[7], lrow + (b + 2) * 16);
+    Scale4<FA> s_a;
+    Scale4<FB> s_b;
+    s_a.load(sa, b, t, bad);
+    s_b.load(sb, b, t, bad);
+    const uint4 x0 = *reinterpret_cast<const uint4*>(xrow + (b + 0) * 32);
     const uint4 x1 = *reinterpret_cast<const uint4*>(xrow + (b + 1) * 32);
-    block_mma<FA, FB>(acc, wa0, wb0, x0, sa0, sb0);
-    block_mma<FA, FB>(acc, wa1, wb1, x1, sa1, sb1);
-  }
-  if (b < b1) {
-    uint32_t wa0, wb0;
-    ldmatrix_x2(wa0, wb0, lrow + b * 16);
-    BlockScale<FA> sa0;
-    BlockScale<FB> sb0;
-    sa0.load(sc_a, b, t, bad);
-    sb0.load(sc_b, b, t, bad);
-    const uint4 x0 = *reinterpret_cast<const uint4*>(xrow + b * 32);
-    block_mma<FA, FB>(acc, wa0, wb0, x0, sa0, sb0);
+    const uint4 x2 = *reinterpret_cast<const uint4*>(xrow + (b + 2) * 32);
+    const uint4 x3 = *reinterpret_cast<const uint4*>(xrow + (b + 3) * 32);
+    block_mma<FA, FB>(acc, w[0], w[1], x0, s_a, s_b, 0);
+    block_mma<FA, FB>(acc, w[2], w[3], x1, s_a, s_b, 1);
+    block_mma<FA, FB>(acc, w[4], w[5], x2, s_a, s_b, 2);
+    block_mma<FA, FB>(acc, w[6], w[7], x3, s_a, s_b, 3);
   }
 }
 
-// =================================================================== k1 ==
-template <int FG, int FU>
-__global__ void __launch_bounds__(kThreads, 1) k_gateup(const DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  SmemHead& S = *reinterpret_cast<SmemHead*>(smem);
-  const Geo G = make_geo(a.H, FG, FU);
-  __half* act = reinterpret_cast<__half*>(smem + kHeadBytes);
-  uint8_t* stages = smem + kHeadBytes + (size_t)a.rows_act * G.act_stride * 2;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nstage = a.stages;
-  const int tn = a.rows_act;  // token columns per tile = staged activation rows (<= 8)
+// Release the writes of this thread (and, through the preceding warp barrier,
+// of its warp) and acquire those of earlier arrivals.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 
-  pdl_launch_dependents();
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < a.n_counters; i += blockDim.x) a.counters[i] = 0;
+// cp.async global -> shared (L2 only), 16 bytes with an L2 evict-first hint, or 4 bytes.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
+               "l"(src), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_dyn(int n) {  // n in [0, kMaxD)
+  switch (n) {
+    case 0: cp_async_wait<0>(); break;
+    case 1: cp_async_wait<1>(); break;
+    case 2: cp_async_wait<2>(); break;
+    default: cp_async_wait<3>(); break;
+  }
+}
 
-  build_route(a.ids, a.P, a.E, S.R);
-  const int R1 = a.I / 8;
-  const int U = S.R.n_active * R1;
-  const int u0 = (int)((int64_t)U * blockIdx.x / gridDim.x);
-  const int u1 = (int)((int64_t)U * (blockIdx.x + 1) / gridDim.x);
-  const int n = u1 - u0;
-  if (n <= 0) return;
+// ------------------------------------------------------------- staging --
+// Stage the segment's activation rows as f16 scaled by 2^-shift[row]:
+// k_gateup: token rows of x (bf16 [T][H]); shift from the row's absmax.
+// k_down: pair rows of h (fp32 [P][I]); shift from k_gateup's per-tile maxima.
+// stage_issue() puts each thread's first batch of 16-byte loads in flight (it
+// runs before the weight stream starts); stage_finish() reduces the absmax,
+// converts and stores.
+constexpr int kBatch = 16;
 
-  const uint64_t pol = policy_evict_first();
-  auto issue = [&](int i) {
-    const int u = u0 + i, s = i % nstage;
-    const int e = S.R.act_expert[u / R1];
-    const int64_t row0 = (int64_t)e * a.I + (int64_t)(u % R1) * 8;
-    issue_unit(stages + (size_t)s * G.stage, &S.full[s], G, a.gate.q, a.gate.scales, row0, a.up.q,
-               a.up.scales, row0, pol);
-  };
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < nstage; ++s) mbar_init(&S.full[s], 1);
-    fence_mbar_init();
-    for (int i = 0; i < min(n, nstage); ++i) issue(i);
+struct StageRegs {
+  uint4 buf[kBatch];
+  float am[kXCap];
+};
+
+template <bool GATEUP>
+__device__ __forceinline__ const uint4* stage_src(const DecodeArgs& a, const DHead& S, int j, int nvec) {
+  const int row = j / nvec, q = j - row * nvec;
+  const int key = S.row_key[row];
+  return GATEUP ? reinterpret_cast<const uint4*>(a.x + (size_t)key * a.H) + q
+                : reinterpret_cast<const uint4*>(a.h + (size_t)key * a.I) + q;
+}
+
+template <bool GATEUP>
+__device__ __forceinline__ void stage_issue(const DecodeArgs& a, const DHead& S, StageRegs& R,
+                                            int nrows) {
+  const int tid = threadIdx.x, nth = kDW * 32;
+  const int nvec = GATEUP ? a.H / 8 : a.I / 4;  // 16-byte vectors per source row
+  const int total = nrows * nvec;
+#pragma unroll
+  for (int i = 0; i < kXCap; ++i) R.am[i] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kBatch; ++i) {
+    const int j = i * nth + tid;
+    if (j < total) R.buf[i] = GATEUP ? __ldg(stage_src<GATEUP>(a, S, j, nvec)) : __ldcg(stage_src<GATEUP>(a, S, j, nvec));
+  }
+  if (!GATEUP) {
+    const int R1 = a.I / 8;
+    for (int j = tid; j < nrows * R1; j += nth) {
+      const int row = j / R1;
+      const float m = __ldcg(a.hmax + (size_t)S.row_key[row] * R1 + (j - row * R1));
+#pragma unroll
+      for (int r = 0; r < kXCap; ++r)
+        if (r == row) R.am[r] = fmaxf(R.am[r], m);
+    }
+  }
+}
+
+__device__ __forceinline__ float bf16x8_absmax(const uint4& v) {
+  const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(wv[e] & 0xFFFFu)), fabsf(bf16_bits_to_f32(wv[e] >> 16))));
+  return m;
+}
+
+template <bool GATEUP>
+__device__ __forceinline__ void stage_finish(const DecodeArgs& a, DHead& S, StageRegs& R,
+                                             __half* act, int stride, int nrows) {
+  const int tid = threadIdx.x, nth = kDW * 32;
+  const int nvec = GATEUP ? a.H / 8 : a.I / 4;
+  const int total = nrows * nvec;
+  const bool held = total <= kBatch * nth;
+  if (GATEUP) {  // absmax over the x rows (first batch in registers, the rest re-read)
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int j = i * nth + tid;
+      if (j < total) {
+        const float m = bf16x8_absmax(R.buf[i]);
+        const int row = j / nvec;
+#pragma unroll
+        for (int r = 0; r < kXCap; ++r)
+          if (r == row) R.am[r] = fmaxf(R.am[r], m);
+      }
+    }
+    for (int j = kBatch * nth + tid; j < total; j += nth) {
+      const float m = bf16x8_absmax(__ldg(stage_src<GATEUP>(a, S, j, nvec)));
+      const int row = j / nvec;
+#pragma unroll
+      for (int r = 0; r < kXCap; ++r)
+        if (r == row) R.am[r] = fmaxf(R.am[r], m);
+    }
+  }
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int r = 0; r < kXCap; ++r) {
+    float m = R.am[r];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) S.red8[warp][r] = m;
   }
   __syncthreads();
-
-  bool bad = false;
-  int cur_a = -1;
-  const unsigned long long limit = g_wait_limit_ns;
-  for (int i = 0; i < n; ++i) {
-    const int u = u0 + i, s = i % nstage;
-    const int as = u / R1, r = u % R1;
-    const int e = S.R.act_expert[as];
-    const int p0 = S.R.act_off[as], np = S.R.act_off[as + 1] - p0;
-    const uint8_t* st = stages + (size_t)s * G.stage;
-    const bool ready = mbar_wait_bounded(&S.full[s], (i / nstage) & 1, limit);
-    if (__syncthreads_or(!ready)) {
-      drain_stages(S.full, i, min(n, i + nstage), nstage);
-      return;
-    }
-    for (int tile = 0; tile * tn < np; ++tile) {
-      const int nt = min(tn, np - tile * tn);
-      if (as != cur_a || np > tn) {
-        if (threadIdx.x < kTileN)
-          S.rows[threadIdx.x] =
-              threadIdx.x < nt ? S.R.pair_list[p0 + tile * tn + threadIdx.x] / a.k : 0;
-        __syncthreads();
-        stage_bf16_rows(a.x, S.rows, nt, a.H, act, G.act_stride, S.shift, S.mx_red, S.mx_out);
-        cur_a = as;
+  if (tid < nrows) {
+    float m = 0.f;
+    for (int w = 0; w < kDW; ++w) m = fmaxf(m, S.red8[w][tid]);
+    S.shift[tid] = clamp_shift(f16_shift_for(m));
+  }
+  __syncthreads();
+  for (int base = 0; base < total; base += kBatch * nth) {
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int j = base + i * nth + tid;
+      if (j >= total) continue;
+      const uint4 v = (held || base == 0) ? R.buf[i]
+                      : (GATEUP ? __ldg(stage_src<GATEUP>(a, S, j, nvec))
+                                : __ldcg(stage_src<GATEUP>(a, S, j, nvec)));
+      const int row = j / nvec, q = j - row * nvec;
+      const float sc = pow2f(-S.shift[row]);
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      if (GATEUP) {  // 8 bf16 -> 8 f16
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          o[e] = pack_f16x2(bf16_bits_to_f32(wv[e] & 0xFFFFu) * sc, bf16_bits_to_f32(wv[e] >> 16) * sc);
+        reinterpret_cast<uint4*>(act + (size_t)row * stride)[q] = make_uint4(o[0], o[1], o[2], o[3]);
+      } else {  // 4 fp32 -> 4 f16
+        const uint2 o = make_uint2(pack_f16x2(__uint_as_float(wv[0]) * sc, __uint_as_float(wv[1]) * sc),
+                                   pack_f16x2(__uint_as_float(wv[2]) * sc, __uint_as_float(wv[3]) * sc));
+        reinterpret_cast<uint2*>(act + (size_t)row * stride)[q] = o;
       }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      unit_mma<FG, FU>(acc, st, G, act, a.rows_act, warp, lane, bad);
-      if (reduce_warps(acc, S.red, warp, lane)) {
-        const int g = lane >> 2, t = lane & 3;
-        const float s2g = FG == QK_FMT_NVFP4 ? a.gate.scale_2[e] : 1.f;
-        const float s2u = FU == QK_FMT_NVFP4 ? a.up.scale_2[e] : 1.f;
+    }
+  }
+}
+
+// ------------------------------------------------------------ the kernel --
+// Unit u = v * RT + r; chunk c = u * nk + kc.
+template <int FA, int FB, bool GATEUP>
+__global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ DArgs P) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  DHead& S = *reinterpret_cast<DHead*>(smem);
+  const DecodeArgs& a = P.a;
+  const DGeo& G = P.G;
+  __half* act = reinterpret_cast<__half*>(smem + kDHead);
+  uint8_t* rings = smem + kDHead + (size_t)G.xcap * G.act_stride * 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  uint8_t* ring = rings + (size_t)warp * G.D * G.stage;
+  const int RT = P.RT, nk = G.nk;
+  const qk_weight& WA = GATEUP ? a.gate : a.down;
+  const qk_weight& WB = GATEUP ? a.up : a.down;
+  const int rows_per_e = GATEUP ? a.I : a.H;  // weight rows of one expert
+
+  if (GATEUP) pdl_launch_dependents();
+  build_route(a.ids, a.P, a.E, S.R);
+  const int64_t C = (int64_t)S.R.n_v * RT * nk;
+  const int64_t c0 = C * blockIdx.x / gridDim.x, c1 = C * (blockIdx.x + 1) / gridDim.x;
+  if (c0 >= c1) return;
+
+  const uint64_t pol = policy_evict_first();
+  const int vpr = G.Kc / 32;  // 16-byte vectors per packed chunk row
+  // All 32 lanes: cp.async of chunk c into stage `slot` (not committed).
+  auto issue = [&](int64_t c, int slot) {
+    uint8_t* st = ring + (size_t)slot * G.stage;
+    const int64_t u = c / nk;
+    const int kc = (int)(c - u * nk);
+    const int v = (int)(u / RT), r = (int)(u - (int64_t)v * RT);
+    const int e = S.R.v_expert[v];
+    const int64_t rowA0 = (int64_t)e * rows_per_e + (GATEUP ? r * 8 : r * 16);
+    const int64_t rowB0 = GATEUP ? rowA0 : rowA0 + 8;
+    const uint8_t* qa = WA.q + rowA0 * (G.K / 2) + (size_t)kc * (G.Kc / 2);
+    const uint8_t* qb = WB.q + rowB0 * (G.K / 2) + (size_t)kc * (G.Kc / 2);
+#pragma unroll 4
+    for (int idx = lane; idx < 16 * vpr; idx += 32) {
+      const int row = idx / vpr, vi = idx - row * vpr;
+      const uint8_t* src = (row < 8 ? qa + (size_t)row * (G.K / 2) : qb + (size_t)(row - 8) * (G.K / 2)) + vi * 16;
+      cp_async16(st + row * G.nib + vi * 16, src, pol);
+    }
+    const uint8_t* sa = WA.scales + rowA0 * G.sca_g + (size_t)kc * G.sca;
+    const uint8_t* sb = WB.scales + rowB0 * G.scb_g + (size_t)kc * G.scb;
+    uint8_t* sd = st + G.sc_off;
+    const int pa = G.sca / G.sc_vec, pb = G.scb / G.sc_vec;  // pieces per row
+    for (int idx = lane; idx < 8 * (pa + pb); idx += 32) {
+      const bool isb = idx >= 8 * pa;
+      const int k2 = isb ? idx - 8 * pa : idx;
+      const int pr = isb ? pb : pa;
+      const int row = k2 / pr, pc = k2 - row * pr;
+      const uint8_t* src = isb ? sb + (size_t)row * G.scb_g + pc * G.sc_vec
+                               : sa + (size_t)row * G.sca_g + pc * G.sc_vec;
+      uint8_t* dst = sd + (isb ? 8 * G.sca + row * G.scb : row * G.sca) + pc * G.sc_vec;
+      if (G.sc_vec == 16) cp_async16(dst, src, pol);
+      else cp_async4(dst, src);
+    }
+  };
+
+  int64_t done = 0;  // chunks consumed by this warp (ring position)
+  bool bad = false;
+  bool waited_pdl = false;
+  StageRegs SR;
+  int64_t c = c0;
+  while (c < c1) {
+    // ---- plan a segment: consecutive virtual experts whose rows fit xcap
+    if (threadIdx.x == 0) {
+      const int v0 = (int)(c / nk / RT);
+      const int vlast = (int)((c1 - 1) / nk / RT);
+      int rows = 0, v = v0;
+      for (; v <= vlast; ++v) {
+        const int n = S.R.v_n[v];
+        int add = 0;
+        bool fits = true;
+        int8_t cr[kTileN];
+        for (int j = 0; j < n && fits; ++j) {
+          const int pr = S.R.pair_list[S.R.v_p0[v] + j];
+          const int key = GATEUP ? pr / a.k : pr;
+          int found = -1;
+          for (int i = 0; i < rows + add; ++i)
+            if (S.row_key[i] == key) found = i;
+          if (found < 0) {
+            if (rows + add >= G.xcap) {
+              fits = false;
+            } else {
+              S.row_key[rows + add] = (int16_t)key;
+              found = rows + add;
+              ++add;
+            }
+          }
+          cr[j] = (int8_t)found;
+        }
+        if (!fits) break;  // v starts the next segment
+        for (int j = 0; j < n; ++j) S.col_row[(v - v0) * kTileN + j] = cr[j];
+        rows += add;
+      }
+      S.seg_v0 = v0;
+      S.seg_v1 = v;  // exclusive; v > v0 always (one virtual expert has <= xcap rows)
+      S.seg_rows = rows;
+    }
+    __syncthreads();
+    const int seg_v0 = S.seg_v0, seg_v1 = S.seg_v1, seg_rows = S.seg_rows;
+    if (seg_v1 <= seg_v0) {  // cannot happen; never loop forever
+      set_status(QK_ERR_INVALID_ARG);
+      break;
+    }
+    const int64_t s_end = min(c1, (int64_t)seg_v1 * RT * nk);
+    const int64_t n_seg = s_end - c;
+    const int64_t w0 = c + n_seg * warp / kDW, w1 = c + n_seg * (warp + 1) / kDW;
+    const int64_t wn = w1 - w0;
+
+    // ---- activation loads first, then the weight prefetch (D-1 chunks), then staging
+    if (GATEUP) stage_issue<true>(a, S, SR, seg_rows);
+    for (int i = 0; i < G.D - 1; ++i) {
+      if (i < wn) issue(w0 + i, (int)((done + i) % G.D));
+      cp_async_commit();
+    }
+    if (!GATEUP) {
+      if (!waited_pdl) {
+        pdl_wait();  // h and hmax come from k_gateup
+        waited_pdl = true;
+      }
+      stage_issue<false>(a, S, SR, seg_rows);
+    }
+    stage_finish<GATEUP>(a, S, SR, act, G.act_stride, seg_rows);
+    __syncthreads();
+
+    // ---- stream this warp's chunks
+    int64_t cur_u = -1;
+    int kc_start = 0, kc_last = 0;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    auto emit = [&]() {
+      const int v = (int)(cur_u / RT), r = (int)(cur_u - (int64_t)v * RT);
+      const int e = S.R.v_expert[v], n = S.R.v_n[v];
+      const float s2a = WA.fmt == QK_FMT_NVFP4 ? WA.scale_2[e] : 1.f;
+      const float s2b = WB.fmt == QK_FMT_NVFP4 ? WB.scale_2[e] : 1.f;
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int col = 2 * t + jj;
+        const float sx = col < n ? pow2f(S.shift[S.col_row[(v - seg_v0) * kTileN + col]]) : 0.f;
+        acc[jj] *= sx * s2a;
+        acc[2 + jj] *= sx * s2b;
+      }
+      const int len = kc_last + 1 - kc_start;
+      float4 fin = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      bool ready = GATEUP && kc_start == 0 && len == nk;
+      if (!ready) {
+        // publish this piece; the last contributor finishes the unit (k_gateup)
+        // or the whole row tile (k_down)
+        const int64_t slot = cur_u * nk + kc_start;
+        float4* part = reinterpret_cast<float4*>(GATEUP ? a.part1 : a.part2);
+        part[slot * 32 + lane] = fin;
+        if (lane == 0) (GATEUP ? a.len1 : a.len2)[slot] = (uint8_t)len;
+        __syncwarp();
+        uint32_t last = 0;
+        if (lane == 0) {
+          const uint32_t need = GATEUP ? (uint32_t)nk : (uint32_t)(S.R.n_v * nk);
+          uint32_t* cnt = GATEUP ? a.cnt1 + cur_u : a.cnt2 + r;
+          last = (atom_add_acq_rel(cnt, (uint32_t)len) + (uint32_t)len == need) ? 1u : 0u;
+        }
+        ready = __shfl_sync(0xffffffffu, last, 0) != 0;
+        if (ready) {
+          __threadfence();
+          if (GATEUP) {  // sum the unit's pieces in chunk order
+            fin = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int kc = 0; kc < nk;) {
+              const int64_t sl = cur_u * nk + kc;
+              const float4 f = __ldcg(part + sl * 32 + lane);
+              fin.x += f.x; fin.y += f.y; fin.z += f.z; fin.w += f.w;
+              kc += __ldcg(a.len1 + sl);
+            }
+          }
+        }
+      }
+      if (!ready) return;
+      if (GATEUP) {
+        const float fv[4] = {fin.x, fin.y, fin.z, fin.w};
         float hm[2];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int col = 2 * t + j;
-          hm[j] = 0.f;
-          if (col < nt) {
-            const float sx = pow2f(S.shift[col]);
-            const float gv = acc[j] * sx * s2g, uv = acc[2 + j] * sx * s2u;
-            const float hv = silu_mul(gv, uv);
-            const int p = S.R.pair_list[p0 + tile * tn + col];
+        for (int jj = 0; jj < 2; ++jj) {
+          const int col = 2 * t + jj;
+          hm[jj] = 0.f;
+          if (col < n) {
+            const float hv = silu_mul(fv[jj], fv[2 + jj]);
+            const int p = S.R.pair_list[S.R.v_p0[v] + col];
             a.h[(size_t)p * a.I + r * 8 + g] = hv;
-            hm[j] = fabsf(hv);
+            hm[jj] = fabsf(hv);
           }
         }
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
+        for (int jj = 0; jj < 2; ++jj)
 #pragma unroll
-          for (int o = 4; o < 32; o <<= 1) hm[j] = fmaxf(hm[j], __shfl_xor_sync(0xffffffffu, hm[j], o));
-        }
+          for (int o = 4; o < 32; o <<= 1)
+            hm[jj] = fmaxf(hm[jj], __shfl_xor_sync(0xffffffffu, hm[jj], o));
         if (g == 0) {
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int col = 2 * t + j;
-            if (col < nt) a.hmax[(size_t)S.R.pair_list[p0 + tile * tn + col] * R1 + r] = hm[j];
+          for (int jj = 0; jj < 2; ++jj) {
+            const int col = 2 * t + jj;
+            if (col < n) a.hmax[(size_t)S.R.pair_list[S.R.v_p0[v] + col] * (a.I / 8) + r] = hm[jj];
           }
         }
-      }
-      __syncthreads();
-    }
-    if (threadIdx.x == 0 && i + nstage < n) issue(i + nstage);
-  }
-  if (bad) set_status(QK_ERR_NAN_SCALE);
-}
-
-// =================================================================== k2 ==
-template <int FD>
-__global__ void __launch_bounds__(kThreads, 1) k_down(const DecodeArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  SmemHead& S = *reinterpret_cast<SmemHead*>(smem);
-  const Geo G = make_geo(a.I, FD, FD);
-  __half* act = reinterpret_cast<__half*>(smem + kHeadBytes);
-  uint8_t* stages = smem + kHeadBytes + (size_t)a.rows_act * G.act_stride * 2;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nstage = a.stages;
-  const int tn = a.rows_act;  // token columns per tile = staged activation rows (<= 8)
-
-  build_route(a.ids, a.P, a.E, S.R);
-  const int R1 = a.I / 8, R2 = a.H / 16;
-  const int U = S.R.n_active * R2;
-  const int u0 = (int)((int64_t)U * blockIdx.x / gridDim.x);
-  const int u1 = (int)((int64_t)U * (blockIdx.x + 1) / gridDim.x);
-  const int n = u1 - u0;
-  if (n <= 0) {
-    pdl_wait();
-    return;
-  }
-  const uint64_t pol = policy_evict_first();
-  auto issue = [&](int i) {
-    const int u = u0 + i, s = i % nstage;
-    const int e = S.R.act_expert[u / R2];
-    const int64_t row0 = (int64_t)e * a.H + (int64_t)(u % R2) * 16;
-    issue_unit(stages + (size_t)s * G.stage, &S.full[s], G, a.down.q, a.down.scales, row0, a.down.q,
-               a.down.scales, row0 + 8, pol);
-  };
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < nstage; ++s) mbar_init(&S.full[s], 1);
-    fence_mbar_init();
-    for (int i = 0; i < min(n, nstage); ++i) issue(i);  // weights do not depend on k_gateup
-  }
-  __syncthreads();
-  pdl_wait();  // h, hmax and the counters are written by k_gateup
-
-  bool bad = false;
-  int cur_a = -1;
-  const unsigned long long limit = g_wait_limit_ns;
-  for (int i = 0; i < n; ++i) {
-    const int u = u0 + i, s = i % nstage;
-    const int as = u / R2, r = u % R2;
-    const int e = S.R.act_expert[as];
-    const int p0 = S.R.act_off[as], np = S.R.act_off[as + 1] - p0;
-    const uint8_t* st = stages + (size_t)s * G.stage;
-    const bool ready = mbar_wait_bounded(&S.full[s], (i / nstage) & 1, limit);
-    if (__syncthreads_or(!ready)) {
-      drain_stages(S.full, i, min(n, i + nstage), nstage);
-      return;
-    }
-    for (int tile = 0; tile * tn < np; ++tile) {
-      const int nt = min(tn, np - tile * tn);
-      if (as != cur_a || np > tn) {
-        // pair rows and their absmax over all of h (from k_gateup's per-tile maxima)
-        float v[kTileN];
-#pragma unroll
-        for (int j = 0; j < kTileN; ++j) {
-          v[j] = 0.f;
-          if (j < nt) {
-            const int p = S.R.pair_list[p0 + tile * tn + j];
-            for (int q = threadIdx.x; q < R1; q += blockDim.x) v[j] = fmaxf(v[j], __ldcg(a.hmax + (size_t)p * R1 + q));
+      } else {
+        // every piece of row tile r is in: y[t][r*16+m] = sum_s w * sum_pieces
+        const float* part = a.part2;
+        for (int idx = lane; idx < a.T * 16; idx += 32) {
+          const int tok = idx >> 4, m = idx & 15;
+          const int ln = (m & 7) * 4, el = (m >= 8) ? 2 : 0;
+          float yv = 0.f;
+          for (int sl = 0; sl < a.k; ++sl) {
+            const int p = tok * a.k + sl;
+            const int pv = S.R.pair_v[p];
+            if (pv < 0) continue;
+            const int j = S.R.pair_j[p];
+            const int64_t uu = (int64_t)pv * RT + r;
+            float d = 0.f;
+            for (int kc = 0; kc < nk;) {
+              const int64_t sl2 = uu * nk + kc;
+              d += __ldcg(part + (sl2 * 32 + ln + (j >> 1)) * 4 + el + (j & 1));
+              kc += __ldcg(a.len2 + sl2);
+            }
+            yv = fmaf(a.w[p], d, yv);
           }
-        }
-        if (threadIdx.x < kTileN)
-          S.rows[threadIdx.x] = threadIdx.x < nt ? S.R.pair_list[p0 + tile * tn + threadIdx.x] : 0;
-        block_max8(v, S.mx_red, S.mx_out);
-        stage_f32_rows(a.h, S.rows, nt, a.I, S.mx_out, act, G.act_stride, S.shift);
-        cur_a = as;
-      }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      unit_mma<FD, FD>(acc, st, G, act, a.rows_act, warp, lane, bad);
-      if (reduce_warps(acc, S.red, warp, lane)) {
-        const int g = lane >> 2, t = lane & 3;
-        const float s2 = FD == QK_FMT_NVFP4 ? a.down.scale_2[e] : 1.f;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int col = 2 * t + j;
-          if (col < nt) {
-            const float sh = pow2f(S.shift[col]) * s2;
-            const int p = S.rows[col];
-            float* pr = a.part + (size_t)p * a.H + r * 16;
-            pr[g] = acc[j] * sh;
-            pr[g + 8] = acc[2 + j] * sh;
-          }
+          const size_t o = (size_t)tok * a.H + r * 16 + m;
+          if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(yv);
+          else reinterpret_cast<float*>(a.y)[o] = yv;
         }
       }
-      __syncthreads();
+    };
+
+    for (int64_t i = 0; i < wn; ++i) {
+      // keep D-1 chunks in flight: issue chunk i+D-1, then wait for chunk i
+      if (i + G.D - 1 < wn) issue(w0 + i + G.D - 1, (int)((done + G.D - 1) % G.D));
+      cp_async_commit();
+      cp_async_wait_dyn(G.D - 1);
+      __syncwarp();
+      const int slot = (int)(done % G.D);
+      const int64_t cc = w0 + i;
+      const int64_t u = cc / nk;
+      const int kc = (int)(cc - u * nk);
+      if (u != cur_u) {
+        if (cur_u >= 0) emit();
+        cur_u = u;
+        kc_start = kc;
+        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+      }
+      kc_last = kc;
+      const int v = (int)(u / RT);
+      const int n = S.R.v_n[v];
+      const int row = S.col_row[(v - seg_v0) * kTileN + (g < n ? g : 0)];
+      const __half* xrow = act + (size_t)row * G.act_stride + 8 * t + (size_t)kc * G.Kc;
+      chunk_mma<FA, FB>(acc, ring + (size_t)slot * G.stage, G, xrow, lane, bad);
+      ++done;
+      __syncwarp();  // every lane is done with this stage before it is refilled
     }
-    // last expert to finish row tile r combines it, in slot order
-    __threadfence();
+    if (cur_u >= 0) emit();
+    cp_async_wait<0>();
     __syncthreads();
-    if (threadIdx.x == 0) S.flag = (atomicAdd(&a.counters[r], 1) == S.R.n_active - 1);
-    __syncthreads();
-    if (S.flag) {
-      __threadfence();
-      for (int idx = threadIdx.x; idx < a.T * 16; idx += blockDim.x) {
-        const int tok = idx >> 4, m = r * 16 + (idx & 15);
-        float yv = 0.f;
-        for (int sl = 0; sl < a.k; ++sl) {
-          const int p = tok * a.k + sl;
-          const int ep = a.ids[p];
-          if (ep < 0 || ep >= a.E) continue;
-          yv = fmaf(a.w[p], __ldcg(a.part + (size_t)p * a.H + m), yv);
-        }
-        if (a.y_bf16)
-          reinterpret_cast<__nv_bfloat16*>(a.y)[(size_t)tok * a.H + m] = __float2bfloat16_rn(yv);
-        else
-          reinterpret_cast<float*>(a.y)[(size_t)tok * a.H + m] = yv;
-      }
-    }
-    if (threadIdx.x == 0 && i + nstage < n) issue(i + nstage);
+    c = s_end;
   }
   if (bad) set_status(QK_ERR_NAN_SCALE);
 }
 
 // ================================================================= host ==
-// Deepest ring (2..kMaxStages) that fits `budget` bytes of shared memory.
-static int plan_stages(const Geo& G, int rows_act, size_t budget, size_t& smem) {
-  const size_t fixed = kHeadBytes + (size_t)rows_act * G.act_stride * 2;
-  const size_t cap = std::min(budget, (size_t)max_smem_optin());
-  int s = kMaxStages;
-  while (s > 2 && fixed + (size_t)s * G.stage > cap) --s;
-  smem = fixed + (size_t)s * G.stage;
-  return (smem <= (size_t)max_smem_optin()) ? s : 0;
+// Largest chunk (<= 1024, dividing K, >= 128) whose rings of at least 3 stages
+// per warp fit in shared memory (else 2 stages), ring depth up to kMaxD.
+static DGeo plan_geo(int K, int fa, int fb, int xcap) {
+  const int cap = max_smem_optin();
+  DGeo two = make_dgeo(K, 128, fa, fb, xcap, 2);
+  two.smem = 0;
+  for (int Kc = 1024; Kc >= 128; Kc >>= 1) {
+    if (K % Kc) continue;
+    for (int D = kMaxD; D >= 2; --D) {
+      const DGeo g = make_dgeo(K, Kc, fa, fb, xcap, D);
+      if (g.smem > cap) continue;
+      if (D >= 3) return g;
+      if (!two.smem) two = g;
+      break;
+    }
+  }
+  return two;
 }
 
-// Budgets chosen so one k_gateup CTA and one k_down CTA fit on an SM together
-// (228 KB): the dependent down kernel starts streaming its weights while the
-// gate/up kernel drains.
-constexpr size_t kBudgetGateUp = 132 * 1024;
-constexpr size_t kBudgetDown = 92 * 1024;
-
-template <int FG, int FU>
-static qk_status launch_gateup(DecodeArgs& args, int grid, cudaStream_t st) {
-  size_t smem = 0;
-  const int s = plan_stages(make_geo(args.H, FG, FU), args.rows_act, kBudgetGateUp, smem);
-  if (!s) return QK_ERR_UNSUPPORTED;
-  args.stages = s;
-  return launch_k(k_gateup<FG, FU>, smem, grid, args, st, false);
-}
-
-template <int FD>
-static qk_status launch_down(DecodeArgs& args, int grid, cudaStream_t st) {
-  size_t smem = 0;
-  const int s = plan_stages(make_geo(args.I, FD, FD), args.rows_act, kBudgetDown, smem);
-  if (!s) return QK_ERR_UNSUPPORTED;
-  args.stages = s;
-  return launch_k(k_down<FD>, smem, grid, args, st, true);
+template <int FA, int FB, bool GATEUP>
+static qk_status go(DArgs& P, cudaStream_t st, bool pdl) {
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), P.C_max));
+  auto kern = k_decode<FA, FB, GATEUP>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P.G.smem) !=
+      cudaSuccess)
+    return QK_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDW * 32);
+  cfg.dynamicSmemBytes = P.G.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, P) == cudaSuccess ? QK_OK : QK_ERR_CUDA;
 }
 
 qk_status decode_forward(DecodeArgs args, cudaStream_t st) {
-  const int sms = num_sms();
-  args.rows_act = std::min(args.T, kTileN);
-  const int amax = std::min(args.E, args.P);
-  const int grid1 = std::max(1, std::min(sms, amax * (args.I / 8)));
-  const int grid2 = std::max(1, std::min(sms, amax * (args.H / 16)));
+  // the piece counters start at zero on every call
+  if (cudaMemsetAsync(args.cnt1, 0, args.cnt_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
+  DArgs P1 = {};
+  P1.a = args;
+  P1.RT = args.I / 8;
+  P1.G = plan_geo(args.H, args.gate.fmt, args.up.fmt, std::min(args.T, kXCap));
+  if (!P1.G.smem) return QK_ERR_UNSUPPORTED;
+  P1.C_max = (int64_t)args.P * P1.RT * P1.G.nk;  // virtual experts <= pairs
+  DArgs P2 = {};
+  P2.a = args;
+  P2.RT = args.H / 16;
+  P2.G = plan_geo(args.I, args.down.fmt, args.down.fmt, std::min(args.P, kXCap));
+  if (!P2.G.smem) return QK_ERR_UNSUPPORTED;
+  P2.C_max = (int64_t)args.P * P2.RT * P2.G.nk;
+  constexpr int MX = QK_FMT_MXFP4, NV = QK_FMT_NVFP4;
   const int fg = args.gate.fmt, fu = args.up.fmt, fd = args.down.fmt;
   qk_status rc;
-  if (fg == QK_FMT_MXFP4 && fu == QK_FMT_MXFP4) rc = launch_gateup<QK_FMT_MXFP4, QK_FMT_MXFP4>(args, grid1, st);
-  else if (fg == QK_FMT_MXFP4) rc = launch_gateup<QK_FMT_MXFP4, QK_FMT_NVFP4>(args, grid1, st);
-  else if (fu == QK_FMT_MXFP4) rc = launch_gateup<QK_FMT_NVFP4, QK_FMT_MXFP4>(args, grid1, st);
-  else rc = launch_gateup<QK_FMT_NVFP4, QK_FMT_NVFP4>(args, grid1, st);
+  if (fg == MX && fu == MX) rc = go<MX, MX, true>(P1, st, false);
+  else if (fg == MX) rc = go<MX, NV, true>(P1, st, false);
+  else if (fu == MX) rc = go<NV, MX, true>(P1, st, false);
+  else rc = go<NV, NV, true>(P1, st, false);
   if (rc != QK_OK) return rc;
-  return fd == QK_FMT_MXFP4 ? launch_down<QK_FMT_MXFP4>(args, grid2, st)
-                            : launch_down<QK_FMT_NVFP4>(args, grid2, st);
+  return fd == MX ? go<MX, MX, false>(P2, st, true) : go<NV, NV, false>(P2, st, true);
 }
 
-size_t decode_workspace_bytes(int T, int k, int H, int I) {
+// Workspace: h [P][I] f32 | hmax [P][I/8] | part1 [U1*nk1][32] float4 |
+// part2 [U2*nk2][32] float4 | len1 | len2 | cnt1 [U1] | cnt2 [H/16].
+// Chunk counts are sized for the smallest chunk the planner may pick (128).
+struct WsLayout {
+  size_t h, hmax, part1, part2, len1, len2, cnt1, cnt2, total;
+};
+
+static WsLayout ws_layout(int T, int k, int H, int I) {
   const size_t P = (size_t)T * k;
-  return align256(P * I * 4) + align256(P * (I / 8) * 4) + align256(P * H * 4) +
-         align256((size_t)(H / 16) * 4);
+  const size_t nk1 = (size_t)H / 128, nk2 = (size_t)I / 128;
+  const size_t U1 = P * (I / 8), U2 = P * (H / 16);
+  WsLayout L;
+  size_t o = 0;
+  L.h = o; o += align256(P * I * 4);
+  L.hmax = o; o += align256(P * (I / 8) * 4);
+  L.part1 = o; o += align256(U1 * nk1 * 512);
+  L.part2 = o; o += align256(U2 * nk2 * 512);
+  L.len1 = o; o += align256(U1 * nk1);
+  L.len2 = o; o += align256(U2 * nk2);
+  L.cnt1 = o; o += U1 * 4;
+  L.cnt2 = o; o += (size_t)(H / 16) * 4;
+  L.total = align256(o);
+  return L;
 }
+
+size_t decode_workspace_bytes(int T, int k, int H, int I) { return ws_layout(T, k, H, I).total; }
 
 void decode_carve(DecodeArgs& a, void* ws) {
-  const size_t P = (size_t)a.P;
+  const WsLayout L = ws_layout(a.T, a.k, a.H, a.I);
   uint8_t* p = static_cast<uint8_t*>(ws);
-  a.h = reinterpret_cast<float*>(p);
-  p += align256(P * a.I * 4);
-  a.hmax = reinterpret_cast<float*>(p);
-  p += align256(P * (a.I / 8) * 4);
-  a.part = reinterpret_cast<float*>(p);
-  p += align256(P * a.H * 4);
-  a.counters = reinterpret_cast<int*>(p);
-  a.n_counters = a.H / 16;
+  a.h = reinterpret_cast<float*>(p + L.h);
+  a.hmax = reinterpret_cast<float*>(p + L.hmax);
+  a.part1 = reinterpret_cast<float*>(p + L.part1);
+  a.part2 = reinterpret_cast<float*>(p + L.part2);
+  a.len1 = p + L.len1;
+  a.len2 = p + L.len2;
+  a.cnt1 = reinterpret_cast<uint32_t*>(p + L.cnt1);
+  a.cnt2 = reinterpret_cast<uint32_t*>(p + L.cnt2);
+  a.cnt_bytes = L.total - L.cnt1;
 }
 
 }  // namespace qk

@@ -23,14 +23,16 @@ struct DecodeArgs {
   void* y;
   int T, k, E, H, I, P;
   int y_bf16;
-  int stages;
-  int rows_act;       // activation rows staged per tile (<= 8)
   // workspace
-  float* h;           // [P][I] fp32
-  float* hmax;        // [P][I/8] per-tile absmax of h
-  float* part;        // [P][H] fp32 per-pair expert outputs
-  int* counters;      // [H/16]
-  int n_counters;
+  float* h;           // [P][I] fp32 SwiGLU output
+  float* hmax;        // [P][I/8] absmax of h per 8-row tile
+  float* part1;       // k_gateup pieces of split units
+  float* part2;       // k_down pieces (every unit)
+  uint8_t* len1;      // chunks per piece
+  uint8_t* len2;
+  uint32_t* cnt1;     // chunks finished per k_gateup unit
+  uint32_t* cnt2;     // chunks finished per k_down row tile (follows cnt1)
+  size_t cnt_bytes;   // bytes zeroed from cnt1 on every call
 };
 
 qk_status decode_forward(DecodeArgs args, cudaStream_t st);

@@ -27,8 +27,10 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route(const float* __restr
   float* v = srow + (size_t)warp * E;
   for (int i = lane; i < E; i += 32) v[i] = logits[(size_t)t * E + i];
   __syncwarp();
-  float sel_v[32];
-  int sel_i[32];
+  // lane s keeps slot s (top_k <= 32): no local-memory arrays
+  float my_v = -INFINITY;
+  int my_i = 0;
+  float lmax = -INFINITY;
   for (int s = 0; s < k; ++s) {
     float bv = -INFINITY;
     int bi = 0x7fffffff;
@@ -52,20 +54,22 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route(const float* __restr
     if (bi >= E) bi = 0;
     if (lane == 0) v[bi] = NAN;
     __syncwarp();
-    sel_v[s] = bv;
-    sel_i[s] = bi;
+    if (s == 0) lmax = bv;
+    if (lane == s) {
+      my_v = bv;
+      my_i = bi;
+    }
   }
-  const float lmax = sel_v[0];
   if (!(lmax > -INFINITY) || !isfinite(lmax)) {
     if (lane == 0) set_status(QK_ERR_INVALID_ARG);
   }
-  float z = 0.f;
-  for (int s = 0; s < k; ++s) z += expf(sel_v[s] - lmax);
-  if (lane == 0) {
-    for (int s = 0; s < k; ++s) {
-      ids[(size_t)t * k + s] = sel_i[s];
-      w[(size_t)t * k + s] = expf(sel_v[s] - lmax) / z;
-    }
+  const float ex = lane < k ? expf(my_v - lmax) : 0.f;
+  float z = ex;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  if (lane < k) {
+    ids[(size_t)t * k + lane] = my_i;
+    w[(size_t)t * k + lane] = ex / z;
   }
 }
 

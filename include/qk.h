@@ -92,7 +92,7 @@ typedef struct qk_moe_layer {
  *  x_bf16    [T][hidden] bf16.        topk_ids [T][top_k] int32 in [0, E).
  *  topk_w    [T][top_k] fp32.         y        [T][hidden] fp32 (y_is_bf16=0) or bf16.
  *  act_quant QK_ACT_NONE.             workspace >= moe_expert_workspace_size(), 256-B aligned.
- * Shapes: hidden and inter multiples of 64; 1 <= top_k <= 8.  Token counts
+ * Shapes: hidden and inter multiples of 128; 1 <= top_k <= 8.  Token counts
  * 1..16 run the decode path (CUDA-core decode of nibbles and scales in
  * registers, tensor-core m16n8k16 products, fp32 accumulation); larger counts
  * run the grouped path.  T = 0 returns QK_OK and launches nothing.

@@ -49,7 +49,7 @@ def test_workspace_query_and_shape_validation():
     n16 = L.moe_expert_workspace_size(ctypes.byref(lay), 16, 6)
     assert 0 < n1 < n16
     assert L.moe_expert_workspace_size(ctypes.byref(lay), 1, 9) == 0        # top_k > 8
-    assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(H=4032 + 16)), 1, 6) == 0
+    assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(H=4096 + 64)), 1, 6) == 0
     assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(fmts=(1, 3, 1))), 1, 6) == 0
     bad = _fake_layer()
     bad.down.rows = 2048
