@@ -22,20 +22,27 @@
 // a given grid).
 //
 // Data path.  Each warp streams its chunks through its own ring of shared-
-// memory stages with cp.async (16 bytes per lane, one instruction per 512-byte
-// packed row, asynchronous issue), rows padded by 16 bytes so ldmatrix reads
-// them without bank conflicts.  A thread forms m16n8k16 A fragments with
-// ldmatrix and the hardware e2m1x2 -> f16x2 conversion (exact) and multiplies
-// on the tensor cores with f16 activations (fp32 accumulate):
+// memory stages.  Packed rows arrive by tensor-map TMA as 3-D boxes of 8 or 16
+// rows x Kc/2 bytes in the 128-byte-swizzled layout (16-byte chunk c of row r
+// stored at c ^ (r & 7)), so ldmatrix reads them without bank conflicts; the
+// matching scale-row slices arrive by cp.async; both complete on the stage's
+// mbarrier.  (Shapes whose rows or scale slices are not 256 / 16-byte
+// multiples fall back to one cp.async per 16 bytes into padded rows.)  A
+// thread forms m16n8k16 A fragments with ldmatrix and the hardware
+// e2m1x2 -> f16x2 conversion (exact) and multiplies on the tensor cores with
+// f16 activations (fp32 accumulate):
 //   MXFP4: the fp32 partial of each 32-block is scaled by 2^(c-127) (exact);
 //   NVFP4: the e4m3 scale is folded into the f16 fragment (e2m1 * e4m3 is exact
 //          in f16) and scale_2 is applied at the end.
 // Activations are staged once per CTA segment as f16 rows scaled by a power of
 // two per row, chosen so the row's largest magnitude sits in [2^14, 2^15); their
 // loads are issued ahead of the weight stream.
+#include <cuda.h>
+
 #include <algorithm>
 
 #include "qk_common.cuh"
+#include "qk_tmap.h"
 
 namespace qk {
 
@@ -168,22 +175,25 @@ __device__ void build_route(const int32_t* __restrict__ ids, int P, int E, Route
 }
 
 // ------------------------------------------------------------- geometry --
-// Shared by host and device: one warp's stage holds a chunk's 16 packed rows
-// (stride Kc/2 + 16 bytes) followed by its 16 scale-row slices.
+// Shared by host and device.  Per warp: D nibble stages (1024-byte aligned)
+// and D scale stages; then the staged activation rows.
 struct DGeo {
   int K, Kc;        // reduction length, chunk length
   int nk;           // chunks per unit
   int nbc;          // 32-blocks per chunk
-  int nib;          // padded bytes per packed smem row (Kc/2 + 16)
-  int sc_off;       // offset of the scale rows in a stage
+  int tmap;         // 1: packed rows by tensor-map TMA (swizzled), 0: cp.async rows
+  int nseg;         // 128-byte segments per packed chunk row
+  int nib;          // padded bytes per packed smem row (row mode)
+  int nib_stage;    // bytes of one stage's packed rows (1024-multiple)
   int sca, scb;     // scale bytes per chunk row, rows 0..7 / 8..15
   int sca_g, scb_g; // scale bytes per global row (full K)
   int sc_vec;       // bytes per scale cp.async (16 or 4)
-  int stage;        // bytes per stage (128-multiple)
+  int sc_stage;     // bytes of one stage's scale rows (16-multiple)
   int act_stride;   // halves per staged activation row
   int xcap;         // staged activation rows
   int D;            // stages per warp
-  int smem;         // total dynamic shared memory
+  int off_rings, off_scales, off_act;  // from the 1024-aligned base
+  int smem;         // total dynamic shared memory (with alignment slack)
 };
 
 __host__ __device__ inline int sc_row_bytes(int fmt, int K) {
@@ -196,28 +206,37 @@ struct DHead {
   int16_t row_key[kXCap];               // staged row -> token (k_gateup) or pair (k_down)
   int8_t col_row[kMaxPairs * kTileN];   // (v - seg_v0, column) -> staged row
   int shift[kXCap];
+  int dead;                             // a warp's copies did not land in time
   float red8[kDW][kXCap];
+  alignas(8) uint64_t full[kDW][kMaxD];
 };
 constexpr int kDHead = (int)((sizeof(DHead) + 127) / 128 * 128);
 
-__host__ __device__ inline DGeo make_dgeo(int K, int Kc, int fa, int fb, int xcap, int D) {
+__host__ __device__ inline int up_to(int x, int a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline DGeo make_dgeo(int K, int Kc, int fa, int fb, int xcap, int D, bool tmap_ok) {
   DGeo g;
   g.K = K;
   g.Kc = Kc;
   g.nk = K / Kc;
   g.nbc = Kc / 32;
-  g.nib = Kc / 2 + 16;
   g.sca_g = sc_row_bytes(fa, K);
   g.scb_g = sc_row_bytes(fb, K);
   g.sca = sc_row_bytes(fa, Kc);
   g.scb = sc_row_bytes(fb, Kc);
   g.sc_vec = (g.sca % 16 || g.scb % 16 || g.sca_g % 16 || g.scb_g % 16) ? 4 : 16;
-  g.sc_off = 16 * g.nib;
-  g.stage = (g.sc_off + 8 * g.sca + 8 * g.scb + 127) / 128 * 128;
+  g.tmap = (tmap_ok && K % 256 == 0 && Kc % 256 == 0) ? 1 : 0;
+  g.nseg = Kc / 256;
+  g.nib = Kc / 2 + 16;
+  g.nib_stage = g.tmap ? 16 * (Kc / 2) : up_to(16 * g.nib, 1024);
+  g.sc_stage = up_to(8 * g.sca + 8 * g.scb, 16);
   g.act_stride = K + 32;  // 2K+64 bytes: conflict-free 16-byte fragment loads
   g.xcap = xcap;
   g.D = D;
-  g.smem = kDHead + xcap * g.act_stride * 2 + kDW * D * g.stage;
+  g.off_rings = up_to(kDHead, 1024);
+  g.off_scales = g.off_rings + kDW * D * g.nib_stage;
+  g.off_act = up_to(g.off_scales + kDW * D * g.sc_stage, 16);
+  g.smem = g.off_act + xcap * g.act_stride * 2 + 1024;  // + slack to align the base
   return g;
 }
 
@@ -226,6 +245,7 @@ struct DArgs {
   DGeo G;
   int RT;          // units (row tiles) per virtual expert
   int64_t C_max;   // upper bound of chunks (grid sizing only)
+  alignas(64) CUtensorMap tqa, tqb;  // packed rows of the A / B projections (tensor-map mode)
 };
 
 // ---------------------------------------------------------- fragments --
@@ -328,23 +348,28 @@ __device__ __forceinline__ void block_mma(float (&acc)[4], uint32_t wa, uint32_t
 }
 
 // One chunk of one unit (warp): 16 rows x Kc against one token tile.
-// st: the stage (packed rows, then scale rows); xrow: this thread's activation
-// row at the chunk's first block.
-template <int FA, int FB>
-__device__ __forceinline__ void chunk_mma(float (&acc)[4], const uint8_t* st, const DGeo& G,
-                                          const __half* xrow, int lane, bool& bad) {
+// st: the stage's packed rows; sc: its scale rows; xrow: this thread's
+// activation row at the chunk's first block.
+template <int FA, int FB, bool GATEUP>
+__device__ __forceinline__ void chunk_mma(float (&acc)[4], const uint8_t* st, const uint8_t* sc,
+                                          const DGeo& G, const __half* xrow, int lane, bool& bad) {
   const int g = lane >> 2, t = lane & 3;
   const int mj = lane >> 3, mr = lane & 7;
-  // ldmatrix row address: matrix mj (0: rows 0-7 blk b, 1: rows 8-15 blk b,
-  // 2: rows 0-7 blk b+1, 3: rows 8-15 blk b+1), row mr
-  const uint8_t* lrow = st + ((mj & 1) * 8 + mr) * G.nib + (mj >> 1) * 16;
-  const uint8_t* sa = st + G.sc_off + g * G.sca;
-  const uint8_t* sb = st + G.sc_off + 8 * G.sca + g * G.scb;
+  // ldmatrix: lane supplies row r = (mj&1)*8 + mr of block b + (mj>>1)
+  const int r = (mj & 1) * 8 + mr;
+  constexpr int RB = GATEUP ? 8 : 16;  // rows per TMA box
+  const uint8_t* lbase = G.tmap ? st + (r / RB) * (RB * 128 * G.nseg) + (r % RB) * 128
+                                : st + r * G.nib;
+  const uint8_t* sa = sc + g * G.sca;
+  const uint8_t* sb = sc + 8 * G.sca + g * G.scb;
+  auto laddr = [&](int bb) -> const uint8_t* {
+    return G.tmap ? lbase + (bb >> 3) * (RB * 128) + (((bb & 7) ^ mr) << 4) : lbase + bb * 16;
+  };
 #pragma unroll 2
   for (int b = 0; b < G.nbc; b += 4) {
     uint32_t w[8];
-    ldmatrix_x4(w[0], w[1], w[2], w[3], lrow + b * 16);
-    ldmatrix_x4(w[4], w[5], w[6], w[7], lrow + (b + 2) * 16);
+    ldmatrix_x4(w[0], w[1], w[2], w[3], laddr(b + (mj >> 1)));
+    ldmatrix_x4(w[4], w[5], w[6], w[7], laddr(b + 2 + (mj >> 1)));
     Scale4<FA> s_a;
     Scale4<FB> s_b;
     s_a.load(sa, b, t, bad);
@@ -377,18 +402,10 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint64_t 
 __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_dyn(int n) {  // n in [0, kMaxD)
-  switch (n) {
-    case 0: cp_async_wait<0>(); break;
-    case 1: cp_async_wait<1>(); break;
-    case 2: cp_async_wait<2>(); break;
-    default: cp_async_wait<3>(); break;
-  }
+// The mbarrier receives one (pre-counted) arrival once this thread's earlier
+// cp.asyncs land.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // ------------------------------------------------------------- staging --
@@ -517,50 +534,67 @@ __device__ __forceinline__ void stage_finish(const DecodeArgs& a, DHead& S, Stag
 
 // ------------------------------------------------------------ the kernel --
 // Unit u = v * RT + r; chunk c = u * nk + kc.
+// Every warp fills its own ring: its lanes cp.async the chunk's scale slices
+// (and, in row mode, its packed rows) and lane 0 issues the tensor-map copies
+// of the packed rows.  A stage's mbarrier completes on 33 arrivals (one
+// deferred arrival per lane once its cp.asyncs land, plus lane 0's
+// expect-tx arrival) and the TMA bytes.  Issuing from every warp keeps the
+// per-instruction cost of a tensor copy off the critical path.
 template <int FA, int FB, bool GATEUP>
 __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ DArgs P) {
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   DHead& S = *reinterpret_cast<DHead*>(smem);
   const DecodeArgs& a = P.a;
   const DGeo& G = P.G;
-  __half* act = reinterpret_cast<__half*>(smem + kDHead);
-  uint8_t* rings = smem + kDHead + (size_t)G.xcap * G.act_stride * 2;
+  __half* act = reinterpret_cast<__half*>(smem + G.off_act);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  uint8_t* ring = rings + (size_t)warp * G.D * G.stage;
+  uint8_t* nring = smem + G.off_rings + (size_t)warp * G.D * G.nib_stage;
+  uint8_t* sring = smem + G.off_scales + (size_t)warp * G.D * G.sc_stage;
+  uint64_t* full = S.full[warp];
   const int RT = P.RT, nk = G.nk;
   const qk_weight& WA = GATEUP ? a.gate : a.down;
   const qk_weight& WB = GATEUP ? a.up : a.down;
   const int rows_per_e = GATEUP ? a.I : a.H;  // weight rows of one expert
 
   if (GATEUP) pdl_launch_dependents();
-  build_route(a.ids, a.P, a.E, S.R);
+  if (lane == 0) {
+    for (int i = 0; i < G.D; ++i) mbar_init(&full[i], 33);
+    fence_mbar_init();
+  }
+  if (threadIdx.x == 0) S.dead = 0;
+  build_route(a.ids, a.P, a.E, S.R);  // ends with a block barrier
   const int64_t C = (int64_t)S.R.n_v * RT * nk;
   const int64_t c0 = C * blockIdx.x / gridDim.x, c1 = C * (blockIdx.x + 1) / gridDim.x;
   if (c0 >= c1) return;
 
   const uint64_t pol = policy_evict_first();
+  const unsigned long long limit = g_wait_limit_ns;
   const int vpr = G.Kc / 32;  // 16-byte vectors per packed chunk row
-  // All 32 lanes: cp.async of chunk c into stage `slot` (not committed).
+  // Chunk c into stage `slot`.
   auto issue = [&](int64_t c, int slot) {
-    uint8_t* st = ring + (size_t)slot * G.stage;
+    uint8_t* st = nring + (size_t)slot * G.nib_stage;
+    uint8_t* sd = sring + (size_t)slot * G.sc_stage;
+    uint64_t* bar = &full[slot];
     const int64_t u = c / nk;
     const int kc = (int)(c - u * nk);
     const int v = (int)(u / RT), r = (int)(u - (int64_t)v * RT);
     const int e = S.R.v_expert[v];
     const int64_t rowA0 = (int64_t)e * rows_per_e + (GATEUP ? r * 8 : r * 16);
     const int64_t rowB0 = GATEUP ? rowA0 : rowA0 + 8;
-    const uint8_t* qa = WA.q + rowA0 * (G.K / 2) + (size_t)kc * (G.Kc / 2);
-    const uint8_t* qb = WB.q + rowB0 * (G.K / 2) + (size_t)kc * (G.Kc / 2);
-#pragma unroll 4
-    for (int idx = lane; idx < 16 * vpr; idx += 32) {
-      const int row = idx / vpr, vi = idx - row * vpr;
-      const uint8_t* src = (row < 8 ? qa + (size_t)row * (G.K / 2) : qb + (size_t)(row - 8) * (G.K / 2)) + vi * 16;
-      cp_async16(st + row * G.nib + vi * 16, src, pol);
+    if (!G.tmap) {
+      const uint8_t* qa = WA.q + rowA0 * (G.K / 2) + (size_t)kc * (G.Kc / 2);
+      const uint8_t* qb = WB.q + rowB0 * (G.K / 2) + (size_t)kc * (G.Kc / 2);
+      for (int idx = lane; idx < 16 * vpr; idx += 32) {
+        const int row = idx / vpr, vi = idx - row * vpr;
+        const uint8_t* src =
+            (row < 8 ? qa + (size_t)row * (G.K / 2) : qb + (size_t)(row - 8) * (G.K / 2)) + vi * 16;
+        cp_async16(st + row * G.nib + vi * 16, src, pol);
+      }
     }
     const uint8_t* sa = WA.scales + rowA0 * G.sca_g + (size_t)kc * G.sca;
     const uint8_t* sb = WB.scales + rowB0 * G.scb_g + (size_t)kc * G.scb;
-    uint8_t* sd = st + G.sc_off;
     const int pa = G.sca / G.sc_vec, pb = G.scb / G.sc_vec;  // pieces per row
     for (int idx = lane; idx < 8 * (pa + pb); idx += 32) {
       const bool isb = idx >= 8 * pa;
@@ -573,9 +607,25 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
       if (G.sc_vec == 16) cp_async16(dst, src, pol);
       else cp_async4(dst, src);
     }
+    cp_async_arrive(bar);
+    if (lane == 0) {
+      if (G.tmap) {
+        mbar_arrive_expect_tx(bar, 16u * (uint32_t)(G.Kc / 2));
+        const int z = kc * G.nseg;
+        if (GATEUP) {
+          tma_load_3d(st, &P.tqa, 0, (int)rowA0, z, bar, pol);
+          tma_load_3d(st + 8 * (G.Kc / 2), &P.tqb, 0, (int)rowB0, z, bar, pol);
+        } else {
+          tma_load_3d(st, &P.tqa, 0, (int)rowA0, z, bar, pol);
+        }
+      } else {
+        mbar_arrive_expect_tx(bar, 0u);
+      }
+    }
   };
 
   int64_t done = 0;  // chunks consumed by this warp (ring position)
+  bool dead = false;
   bool bad = false;
   bool waited_pdl = false;
   StageRegs SR;
@@ -629,10 +679,7 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
 
     // ---- activation loads first, then the weight prefetch (D-1 chunks), then staging
     if (GATEUP) stage_issue<true>(a, S, SR, seg_rows);
-    for (int i = 0; i < G.D - 1; ++i) {
-      if (i < wn) issue(w0 + i, (int)((done + i) % G.D));
-      cp_async_commit();
-    }
+    for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (int)((done + i) % G.D));
     if (!GATEUP) {
       if (!waited_pdl) {
         pdl_wait();  // h and hmax come from k_gateup
@@ -748,10 +795,20 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     for (int64_t i = 0; i < wn; ++i) {
       // keep D-1 chunks in flight: issue chunk i+D-1, then wait for chunk i
       if (i + G.D - 1 < wn) issue(w0 + i + G.D - 1, (int)((done + G.D - 1) % G.D));
-      cp_async_commit();
-      cp_async_wait_dyn(G.D - 1);
-      __syncwarp();
       const int slot = (int)(done % G.D);
+      const bool landed = mbar_wait_bounded(&full[slot], (uint32_t)((done / G.D) & 1), limit);
+      if (__any_sync(0xffffffffu, !landed)) {
+        // the copies did not land in time: report, drain what this warp has in
+        // flight, and stop the block at the end of the segment
+        set_status(QK_ERR_TIMEOUT);
+        const int64_t inflight = (wn - i < G.D) ? wn - i : (int64_t)G.D;
+        for (int64_t q = 0; q < inflight; ++q)
+          if (!mbar_wait_bounded(&full[(done + q) % G.D], (uint32_t)(((done + q) / G.D) & 1),
+                                 kDrainLimitNs))
+            break;
+        dead = true;
+        break;
+      }
       const int64_t cc = w0 + i;
       const int64_t u = cc / nk;
       const int kc = (int)(cc - u * nk);
@@ -766,13 +823,18 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
       const int n = S.R.v_n[v];
       const int row = S.col_row[(v - seg_v0) * kTileN + (g < n ? g : 0)];
       const __half* xrow = act + (size_t)row * G.act_stride + 8 * t + (size_t)kc * G.Kc;
-      chunk_mma<FA, FB>(acc, ring + (size_t)slot * G.stage, G, xrow, lane, bad);
+      chunk_mma<FA, FB, GATEUP>(acc, nring + (size_t)slot * G.nib_stage, sring + (size_t)slot * G.sc_stage,
+                                G, xrow, lane, bad);
       ++done;
       __syncwarp();  // every lane is done with this stage before it is refilled
     }
-    if (cur_u >= 0) emit();
-    cp_async_wait<0>();
+    if (dead) {
+      if (lane == 0) S.dead = 1;
+    } else if (cur_u >= 0) {
+      emit();
+    }
     __syncthreads();
+    if (S.dead) break;
     c = s_end;
   }
   if (bad) set_status(QK_ERR_NAN_SCALE);
@@ -781,14 +843,14 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
 // ================================================================= host ==
 // Largest chunk (<= 1024, dividing K, >= 128) whose rings of at least 3 stages
 // per warp fit in shared memory (else 2 stages), ring depth up to kMaxD.
-static DGeo plan_geo(int K, int fa, int fb, int xcap) {
+static DGeo plan_geo(int K, int fa, int fb, int xcap, bool tmap_ok) {
   const int cap = max_smem_optin();
-  DGeo two = make_dgeo(K, 128, fa, fb, xcap, 2);
+  DGeo two = make_dgeo(K, 128, fa, fb, xcap, 2, tmap_ok);
   two.smem = 0;
   for (int Kc = 1024; Kc >= 128; Kc >>= 1) {
     if (K % Kc) continue;
     for (int D = kMaxD; D >= 2; --D) {
-      const DGeo g = make_dgeo(K, Kc, fa, fb, xcap, D);
+      const DGeo g = make_dgeo(K, Kc, fa, fb, xcap, D, tmap_ok);
       if (g.smem > cap) continue;
       if (D >= 3) return g;
       if (!two.smem) two = g;
@@ -796,6 +858,17 @@ static DGeo plan_geo(int K, int fa, int fb, int xcap) {
     }
   }
   return two;
+}
+
+// Packed rows [rows][K/2] bytes as a 3-D map of 4-byte words:
+// {32 words of a 128-byte segment, row, segment}, boxes of `box_rows` rows x
+// `nseg` segments, 128-byte swizzle.
+static bool encode_rows(CUtensorMap* m, const uint8_t* q, int64_t rows, int K, int box_rows, int nseg) {
+  const uint64_t dims[3] = {32, (uint64_t)rows, (uint64_t)(K / 256)};
+  const uint64_t strides[2] = {(uint64_t)K / 2, 128};
+  const uint32_t box[3] = {32, (uint32_t)box_rows, (uint32_t)nseg};
+  return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, q, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <int FA, int FB, bool GATEUP>
@@ -824,13 +897,25 @@ qk_status decode_forward(DecodeArgs args, cudaStream_t st) {
   DArgs P1 = {};
   P1.a = args;
   P1.RT = args.I / 8;
-  P1.G = plan_geo(args.H, args.gate.fmt, args.up.fmt, std::min(args.T, kXCap));
+  const int x1 = std::min(args.T, kXCap);
+  P1.G = plan_geo(args.H, args.gate.fmt, args.up.fmt, x1, true);
+  if (P1.G.tmap) {
+    const int64_t rows = (int64_t)args.E * args.I;
+    if (!encode_rows(&P1.tqa, args.gate.q, rows, args.H, 8, P1.G.nseg) ||
+        !encode_rows(&P1.tqb, args.up.q, rows, args.H, 8, P1.G.nseg))
+      P1.G = plan_geo(args.H, args.gate.fmt, args.up.fmt, x1, false);
+  }
   if (!P1.G.smem) return QK_ERR_UNSUPPORTED;
   P1.C_max = (int64_t)args.P * P1.RT * P1.G.nk;  // virtual experts <= pairs
   DArgs P2 = {};
   P2.a = args;
   P2.RT = args.H / 16;
-  P2.G = plan_geo(args.I, args.down.fmt, args.down.fmt, std::min(args.P, kXCap));
+  const int x2 = std::min(args.P, kXCap);
+  P2.G = plan_geo(args.I, args.down.fmt, args.down.fmt, x2, true);
+  if (P2.G.tmap) {
+    if (!encode_rows(&P2.tqa, args.down.q, (int64_t)args.E * args.H, args.I, 16, P2.G.nseg))
+      P2.G = plan_geo(args.I, args.down.fmt, args.down.fmt, x2, false);
+  }
   if (!P2.G.smem) return QK_ERR_UNSUPPORTED;
   P2.C_max = (int64_t)args.P * P2.RT * P2.G.nk;
   constexpr int MX = QK_FMT_MXFP4, NV = QK_FMT_NVFP4;
