@@ -14,12 +14,14 @@
 // of its routed pairs (one m16n8k16 N-tile); experts with more pairs become
 // several virtual experts.  A unit is one 16-row MMA tile of a virtual expert
 // (k_gateup: 8 gate rows + the same 8 up rows; k_down: 16 down rows) over the
-// full reduction length, cut into chunks of Kc.  All chunks of the call are
-// split evenly and contiguously over the CTAs, and each CTA's range evenly over
-// its warps, so every warp streams about the same number of bytes.  A unit cut
-// by a range boundary is finished by the last of its owners (a per-unit
-// counter; partial sums added in chunk order, so results are deterministic for
-// a given grid).
+// full reduction length, cut into chunks of Kc.  The units of the call are
+// split evenly over the CTAs (whole units), and each CTA's chunks evenly and
+// contiguously over its warps, so every warp streams about the same number of
+// bytes.  A unit cut by a warp boundary is summed in shared memory by the warp
+// holding its first chunk, adding the pieces in chunk order (deterministic for
+// a given grid).  k_down writes each unit's 16 x 8 result; the last unit of a
+// row tile to finish (a per-row-tile counter) forms y for those 16 rows in
+// fixed slot order.
 //
 // Data path.  Each warp streams its chunks through its own ring of shared-
 // memory stages.  Packed rows arrive by tensor-map TMA as 3-D boxes of 8 or 16
@@ -191,6 +193,7 @@ struct DGeo {
   int sc_stage;     // bytes of one stage's scale rows (16-multiple)
   int act_stride;   // halves per staged activation row
   int xcap;         // staged activation rows
+  int fast;         // every row of the call is staged once (rows <= xcap)
   int D;            // stages per warp
   int off_rings, off_scales, off_act;  // from the 1024-aligned base
   int smem;         // total dynamic shared memory (with alignment slack)
@@ -202,12 +205,16 @@ __host__ __device__ inline int sc_row_bytes(int fmt, int K) {
 
 struct DHead {
   Route R;
-  int seg_v0, seg_v1, seg_rows;
+  int seg_u0, seg_u1, seg_v0, seg_rows;  // units [seg_u0, seg_u1) of the current segment
   int16_t row_key[kXCap];               // staged row -> token (k_gateup) or pair (k_down)
   int8_t col_row[kMaxPairs * kTileN];   // (v - seg_v0, column) -> staged row
   int shift[kXCap];
   int dead;                             // a warp's copies did not land in time
+  int pu[kDW][2];                       // unit of the warp's first / last piece (-1: none)
+  int pstart[kDW][2];                   // first chunk of that piece within its unit
+  int wempty[kDW];                      // the warp has no chunk in this segment
   float red8[kDW][kXCap];
+  float4 piece[kDW][2][32];             // partial sums of units cut by a warp boundary
   alignas(8) uint64_t full[kDW][kMaxD];
 };
 constexpr int kDHead = (int)((sizeof(DHead) + 127) / 128 * 128);
@@ -232,6 +239,7 @@ __host__ __device__ inline DGeo make_dgeo(int K, int Kc, int fa, int fb, int xca
   g.sc_stage = up_to(8 * g.sca + 8 * g.scb, 16);
   g.act_stride = K + 32;  // 2K+64 bytes: conflict-free 16-byte fragment loads
   g.xcap = xcap;
+  g.fast = 0;
   g.D = D;
   g.off_rings = up_to(kDHead, 1024);
   g.off_scales = g.off_rings + kDW * D * g.nib_stage;
@@ -244,7 +252,7 @@ struct DArgs {
   DecodeArgs a;
   DGeo G;
   int RT;          // units (row tiles) per virtual expert
-  int64_t C_max;   // upper bound of chunks (grid sizing only)
+  int U_max;       // upper bound of units (grid sizing only)
   alignas(64) CUtensorMap tqa, tqb;  // packed rows of the A / B projections (tensor-map mode)
 };
 
@@ -412,9 +420,9 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 // Stage the segment's activation rows as f16 scaled by 2^-shift[row]:
 // k_gateup: token rows of x (bf16 [T][H]); shift from the row's absmax.
 // k_down: pair rows of h (fp32 [P][I]); shift from k_gateup's per-tile maxima.
-// stage_issue() puts each thread's first batch of 16-byte loads in flight (it
-// runs before the weight stream starts); stage_finish() reduces the absmax,
-// converts and stores.
+// stage_issue() puts each thread's first batch of 16-byte loads in flight;
+// stage_finish() reduces the absmax, converts and stores.  With `ident`, row i
+// is token / pair i (every row of the call staged; row_key is not read).
 constexpr int kBatch = 16;
 
 struct StageRegs {
@@ -423,16 +431,17 @@ struct StageRegs {
 };
 
 template <bool GATEUP>
-__device__ __forceinline__ const uint4* stage_src(const DecodeArgs& a, const DHead& S, int j, int nvec) {
+__device__ __forceinline__ const uint4* stage_src(const DecodeArgs& a, const DHead& S, int j, int nvec,
+                                                  bool ident) {
   const int row = j / nvec, q = j - row * nvec;
-  const int key = S.row_key[row];
+  const int key = ident ? row : S.row_key[row];
   return GATEUP ? reinterpret_cast<const uint4*>(a.x + (size_t)key * a.H) + q
                 : reinterpret_cast<const uint4*>(a.h + (size_t)key * a.I) + q;
 }
 
 template <bool GATEUP>
 __device__ __forceinline__ void stage_issue(const DecodeArgs& a, const DHead& S, StageRegs& R,
-                                            int nrows) {
+                                            int nrows, bool ident) {
   const int tid = threadIdx.x, nth = kDW * 32;
   const int nvec = GATEUP ? a.H / 8 : a.I / 4;  // 16-byte vectors per source row
   const int total = nrows * nvec;
@@ -441,13 +450,16 @@ __device__ __forceinline__ void stage_issue(const DecodeArgs& a, const DHead& S,
 #pragma unroll
   for (int i = 0; i < kBatch; ++i) {
     const int j = i * nth + tid;
-    if (j < total) R.buf[i] = GATEUP ? __ldg(stage_src<GATEUP>(a, S, j, nvec)) : __ldcg(stage_src<GATEUP>(a, S, j, nvec));
+    if (j < total)
+      R.buf[i] = GATEUP ? __ldg(stage_src<GATEUP>(a, S, j, nvec, ident))
+                        : __ldcg(stage_src<GATEUP>(a, S, j, nvec, ident));
   }
   if (!GATEUP) {
     const int R1 = a.I / 8;
     for (int j = tid; j < nrows * R1; j += nth) {
       const int row = j / R1;
-      const float m = __ldcg(a.hmax + (size_t)S.row_key[row] * R1 + (j - row * R1));
+      const int key = ident ? row : S.row_key[row];
+      const float m = __ldcg(a.hmax + (size_t)key * R1 + (j - row * R1));
 #pragma unroll
       for (int r = 0; r < kXCap; ++r)
         if (r == row) R.am[r] = fmaxf(R.am[r], m);
@@ -466,7 +478,7 @@ __device__ __forceinline__ float bf16x8_absmax(const uint4& v) {
 
 template <bool GATEUP>
 __device__ __forceinline__ void stage_finish(const DecodeArgs& a, DHead& S, StageRegs& R,
-                                             __half* act, int stride, int nrows) {
+                                             __half* act, int stride, int nrows, bool ident) {
   const int tid = threadIdx.x, nth = kDW * 32;
   const int nvec = GATEUP ? a.H / 8 : a.I / 4;
   const int total = nrows * nvec;
@@ -484,7 +496,7 @@ __device__ __forceinline__ void stage_finish(const DecodeArgs& a, DHead& S, Stag
       }
     }
     for (int j = kBatch * nth + tid; j < total; j += nth) {
-      const float m = bf16x8_absmax(__ldg(stage_src<GATEUP>(a, S, j, nvec)));
+      const float m = bf16x8_absmax(__ldg(stage_src<GATEUP>(a, S, j, nvec, ident)));
       const int row = j / nvec;
 #pragma unroll
       for (int r = 0; r < kXCap; ++r)
@@ -512,8 +524,8 @@ __device__ __forceinline__ void stage_finish(const DecodeArgs& a, DHead& S, Stag
       const int j = base + i * nth + tid;
       if (j >= total) continue;
       const uint4 v = (held || base == 0) ? R.buf[i]
-                      : (GATEUP ? __ldg(stage_src<GATEUP>(a, S, j, nvec))
-                                : __ldcg(stage_src<GATEUP>(a, S, j, nvec)));
+                      : (GATEUP ? __ldg(stage_src<GATEUP>(a, S, j, nvec, ident))
+                                : __ldcg(stage_src<GATEUP>(a, S, j, nvec, ident)));
       const int row = j / nvec, q = j - row * nvec;
       const float sc = pow2f(-S.shift[row]);
       const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -539,7 +551,7 @@ __device__ __forceinline__ void stage_finish(const DecodeArgs& a, DHead& S, Stag
 // of the packed rows.  A stage's mbarrier completes on 33 arrivals (one
 // deferred arrival per lane once its cp.asyncs land, plus lane 0's
 // expect-tx arrival) and the TMA bytes.  Issuing from every warp keeps the
-// per-instruction cost of a tensor copy off the critical path.
+// per-instruction cost of a tensor copy off any single warp's critical path.
 template <int FA, int FB, bool GATEUP>
 __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ DArgs P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -557,29 +569,50 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
   const qk_weight& WA = GATEUP ? a.gate : a.down;
   const qk_weight& WB = GATEUP ? a.up : a.down;
   const int rows_per_e = GATEUP ? a.I : a.H;  // weight rows of one expert
+  const bool fast = G.fast != 0;
 
-  if (GATEUP) pdl_launch_dependents();
+  if (GATEUP) {
+    pdl_launch_dependents();
+    // k_down's row-tile counters start at zero; k_down touches them only after
+    // this grid has completed
+    if (blockIdx.x == 0)
+      for (int i = threadIdx.x; i < a.H / 16; i += blockDim.x) a.cnt[i] = 0u;
+  }
   if (lane == 0) {
     for (int i = 0; i < G.D; ++i) mbar_init(&full[i], 33);
     fence_mbar_init();
   }
   if (threadIdx.x == 0) S.dead = 0;
+  StageRegs SR;
+  if (GATEUP && fast) stage_issue<true>(a, S, SR, a.T, true);  // x does not depend on the routing
   build_route(a.ids, a.P, a.E, S.R);  // ends with a block barrier
-  const int64_t C = (int64_t)S.R.n_v * RT * nk;
-  const int64_t c0 = C * blockIdx.x / gridDim.x, c1 = C * (blockIdx.x + 1) / gridDim.x;
-  if (c0 >= c1) return;
+  const int n_v = S.R.n_v;
+  const int U = n_v * RT;
+  const int u_beg = (int)((int64_t)U * blockIdx.x / gridDim.x);
+  const int u_end = (int)((int64_t)U * (blockIdx.x + 1) / gridDim.x);
+  if (u_beg >= u_end) return;
+  if (fast) {  // one segment: every virtual expert, rows = all tokens / pairs
+    for (int i = threadIdx.x; i < n_v * kTileN; i += blockDim.x) {
+      const int v = i / kTileN, j = i - v * kTileN;
+      if (j < S.R.v_n[v]) {
+        const int pr = S.R.pair_list[S.R.v_p0[v] + j];
+        S.col_row[i] = (int8_t)(GATEUP ? pr / a.k : pr);
+      }
+    }
+    if (threadIdx.x < kXCap) S.row_key[threadIdx.x] = (int16_t)threadIdx.x;
+  }
 
   const uint64_t pol = policy_evict_first();
   const unsigned long long limit = g_wait_limit_ns;
   const int vpr = G.Kc / 32;  // 16-byte vectors per packed chunk row
   // Chunk c into stage `slot`.
-  auto issue = [&](int64_t c, int slot) {
+  auto issue = [&](int c, int slot) {
     uint8_t* st = nring + (size_t)slot * G.nib_stage;
     uint8_t* sd = sring + (size_t)slot * G.sc_stage;
     uint64_t* bar = &full[slot];
-    const int64_t u = c / nk;
-    const int kc = (int)(c - u * nk);
-    const int v = (int)(u / RT), r = (int)(u - (int64_t)v * RT);
+    const int u = c / nk;
+    const int kc = c - u * nk;
+    const int v = u / RT, r = u - v * RT;
     const int e = S.R.v_expert[v];
     const int64_t rowA0 = (int64_t)e * rows_per_e + (GATEUP ? r * 8 : r * 16);
     const int64_t rowB0 = GATEUP ? rowA0 : rowA0 + 8;
@@ -624,17 +657,123 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     }
   };
 
-  int64_t done = 0;  // chunks consumed by this warp (ring position)
-  bool dead = false;
-  bool bad = false;
+  // k_down: units this warp finished whose row-tile counters are not yet bumped
+  // (lane i holds the i-th); bumped in batches so the round trips overlap.
+  int pend = -1, npend = 0;
+  auto combine = [&](int r) {  // y rows r*16 .. r*16+15 of every token
+    const float* ures = a.ures;
+    for (int idx = lane; idx < a.T * 16; idx += 32) {
+      const int tok = idx >> 4, m = idx & 15;
+      const int ln = (m & 7) * 4, el = (m >= 8) ? 2 : 0;
+      float d[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {  // issue the loads of up to 8 slots together
+        d[s] = 0.f;
+        if (s < a.k) {
+          const int p = tok * a.k + s;
+          const int pv = S.R.pair_v[p];
+          if (pv >= 0) {
+            const int j = S.R.pair_j[p];
+            d[s] = __ldcg(ures + (((size_t)pv * RT + r) * 32 + ln + (j >> 1)) * 4 + el + (j & 1));
+          }
+        }
+      }
+      float yv = 0.f;
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        if (s < a.k) yv = fmaf(a.w[tok * a.k + s], d[s], yv);
+      for (int s = 8; s < a.k; ++s) {
+        const int p = tok * a.k + s;
+        const int pv = S.R.pair_v[p];
+        if (pv < 0) continue;
+        const int j = S.R.pair_j[p];
+        yv = fmaf(a.w[p], __ldcg(ures + (((size_t)pv * RT + r) * 32 + ln + (j >> 1)) * 4 + el + (j & 1)), yv);
+      }
+      const size_t o = (size_t)tok * a.H + r * 16 + m;
+      if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(yv);
+      else reinterpret_cast<float*>(a.y)[o] = yv;
+    }
+  };
+  auto flush = [&]() {
+    __threadfence();  // this warp's unit results, before the counters
+    __syncwarp();
+    bool last = false;
+    int r = 0;
+    if (lane < npend) {
+      r = pend % RT;
+      last = atom_add_acq_rel(a.cnt + r, 1u) + 1u == (uint32_t)n_v;
+    }
+    unsigned m = __ballot_sync(0xffffffffu, last);
+    if (m) __threadfence();
+    while (m) {
+      const int i = __ffs(m) - 1;
+      m &= m - 1;
+      combine(__shfl_sync(0xffffffffu, r, i));
+    }
+    npend = 0;
+  };
+
+  // A finished unit: scale, then SwiGLU into h (k_gateup) or the unit result (k_down).
+  auto finalize = [&](int u, float4 f, int seg_v0) {
+    const int v = u / RT, r = u - v * RT;
+    const int e = S.R.v_expert[v], n = S.R.v_n[v];
+    const float s2a = WA.fmt == QK_FMT_NVFP4 ? WA.scale_2[e] : 1.f;
+    const float s2b = WB.fmt == QK_FMT_NVFP4 ? WB.scale_2[e] : 1.f;
+    float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int jj = 0; jj < 2; ++jj) {
+      const int col = 2 * t + jj;
+      const float sx = col < n ? pow2f(S.shift[S.col_row[(v - seg_v0) * kTileN + col]]) : 0.f;
+      fv[jj] *= sx * s2a;
+      fv[2 + jj] *= sx * s2b;
+    }
+    if (GATEUP) {
+      float hm[2];
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int col = 2 * t + jj;
+        hm[jj] = 0.f;
+        if (col < n) {
+          const float hv = silu_mul(fv[jj], fv[2 + jj]);
+          const int p = S.R.pair_list[S.R.v_p0[v] + col];
+          a.h[(size_t)p * a.I + r * 8 + g] = hv;
+          hm[jj] = fabsf(hv);
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) hm[jj] = fmaxf(hm[jj], __shfl_xor_sync(0xffffffffu, hm[jj], o));
+      if (g == 0) {
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int col = 2 * t + jj;
+          if (col < n) a.hmax[(size_t)S.R.pair_list[S.R.v_p0[v] + col] * (a.I / 8) + r] = hm[jj];
+        }
+      }
+    } else {
+      reinterpret_cast<float4*>(a.ures)[(size_t)u * 32 + lane] = make_float4(fv[0], fv[1], fv[2], fv[3]);
+      if (lane == npend) pend = u;
+      if (++npend == 32) flush();
+    }
+  };
+
+  int done = 0;  // chunks consumed by this warp (ring position)
+  bool dead = false, bad = false;
   bool waited_pdl = false;
-  StageRegs SR;
-  int64_t c = c0;
-  while (c < c1) {
+  int u_seg = u_beg;
+  while (u_seg < u_end) {
     // ---- plan a segment: consecutive virtual experts whose rows fit xcap
-    if (threadIdx.x == 0) {
-      const int v0 = (int)(c / nk / RT);
-      const int vlast = (int)((c1 - 1) / nk / RT);
+    if (fast) {
+      if (threadIdx.x == 0) {
+        S.seg_u0 = u_beg;
+        S.seg_u1 = u_end;
+        S.seg_v0 = 0;
+        S.seg_rows = GATEUP ? a.T : a.P;
+      }
+    } else if (threadIdx.x == 0) {
+      const int v0 = u_seg / RT;
+      const int vlast = (u_end - 1) / RT;
       int rows = 0, v = v0;
       for (; v <= vlast; ++v) {
         const int n = S.R.v_n[v];
@@ -662,164 +801,83 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
         for (int j = 0; j < n; ++j) S.col_row[(v - v0) * kTileN + j] = cr[j];
         rows += add;
       }
+      S.seg_u0 = u_seg;
+      S.seg_u1 = min(u_end, v * RT);  // v > v0 always (one virtual expert has <= xcap rows)
       S.seg_v0 = v0;
-      S.seg_v1 = v;  // exclusive; v > v0 always (one virtual expert has <= xcap rows)
       S.seg_rows = rows;
     }
     __syncthreads();
-    const int seg_v0 = S.seg_v0, seg_v1 = S.seg_v1, seg_rows = S.seg_rows;
-    if (seg_v1 <= seg_v0) {  // cannot happen; never loop forever
+    const int seg_u0 = S.seg_u0, seg_u1 = S.seg_u1, seg_v0 = S.seg_v0, seg_rows = S.seg_rows;
+    if (seg_u1 <= seg_u0) {  // cannot happen; never loop forever
       set_status(QK_ERR_INVALID_ARG);
       break;
     }
-    const int64_t s_end = min(c1, (int64_t)seg_v1 * RT * nk);
-    const int64_t n_seg = s_end - c;
-    const int64_t w0 = c + n_seg * warp / kDW, w1 = c + n_seg * (warp + 1) / kDW;
-    const int64_t wn = w1 - w0;
+    const int cs = seg_u0 * nk, n_seg = (seg_u1 - seg_u0) * nk;
+    const int w0 = cs + (int)((int64_t)n_seg * warp / kDW);
+    const int w1 = cs + (int)((int64_t)n_seg * (warp + 1) / kDW);
+    const int wn = w1 - w0;
+    if (lane == 0) {
+      S.pu[warp][0] = S.pu[warp][1] = -1;
+      S.wempty[warp] = wn == 0;
+    }
 
-    // ---- activation loads first, then the weight prefetch (D-1 chunks), then staging
-    if (GATEUP) stage_issue<true>(a, S, SR, seg_rows);
-    for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (int)((done + i) % G.D));
+    // ---- weight prefetch (D-1 chunks), then the activation rows
+    for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (done + i) % G.D);
+    if (GATEUP && !fast) stage_issue<true>(a, S, SR, seg_rows, false);
     if (!GATEUP) {
       if (!waited_pdl) {
         pdl_wait();  // h and hmax come from k_gateup
         waited_pdl = true;
       }
-      stage_issue<false>(a, S, SR, seg_rows);
+      stage_issue<false>(a, S, SR, seg_rows, fast);
     }
-    stage_finish<GATEUP>(a, S, SR, act, G.act_stride, seg_rows);
+    stage_finish<GATEUP>(a, S, SR, act, G.act_stride, seg_rows, fast);
     __syncthreads();
 
     // ---- stream this warp's chunks
-    int64_t cur_u = -1;
-    int kc_start = 0, kc_last = 0;
+    int cur_u = -1, kc_start = 0, kc_last = 0, npieces = 0;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    auto emit = [&]() {
-      const int v = (int)(cur_u / RT), r = (int)(cur_u - (int64_t)v * RT);
-      const int e = S.R.v_expert[v], n = S.R.v_n[v];
-      const float s2a = WA.fmt == QK_FMT_NVFP4 ? WA.scale_2[e] : 1.f;
-      const float s2b = WB.fmt == QK_FMT_NVFP4 ? WB.scale_2[e] : 1.f;
-#pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int col = 2 * t + jj;
-        const float sx = col < n ? pow2f(S.shift[S.col_row[(v - seg_v0) * kTileN + col]]) : 0.f;
-        acc[jj] *= sx * s2a;
-        acc[2 + jj] *= sx * s2b;
-      }
-      const int len = kc_last + 1 - kc_start;
-      float4 fin = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      bool ready = GATEUP && kc_start == 0 && len == nk;
-      if (!ready) {
-        // publish this piece; the last contributor finishes the unit (k_gateup)
-        // or the whole row tile (k_down)
-        const int64_t slot = cur_u * nk + kc_start;
-        float4* part = reinterpret_cast<float4*>(GATEUP ? a.part1 : a.part2);
-        part[slot * 32 + lane] = fin;
-        if (lane == 0) (GATEUP ? a.len1 : a.len2)[slot] = (uint8_t)len;
-        __syncwarp();
-        uint32_t last = 0;
+    auto close = [&]() {
+      const float4 f = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      if (kc_start == 0 && kc_last == nk - 1) {
+        finalize(cur_u, f, seg_v0);
+      } else {  // cut by a warp boundary: the first or the last unit of this warp
+        const int sl = npieces++;
+        S.piece[warp][sl][lane] = f;
         if (lane == 0) {
-          const uint32_t need = GATEUP ? (uint32_t)nk : (uint32_t)(S.R.n_v * nk);
-          uint32_t* cnt = GATEUP ? a.cnt1 + cur_u : a.cnt2 + r;
-          last = (atom_add_acq_rel(cnt, (uint32_t)len) + (uint32_t)len == need) ? 1u : 0u;
-        }
-        ready = __shfl_sync(0xffffffffu, last, 0) != 0;
-        if (ready) {
-          __threadfence();
-          if (GATEUP) {  // sum the unit's pieces in chunk order
-            fin = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int kc = 0; kc < nk;) {
-              const int64_t sl = cur_u * nk + kc;
-              const float4 f = __ldcg(part + sl * 32 + lane);
-              fin.x += f.x; fin.y += f.y; fin.z += f.z; fin.w += f.w;
-              kc += __ldcg(a.len1 + sl);
-            }
-          }
-        }
-      }
-      if (!ready) return;
-      if (GATEUP) {
-        const float fv[4] = {fin.x, fin.y, fin.z, fin.w};
-        float hm[2];
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int col = 2 * t + jj;
-          hm[jj] = 0.f;
-          if (col < n) {
-            const float hv = silu_mul(fv[jj], fv[2 + jj]);
-            const int p = S.R.pair_list[S.R.v_p0[v] + col];
-            a.h[(size_t)p * a.I + r * 8 + g] = hv;
-            hm[jj] = fabsf(hv);
-          }
-        }
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-          for (int o = 4; o < 32; o <<= 1)
-            hm[jj] = fmaxf(hm[jj], __shfl_xor_sync(0xffffffffu, hm[jj], o));
-        if (g == 0) {
-#pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const int col = 2 * t + jj;
-            if (col < n) a.hmax[(size_t)S.R.pair_list[S.R.v_p0[v] + col] * (a.I / 8) + r] = hm[jj];
-          }
-        }
-      } else {
-        // every piece of row tile r is in: y[t][r*16+m] = sum_s w * sum_pieces
-        const float* part = a.part2;
-        for (int idx = lane; idx < a.T * 16; idx += 32) {
-          const int tok = idx >> 4, m = idx & 15;
-          const int ln = (m & 7) * 4, el = (m >= 8) ? 2 : 0;
-          float yv = 0.f;
-          for (int sl = 0; sl < a.k; ++sl) {
-            const int p = tok * a.k + sl;
-            const int pv = S.R.pair_v[p];
-            if (pv < 0) continue;
-            const int j = S.R.pair_j[p];
-            const int64_t uu = (int64_t)pv * RT + r;
-            float d = 0.f;
-            for (int kc = 0; kc < nk;) {
-              const int64_t sl2 = uu * nk + kc;
-              d += __ldcg(part + (sl2 * 32 + ln + (j >> 1)) * 4 + el + (j & 1));
-              kc += __ldcg(a.len2 + sl2);
-            }
-            yv = fmaf(a.w[p], d, yv);
-          }
-          const size_t o = (size_t)tok * a.H + r * 16 + m;
-          if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(yv);
-          else reinterpret_cast<float*>(a.y)[o] = yv;
+          S.pu[warp][sl] = cur_u;
+          S.pstart[warp][sl] = kc_start;
         }
       }
     };
-
-    for (int64_t i = 0; i < wn; ++i) {
+    for (int i = 0; i < wn; ++i) {
       // keep D-1 chunks in flight: issue chunk i+D-1, then wait for chunk i
-      if (i + G.D - 1 < wn) issue(w0 + i + G.D - 1, (int)((done + G.D - 1) % G.D));
-      const int slot = (int)(done % G.D);
+      if (i + G.D - 1 < wn) issue(w0 + i + G.D - 1, (done + G.D - 1) % G.D);
+      const int slot = done % G.D;
       const bool landed = mbar_wait_bounded(&full[slot], (uint32_t)((done / G.D) & 1), limit);
       if (__any_sync(0xffffffffu, !landed)) {
         // the copies did not land in time: report, drain what this warp has in
         // flight, and stop the block at the end of the segment
         set_status(QK_ERR_TIMEOUT);
-        const int64_t inflight = (wn - i < G.D) ? wn - i : (int64_t)G.D;
-        for (int64_t q = 0; q < inflight; ++q)
+        const int inflight = min(wn - i, G.D);
+        for (int q = 0; q < inflight; ++q)
           if (!mbar_wait_bounded(&full[(done + q) % G.D], (uint32_t)(((done + q) / G.D) & 1),
                                  kDrainLimitNs))
             break;
         dead = true;
         break;
       }
-      const int64_t cc = w0 + i;
-      const int64_t u = cc / nk;
-      const int kc = (int)(cc - u * nk);
+      const int cc = w0 + i;
+      const int u = cc / nk;
+      const int kc = cc - u * nk;
       if (u != cur_u) {
-        if (cur_u >= 0) emit();
+        if (cur_u >= 0) close();
         cur_u = u;
         kc_start = kc;
         acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
       }
       kc_last = kc;
-      const int v = (int)(u / RT);
+      const int v = u / RT;
       const int n = S.R.v_n[v];
       const int row = S.col_row[(v - seg_v0) * kTileN + (g < n ? g : 0)];
       const __half* xrow = act + (size_t)row * G.act_stride + 8 * t + (size_t)kc * G.Kc;
@@ -831,12 +889,28 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     if (dead) {
       if (lane == 0) S.dead = 1;
     } else if (cur_u >= 0) {
-      emit();
+      close();
     }
     __syncthreads();
     if (S.dead) break;
-    c = s_end;
+    // ---- units cut by warp boundaries: the warp holding the first chunk adds
+    // the pieces in chunk order
+    for (int sl = 0; sl < 2; ++sl) {
+      const int u = S.pu[warp][sl];
+      if (u < 0 || S.pstart[warp][sl] != 0) continue;
+      float4 f = S.piece[warp][sl][lane];
+      for (int w2 = warp + 1; w2 < kDW; ++w2) {
+        if (S.wempty[w2]) continue;
+        if (S.pu[w2][0] != u) break;
+        const float4 q = S.piece[w2][0][lane];
+        f.x += q.x; f.y += q.y; f.z += q.z; f.w += q.w;
+      }
+      finalize(u, f, seg_v0);
+    }
+    __syncthreads();  // the next segment reuses the staged rows and the pieces
+    u_seg = seg_u1;
   }
+  if (!GATEUP && npend > 0 && !dead) flush();
   if (bad) set_status(QK_ERR_NAN_SCALE);
 }
 
@@ -873,7 +947,7 @@ static bool encode_rows(CUtensorMap* m, const uint8_t* q, int64_t rows, int K, i
 
 template <int FA, int FB, bool GATEUP>
 static qk_status go(DArgs& P, cudaStream_t st, bool pdl) {
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), P.C_max));
+  const int grid = std::max(1, std::min(num_sms(), P.U_max));
   auto kern = k_decode<FA, FB, GATEUP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P.G.smem) !=
       cudaSuccess)
@@ -891,33 +965,35 @@ static qk_status go(DArgs& P, cudaStream_t st, bool pdl) {
   return cudaLaunchKernelEx(&cfg, kern, P) == cudaSuccess ? QK_OK : QK_ERR_CUDA;
 }
 
+// Geometry of one kernel: tensor-map mode when the maps encode, else rows by cp.async.
+static DGeo plan_kernel(int K, int fa, int fb, int rows, CUtensorMap* ta, CUtensorMap* tb,
+                        const uint8_t* qa, const uint8_t* qb, int64_t n_rows, int box_rows) {
+  const int xcap = std::min(rows, kXCap);
+  DGeo G = plan_geo(K, fa, fb, xcap, true);
+  if (G.smem && G.tmap) {
+    bool ok = encode_rows(ta, qa, n_rows, K, box_rows, G.nseg);
+    if (ok && tb) ok = encode_rows(tb, qb, n_rows, K, box_rows, G.nseg);
+    if (!ok) G = plan_geo(K, fa, fb, xcap, false);
+  }
+  G.fast = rows <= kXCap ? 1 : 0;
+  return G;
+}
+
 qk_status decode_forward(DecodeArgs args, cudaStream_t st) {
-  // the piece counters start at zero on every call
-  if (cudaMemsetAsync(args.cnt1, 0, args.cnt_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
   DArgs P1 = {};
   P1.a = args;
   P1.RT = args.I / 8;
-  const int x1 = std::min(args.T, kXCap);
-  P1.G = plan_geo(args.H, args.gate.fmt, args.up.fmt, x1, true);
-  if (P1.G.tmap) {
-    const int64_t rows = (int64_t)args.E * args.I;
-    if (!encode_rows(&P1.tqa, args.gate.q, rows, args.H, 8, P1.G.nseg) ||
-        !encode_rows(&P1.tqb, args.up.q, rows, args.H, 8, P1.G.nseg))
-      P1.G = plan_geo(args.H, args.gate.fmt, args.up.fmt, x1, false);
-  }
+  P1.G = plan_kernel(args.H, args.gate.fmt, args.up.fmt, args.T, &P1.tqa, &P1.tqb, args.gate.q,
+                     args.up.q, (int64_t)args.E * args.I, 8);
   if (!P1.G.smem) return QK_ERR_UNSUPPORTED;
-  P1.C_max = (int64_t)args.P * P1.RT * P1.G.nk;  // virtual experts <= pairs
+  P1.U_max = args.P * P1.RT;  // virtual experts <= pairs
   DArgs P2 = {};
   P2.a = args;
   P2.RT = args.H / 16;
-  const int x2 = std::min(args.P, kXCap);
-  P2.G = plan_geo(args.I, args.down.fmt, args.down.fmt, x2, true);
-  if (P2.G.tmap) {
-    if (!encode_rows(&P2.tqa, args.down.q, (int64_t)args.E * args.H, args.I, 16, P2.G.nseg))
-      P2.G = plan_geo(args.I, args.down.fmt, args.down.fmt, x2, false);
-  }
+  P2.G = plan_kernel(args.I, args.down.fmt, args.down.fmt, args.P, &P2.tqa, nullptr, args.down.q,
+                     nullptr, (int64_t)args.E * args.H, 16);
   if (!P2.G.smem) return QK_ERR_UNSUPPORTED;
-  P2.C_max = (int64_t)args.P * P2.RT * P2.G.nk;
+  P2.U_max = args.P * P2.RT;
   constexpr int MX = QK_FMT_MXFP4, NV = QK_FMT_NVFP4;
   const int fg = args.gate.fmt, fu = args.up.fmt, fd = args.down.fmt;
   qk_status rc;
@@ -929,28 +1005,20 @@ qk_status decode_forward(DecodeArgs args, cudaStream_t st) {
   return fd == MX ? go<MX, MX, false>(P2, st, true) : go<NV, NV, false>(P2, st, true);
 }
 
-// Workspace: h [P][I] f32 | hmax [P][I/8] | part1 [U1*nk1][32] float4 |
-// part2 [U2*nk2][32] float4 | len1 | len2 | cnt1 [U1] | cnt2 [H/16].
-// Chunk counts are sized for the smallest chunk the planner may pick (128).
+// Workspace: h [P][I] f32 | hmax [P][I/8] | ures [P*H/16][32] float4 | cnt [H/16].
 struct WsLayout {
-  size_t h, hmax, part1, part2, len1, len2, cnt1, cnt2, total;
+  size_t h, hmax, ures, cnt, total;
 };
 
 static WsLayout ws_layout(int T, int k, int H, int I) {
   const size_t P = (size_t)T * k;
-  const size_t nk1 = (size_t)H / 128, nk2 = (size_t)I / 128;
-  const size_t U1 = P * (I / 8), U2 = P * (H / 16);
   WsLayout L;
   size_t o = 0;
   L.h = o; o += align256(P * I * 4);
   L.hmax = o; o += align256(P * (I / 8) * 4);
-  L.part1 = o; o += align256(U1 * nk1 * 512);
-  L.part2 = o; o += align256(U2 * nk2 * 512);
-  L.len1 = o; o += align256(U1 * nk1);
-  L.len2 = o; o += align256(U2 * nk2);
-  L.cnt1 = o; o += U1 * 4;
-  L.cnt2 = o; o += (size_t)(H / 16) * 4;
-  L.total = align256(o);
+  L.ures = o; o += align256(P * (H / 16) * 512);
+  L.cnt = o; o += align256((size_t)(H / 16) * 4);
+  L.total = o;
   return L;
 }
 
@@ -961,13 +1029,8 @@ void decode_carve(DecodeArgs& a, void* ws) {
   uint8_t* p = static_cast<uint8_t*>(ws);
   a.h = reinterpret_cast<float*>(p + L.h);
   a.hmax = reinterpret_cast<float*>(p + L.hmax);
-  a.part1 = reinterpret_cast<float*>(p + L.part1);
-  a.part2 = reinterpret_cast<float*>(p + L.part2);
-  a.len1 = p + L.len1;
-  a.len2 = p + L.len2;
-  a.cnt1 = reinterpret_cast<uint32_t*>(p + L.cnt1);
-  a.cnt2 = reinterpret_cast<uint32_t*>(p + L.cnt2);
-  a.cnt_bytes = L.total - L.cnt1;
+  a.ures = reinterpret_cast<float*>(p + L.ures);
+  a.cnt = reinterpret_cast<uint32_t*>(p + L.cnt);
 }
 
 }  // namespace qk

@@ -26,13 +26,8 @@ struct DecodeArgs {
   // workspace
   float* h;           // [P][I] fp32 SwiGLU output
   float* hmax;        // [P][I/8] absmax of h per 8-row tile
-  float* part1;       // k_gateup pieces of split units
-  float* part2;       // k_down pieces (every unit)
-  uint8_t* len1;      // chunks per piece
-  uint8_t* len2;
-  uint32_t* cnt1;     // chunks finished per k_gateup unit
-  uint32_t* cnt2;     // chunks finished per k_down row tile (follows cnt1)
-  size_t cnt_bytes;   // bytes zeroed from cnt1 on every call
+  float* ures;        // [units][32] float4: k_down result of each (virtual expert, row tile)
+  uint32_t* cnt;      // [H/16] k_down units finished per row tile (zeroed by k_gateup)
 };
 
 qk_status decode_forward(DecodeArgs args, cudaStream_t st);
