@@ -213,7 +213,7 @@ struct DHead {
   int pu[kDW][2];                       // unit of the warp's first / last piece (-1: none)
   int pstart[kDW][2];                   // first chunk of that piece within its unit
   int wempty[kDW];                      // the warp has no chunk in this segment
-  float red8[kDW][kXCap];
+  unsigned amax_bits[kXCap];            // row maxima (bit patterns of non-negative floats)
   float4 piece[kDW][2][32];             // partial sums of units cut by a warp boundary
   alignas(8) uint64_t full[kDW][kMaxD];
 };
@@ -417,54 +417,18 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 }
 
 // ------------------------------------------------------------- staging --
-// Stage the segment's activation rows as f16 scaled by 2^-shift[row]:
-// k_gateup: token rows of x (bf16 [T][H]); shift from the row's absmax.
-// k_down: pair rows of h (fp32 [P][I]); shift from k_gateup's per-tile maxima.
-// stage_issue() puts each thread's first batch of 16-byte loads in flight;
-// stage_finish() reduces the absmax, converts and stores.  With `ident`, row i
-// is token / pair i (every row of the call staged; row_key is not read).
-constexpr int kBatch = 16;
-
-struct StageRegs {
-  uint4 buf[kBatch];
-  float am[kXCap];
-};
-
-template <bool GATEUP>
-__device__ __forceinline__ const uint4* stage_src(const DecodeArgs& a, const DHead& S, int j, int nvec,
-                                                  bool ident) {
-  const int row = j / nvec, q = j - row * nvec;
-  const int key = ident ? row : S.row_key[row];
-  return GATEUP ? reinterpret_cast<const uint4*>(a.x + (size_t)key * a.H) + q
-                : reinterpret_cast<const uint4*>(a.h + (size_t)key * a.I) + q;
-}
-
-template <bool GATEUP>
-__device__ __forceinline__ void stage_issue(const DecodeArgs& a, const DHead& S, StageRegs& R,
-                                            int nrows, bool ident) {
-  const int tid = threadIdx.x, nth = kDW * 32;
-  const int nvec = GATEUP ? a.H / 8 : a.I / 4;  // 16-byte vectors per source row
-  const int total = nrows * nvec;
-#pragma unroll
-  for (int i = 0; i < kXCap; ++i) R.am[i] = 0.f;
-#pragma unroll
-  for (int i = 0; i < kBatch; ++i) {
-    const int j = i * nth + tid;
-    if (j < total)
-      R.buf[i] = GATEUP ? __ldg(stage_src<GATEUP>(a, S, j, nvec, ident))
-                        : __ldcg(stage_src<GATEUP>(a, S, j, nvec, ident));
-  }
-  if (!GATEUP) {
-    const int R1 = a.I / 8;
-    for (int j = tid; j < nrows * R1; j += nth) {
-      const int row = j / R1;
-      const int key = ident ? row : S.row_key[row];
-      const float m = __ldcg(a.hmax + (size_t)key * R1 + (j - row * R1));
-#pragma unroll
-      for (int r = 0; r < kXCap; ++r)
-        if (r == row) R.am[r] = fmaxf(R.am[r], m);
-    }
-  }
+// The segment's activation rows are staged as f16 scaled by 2^-shift[row], the
+// shift putting the row's largest magnitude in [2^14, 2^15):
+//   k_gateup: token rows of x (bf16 [T][H]) are copied raw into the staging
+//     area by cp.async (issued before the weight stream), then converted in
+//     place once the row maxima are known;
+//   k_down: pair rows of h (fp32 [P][I]); the row maxima come from k_gateup's
+//     per-tile maxima.
+// The loops stay rolled: they run once per segment, and compact code keeps the
+// cold start of the block short.  With `ident`, row i is token / pair i (every
+// row of the call staged; row_key is not read).
+__device__ __forceinline__ void cp_async16_nohint(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
 __device__ __forceinline__ float bf16x8_absmax(const uint4& v) {
@@ -476,71 +440,81 @@ __device__ __forceinline__ float bf16x8_absmax(const uint4& v) {
   return m;
 }
 
-template <bool GATEUP>
-__device__ __forceinline__ void stage_finish(const DecodeArgs& a, DHead& S, StageRegs& R,
-                                             __half* act, int stride, int nrows, bool ident) {
-  const int tid = threadIdx.x, nth = kDW * 32;
-  const int nvec = GATEUP ? a.H / 8 : a.I / 4;
-  const int total = nrows * nvec;
-  const bool held = total <= kBatch * nth;
-  if (GATEUP) {  // absmax over the x rows (first batch in registers, the rest re-read)
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int j = i * nth + tid;
-      if (j < total) {
-        const float m = bf16x8_absmax(R.buf[i]);
-        const int row = j / nvec;
-#pragma unroll
-        for (int r = 0; r < kXCap; ++r)
-          if (r == row) R.am[r] = fmaxf(R.am[r], m);
-      }
-    }
-    for (int j = kBatch * nth + tid; j < total; j += nth) {
-      const float m = bf16x8_absmax(__ldg(stage_src<GATEUP>(a, S, j, nvec, ident)));
-      const int row = j / nvec;
-#pragma unroll
-      for (int r = 0; r < kXCap; ++r)
-        if (r == row) R.am[r] = fmaxf(R.am[r], m);
-    }
-  }
-  const int lane = tid & 31, warp = tid >> 5;
-#pragma unroll
-  for (int r = 0; r < kXCap; ++r) {
-    float m = R.am[r];
+// Max of m into the row's slot; `row` is warp-uniform when `uniform`.
+__device__ __forceinline__ void row_max(DHead& S, int row, float m, bool uniform) {
+  if (uniform) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) S.red8[warp][r] = m;
+    if ((threadIdx.x & 31) == 0) atomicMax(&S.amax_bits[row], __float_as_uint(m));
+  } else {
+    atomicMax(&S.amax_bits[row], __float_as_uint(m));
   }
+}
+
+// Shifts from the row maxima (non-negative floats order like their bit patterns).
+__device__ __forceinline__ void rows_shift(DHead& S, int nrows) {
   __syncthreads();
-  if (tid < nrows) {
-    float m = 0.f;
-    for (int w = 0; w < kDW; ++w) m = fmaxf(m, S.red8[w][tid]);
-    S.shift[tid] = clamp_shift(f16_shift_for(m));
+  if (threadIdx.x < nrows) S.shift[threadIdx.x] = clamp_shift(f16_shift_for(__uint_as_float(S.amax_bits[threadIdx.x])));
+  __syncthreads();
+}
+
+__device__ __forceinline__ void stage_x_issue(const DecodeArgs& a, const DHead& S, __half* act, int stride,
+                                              int nrows, bool ident) {
+  const int nvec = a.H / 8;
+  for (int j = threadIdx.x; j < nrows * nvec; j += kDW * 32) {
+    const int row = j / nvec, q = j - row * nvec;
+    const int key = ident ? row : S.row_key[row];
+    cp_async16_nohint(act + (size_t)row * stride + q * 8, a.x + (size_t)key * a.H + q * 8);
   }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void stage_x_finish(const DecodeArgs& a, DHead& S, __half* act, int stride,
+                                               int nrows) {
+  const int nvec = a.H / 8;
+  const bool uniform = nvec % 32 == 0;  // a warp's 32 vectors lie in one row
+  if (threadIdx.x < kXCap) S.amax_bits[threadIdx.x] = 0u;
+  asm volatile("cp.async.wait_group 0;" ::: "memory");  // the x group only: ring copies are not grouped
   __syncthreads();
-  for (int base = 0; base < total; base += kBatch * nth) {
+  for (int j = threadIdx.x; j < nrows * nvec; j += kDW * 32) {
+    const int row = j / nvec, q = j - row * nvec;
+    row_max(S, row, bf16x8_absmax(*reinterpret_cast<const uint4*>(act + (size_t)row * stride + q * 8)), uniform);
+  }
+  rows_shift(S, nrows);
+  for (int j = threadIdx.x; j < nrows * nvec; j += kDW * 32) {  // bf16 -> f16 in place
+    const int row = j / nvec, q = j - row * nvec;
+    uint4* pv = reinterpret_cast<uint4*>(act + (size_t)row * stride + q * 8);
+    const uint4 v = *pv;
+    const float sc = pow2f(-S.shift[row]);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int j = base + i * nth + tid;
-      if (j >= total) continue;
-      const uint4 v = (held || base == 0) ? R.buf[i]
-                      : (GATEUP ? __ldg(stage_src<GATEUP>(a, S, j, nvec, ident))
-                                : __ldcg(stage_src<GATEUP>(a, S, j, nvec, ident)));
-      const int row = j / nvec, q = j - row * nvec;
-      const float sc = pow2f(-S.shift[row]);
-      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-      if (GATEUP) {  // 8 bf16 -> 8 f16
-        uint32_t o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          o[e] = pack_f16x2(bf16_bits_to_f32(wv[e] & 0xFFFFu) * sc, bf16_bits_to_f32(wv[e] >> 16) * sc);
-        reinterpret_cast<uint4*>(act + (size_t)row * stride)[q] = make_uint4(o[0], o[1], o[2], o[3]);
-      } else {  // 4 fp32 -> 4 f16
-        const uint2 o = make_uint2(pack_f16x2(__uint_as_float(wv[0]) * sc, __uint_as_float(wv[1]) * sc),
-                                   pack_f16x2(__uint_as_float(wv[2]) * sc, __uint_as_float(wv[3]) * sc));
-        reinterpret_cast<uint2*>(act + (size_t)row * stride)[q] = o;
-      }
-    }
+    for (int e = 0; e < 4; ++e)
+      o[e] = pack_f16x2(bf16_bits_to_f32(wv[e] & 0xFFFFu) * sc, bf16_bits_to_f32(wv[e] >> 16) * sc);
+    *pv = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+__device__ __forceinline__ void stage_h(const DecodeArgs& a, DHead& S, __half* act, int stride, int nrows,
+                                        bool ident) {
+  const int R1 = a.I / 8;  // maxima per pair row
+  if (threadIdx.x < kXCap) S.amax_bits[threadIdx.x] = 0u;
+  __syncthreads();
+  for (int j = threadIdx.x; j < nrows * R1; j += kDW * 32) {
+    const int row = j / R1;
+    const int key = ident ? row : S.row_key[row];
+    row_max(S, row, __ldcg(a.hmax + (size_t)key * R1 + (j - row * R1)), R1 % 32 == 0);
+  }
+  rows_shift(S, nrows);
+  const int nvec = a.I / 4;
+#pragma unroll 4
+  for (int j = threadIdx.x; j < nrows * nvec; j += kDW * 32) {
+    const int row = j / nvec, q = j - row * nvec;
+    const int key = ident ? row : S.row_key[row];
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(a.h + (size_t)key * a.I) + q);
+    const float sc = pow2f(-S.shift[row]);
+    reinterpret_cast<uint2*>(act + (size_t)row * stride)[q] =
+        make_uint2(pack_f16x2(v.x * sc, v.y * sc), pack_f16x2(v.z * sc, v.w * sc));
   }
 }
 
@@ -581,10 +555,13 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
   if (lane == 0) {
     for (int i = 0; i < G.D; ++i) mbar_init(&full[i], 33);
     fence_mbar_init();
+    if (G.tmap && warp == 0) {
+      tmap_prefetch(&P.tqa);
+      if (GATEUP) tmap_prefetch(&P.tqb);
+    }
   }
   if (threadIdx.x == 0) S.dead = 0;
-  StageRegs SR;
-  if (GATEUP && fast) stage_issue<true>(a, S, SR, a.T, true);  // x does not depend on the routing
+  if (GATEUP && fast) stage_x_issue(a, S, act, G.act_stride, a.T, true);  // x does not depend on the routing
   build_route(a.ids, a.P, a.E, S.R);  // ends with a block barrier
   const int n_v = S.R.n_v;
   const int U = n_v * RT;
@@ -821,17 +798,21 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
       S.wempty[warp] = wn == 0;
     }
 
-    // ---- weight prefetch (D-1 chunks), then the activation rows
-    for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (done + i) % G.D);
-    if (GATEUP && !fast) stage_issue<true>(a, S, SR, seg_rows, false);
-    if (!GATEUP) {
+    // ---- k_gateup: x copies (their own cp.async group), weight prefetch (D-1
+    // chunks), then the conversion of x.  k_down: h first (it is in L2 and must
+    // not queue behind the weight stream), then the weight prefetch.
+    if (GATEUP) {
+      if (!fast) stage_x_issue(a, S, act, G.act_stride, seg_rows, false);
+      for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (done + i) % G.D);
+      stage_x_finish(a, S, act, G.act_stride, seg_rows);
+    } else {
       if (!waited_pdl) {
         pdl_wait();  // h and hmax come from k_gateup
         waited_pdl = true;
       }
-      stage_issue<false>(a, S, SR, seg_rows, fast);
+      stage_h(a, S, act, G.act_stride, seg_rows, fast);
+      for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (done + i) % G.D);
     }
-    stage_finish<GATEUP>(a, S, SR, act, G.act_stride, seg_rows, fast);
     __syncthreads();
 
     // ---- stream this warp's chunks
