@@ -92,10 +92,11 @@ typedef struct qk_moe_layer {
  *  x_bf16    [T][hidden] bf16.        topk_ids [T][top_k] int32 in [0, E).
  *  topk_w    [T][top_k] fp32.         y        [T][hidden] fp32 (y_is_bf16=0) or bf16.
  *  act_quant QK_ACT_NONE.             workspace >= moe_expert_workspace_size(), 256-B aligned.
- * Shapes: hidden and inter multiples of 128; 1 <= top_k <= 8.  Token counts
- * 1..16 run the decode path (CUDA-core decode of nibbles and scales in
- * registers, tensor-core m16n8k16 products, fp32 accumulation); larger counts
- * run the grouped path.  T = 0 returns QK_OK and launches nothing.
+ * Shapes: hidden and inter multiples of 128; 1 <= top_k <= 8.  The decode
+ * path (nibbles and scales decoded in registers, tensor-core m16n8k16
+ * products, fp32 accumulation) takes up to floor(128/top_k) tokens per launch;
+ * larger counts run as consecutive launches over slices of that many tokens,
+ * in order, on `stream`.  T = 0 returns QK_OK and launches nothing.
  * Errors: QK_ERR_INVALID_ARG (shapes, pointers, formats), QK_ERR_WORKSPACE,
  * QK_ERR_UNSUPPORTED (act_quant), QK_ERR_CUDA; device: QK_ERR_NAN_SCALE,
  * QK_ERR_INVALID_ARG (id out of range: that pair contributes nothing),

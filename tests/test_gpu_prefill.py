@@ -1,0 +1,72 @@
+"""GPU parity of moe_expert_forward at token counts beyond one launch's
+routing capacity (consecutive launches over token slices), the 43-layer
+stack's mixed-format decode layer, and the 2048-token Zipf prefill layer
+(checked on sampled tokens; the oracle computes those tokens only).
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_quantized_expert_mxfp4_b200 as qk
+import oracle
+from block_quantized_expert_mxfp4_b200 import synth, workload
+from helpers import MX, NV, assert_parity, oracle_moe
+
+pytestmark = pytest.mark.gpu
+
+
+def _forward(layer, x, ids, w):
+    lay = layer.c()
+    T, k = ids.shape
+    y = torch.full((T, x.shape[1]), float("nan"), dtype=torch.float32, device="cuda")
+    ws = torch.empty(qk.moe_expert_workspace_size(lay, T, k), dtype=torch.uint8, device="cuda")
+    qk.moe_expert_forward(lay, x, ids, w, y, ws)
+    assert qk.qk_last_device_status() == qk.QK_OK
+    return y
+
+
+@pytest.mark.parametrize("T", [65, 150])
+def test_token_counts_beyond_one_launch(T):
+    """Tiny layer, top-2: 64 tokens per launch, so 2 and 3 launches."""
+    wl = synth.WORKLOADS["tiny"]
+    layer = workload.make_layer(wl, T, 0)
+    x = synth.activations(T, T, wl.H)
+    lg = synth.router_logits(T, T, wl.E)
+    oids, ow = oracle.route_topk(lg, wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
+    yo = oracle_moe(wl, T, 0, x, oids, ow.astype(np.float32).astype(np.float64))
+    assert_parity(y.cpu().numpy(), yo, what=f"tiny T={T}")
+
+
+def test_stack_layer_mixed_formats():
+    """One layer of the pruned 43-layer stack: 180 experts, top-6, 8 tokens,
+    the seeded per-projection format choice of layer 5."""
+    wl = synth.WORKLOADS["stack43"]
+    fmts = tuple(int(f) for f in synth.format_choice(0, wl.layers)[5])
+    layer = workload.make_layer(wl, 0, 5, fmts)
+    x = synth.activations(0, wl.T, wl.H, stream=5)
+    lg = synth.router_logits(0, wl.T, wl.E, stream=5)
+    oids, ow = oracle.route_topk(lg, wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
+    yo = oracle_moe(wl, 0, 5, x, oids, ow.astype(np.float32).astype(np.float64), fmts)
+    assert_parity(y.cpu().numpy(), yo, what=f"stack layer 5 {fmts}")
+
+
+def test_prefill_zipf_sampled_tokens():
+    """2048 tokens, Zipf-skewed routing over 256 experts; 12 sampled tokens
+    (including ones routed to the most and least loaded experts) against the
+    oracle."""
+    wl = synth.WORKLOADS["prefill"]
+    layer = workload.make_layer(wl, 0, 0)
+    x = synth.activations(0, wl.T, wl.H)
+    lg = synth.zipf_logits(0, wl.T, wl.E, wl.k)
+    oids, ow = oracle.route_topk(lg, wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
+    counts = np.bincount(oids.reshape(-1), minlength=wl.E)
+    hot, cold = int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
+    pick = {int(np.nonzero((oids == hot).any(1))[0][0]), int(np.nonzero((oids == cold).any(1))[0][0])}
+    rng = np.random.default_rng(7)
+    pick |= set(int(t) for t in rng.choice(wl.T, 10, replace=False))
+    pick = sorted(pick)
+    yo = oracle_moe(wl, 0, 0, x[pick], oids[pick], ow[pick].astype(np.float32).astype(np.float64))
+    assert_parity(y.cpu().numpy()[pick], yo, what="prefill sampled tokens")
