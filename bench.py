@@ -128,11 +128,11 @@ def peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the decode kernels' sources (the kernel file and the headers it includes)."""
     from block_quantized_expert_mxfp4_b200 import build as b
     h = hashlib.sha256()
-    for p in sorted(b.sources()) + [os.path.join(b.CSRC, n) for n in sorted(os.listdir(b.CSRC))
-                                    if n.endswith((".cuh", ".h"))]:
-        h.update(open(p, "rb").read())
+    for n in ("qk_decode.cu", "qk_device.cuh", "qk_common.cuh", "qk_internal.h", "qk_tmap.h"):
+        h.update(open(os.path.join(b.CSRC, n), "rb").read())
     return h.hexdigest()[:16]
 
 
