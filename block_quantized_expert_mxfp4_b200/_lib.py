@@ -27,7 +27,7 @@ SYMBOLS = (
     "moe_expert_workspace_size", "moe_expert_forward", "moe_route_topk",
     "quant_convert_mxfp4_to_nvfp4", "fp8_block_linear", "fp8_shared_expert_workspace_size",
     "fp8_shared_expert_forward", "qk_last_device_status", "qk_status_string",
-    "qk_debug_set_wait_limit_ns",
+    "qk_debug_set_wait_limit_ns", "moe_expert_forward_noalloc",
 )
 
 
@@ -65,6 +65,9 @@ def load() -> ctypes.CDLL:
     L.moe_expert_forward.restype = i32
     L.moe_expert_forward.argtypes = [ctypes.POINTER(qk_moe_layer), vp, i32, vp, vp, i32, vp, i32,
                                      i32, vp, sz, vp]
+    L.moe_expert_forward_noalloc.restype = i32
+    L.moe_expert_forward_noalloc.argtypes = [ctypes.POINTER(qk_moe_layer), vp, i32, vp, vp, i32, vp,
+                                             i32, vp]
     L.moe_route_topk.restype = i32
     L.moe_route_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     L.quant_convert_mxfp4_to_nvfp4.restype = i32
@@ -129,6 +132,17 @@ def moe_expert_forward(layer: qk_moe_layer, x: torch.Tensor, topk_ids: torch.Ten
                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _stream(stream))
     _check(rc, "moe_expert_forward")
+
+
+def moe_expert_forward_noalloc(layer: qk_moe_layer, x: torch.Tensor, topk_ids: torch.Tensor,
+                               topk_w: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """moe_expert_forward with the library's fixed scratch array (no workspace)."""
+    T = x.shape[0]
+    k = topk_ids.shape[1] if topk_ids.dim() == 2 else 1
+    rc = load().moe_expert_forward_noalloc(ctypes.byref(layer), _ptr(x), T, _ptr(topk_ids),
+                                           _ptr(topk_w), k, _ptr(y), int(y.dtype == torch.bfloat16),
+                                           _stream(stream))
+    _check(rc, "moe_expert_forward_noalloc")
 
 
 def moe_route_topk(logits: torch.Tensor, top_k: int, ids: torch.Tensor, w: torch.Tensor,

@@ -110,6 +110,28 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
                              void* workspace, size_t workspace_bytes, qk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * moe_expert_forward_noalloc -- moe_expert_forward (act_quant QK_ACT_NONE)
+ * with its scratch taken from a fixed 4 MiB device array inside libqk.so
+ * instead of a caller workspace.  The pages have no counterpart: it exists for
+ * callers that cannot allocate device memory on the call path (a C caller
+ * embedded in a runtime that owns every device allocation).
+ *  Arguments as moe_expert_forward.  The call needs
+ *  moe_expert_workspace_size(L, n_tokens, top_k) <= 4 MiB (hidden 4096,
+ *  inter 2048: up to 28 pairs per launch); larger requests return
+ *  QK_ERR_WORKSPACE and launch nothing.  Nothing in the array has to start at
+ *  zero.  The array is shared by every call on a device: calls that overlap on
+ *  the GPU (other streams, other host threads) race on it and must not be
+ *  issued.  The first call on each device resolves the array's address
+ *  (a host-side runtime query); make that first call before beginning any
+ *  stream capture on that device.
+ * Errors: as moe_expert_forward; QK_ERR_WORKSPACE when the fixed array is too
+ * small.
+ * ---------------------------------------------------------------------- */
+qk_status moe_expert_forward_noalloc(const qk_moe_layer* L, const void* x_bf16, int32_t n_tokens,
+                                     const int32_t* topk_ids, const float* topk_w, int32_t top_k,
+                                     void* y, int32_t y_is_bf16, qk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * moe_route_topk -- router: softmax over E logits, the top_k largest
  * (equal values: lower expert id first), renormalised to sum 1, in
  * descending order.  Only the top_k logits enter the weights:

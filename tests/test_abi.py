@@ -21,7 +21,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = qk.load()
     names = _declared()
-    assert len(names) == 10
+    assert len(names) == 11
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(_lib.SYMBOLS)
@@ -81,6 +81,17 @@ def test_forward_argument_errors_are_synchronous():
     assert L.fp8_shared_expert_workspace_size(8, 4096, 2048) > 0
     assert L.fp8_shared_expert_forward(p, 8, 4096, 2048, p, p, p, p, p, p, p, p, 0, None) == \
         qk.QK_ERR_WORKSPACE
+
+
+def test_noalloc_entry_rejects_before_any_device_work():
+    L = qk.load()
+    lay = _fake_layer()
+    p = ctypes.c_void_p(1 << 24)
+    f = L.moe_expert_forward_noalloc
+    assert f(ctypes.byref(lay), p, 0, p, p, 6, p, 0, None) == qk.QK_OK                # T = 0
+    assert f(ctypes.byref(lay), p, 16, p, p, 6, p, 0, None) == qk.QK_ERR_WORKSPACE    # > 4 MiB
+    assert f(ctypes.byref(lay), p, 1, p, p, 9, p, 0, None) == qk.QK_ERR_INVALID_ARG   # top_k > 8
+    assert f(None, p, 1, p, p, 6, p, 0, None) == qk.QK_ERR_INVALID_ARG
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
