@@ -32,13 +32,15 @@ static qk_status layer_ok(const qk_moe_layer* L) {
 
 extern "C" {
 
-// Tokens per decode launch: the routing tables of one launch hold kMaxPairs pairs.
+// Tokens per decode launch: the routing tables of one launch hold kMaxPairs
+// pairs; more tokens take the grouped path.
 static int decode_chunk(int top_k) { return kMaxPairs / top_k; }
 
 size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_t top_k) {
   if (layer_ok(L) != QK_OK || n_tokens < 0 || top_k < 1 || top_k > 8) return 0;
-  const int t = n_tokens < decode_chunk(top_k) ? n_tokens : decode_chunk(top_k);
-  return decode_workspace_bytes(t, top_k, L->hidden, L->inter);
+  if (n_tokens > decode_chunk(top_k))
+    return group_workspace_bytes(n_tokens, top_k, L->gate.n_experts, L->hidden, L->inter);
+  return decode_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
 }
 
 qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t n_tokens,
@@ -54,22 +56,6 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
   const size_t need = moe_expert_workspace_size(L, n_tokens, top_k);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return QK_ERR_WORKSPACE;
-  // Token counts above one launch's routing capacity run as consecutive
-  // launches over slices of the tokens (same stream, same workspace).
-  const int chunk = decode_chunk(top_k);
-  if (n_tokens > chunk) {
-    const uint16_t* xb = static_cast<const uint16_t*>(x_bf16);
-    const size_t ysz = y_is_bf16 ? 2 : 4;
-    for (int t0 = 0; t0 < n_tokens; t0 += chunk) {
-      const int tn = n_tokens - t0 < chunk ? n_tokens - t0 : chunk;
-      const qk_status rc = moe_expert_forward(
-          L, xb + (size_t)t0 * L->hidden, tn, topk_ids + (size_t)t0 * top_k, topk_w + (size_t)t0 * top_k,
-          top_k, static_cast<uint8_t*>(y) + (size_t)t0 * L->hidden * ysz, y_is_bf16, act_quant, workspace,
-          workspace_bytes, stream);
-      if (rc != QK_OK) return rc;
-    }
-    return QK_OK;
-  }
   DecodeArgs a = {};
   a.gate = L->gate;
   a.up = L->up;
@@ -85,6 +71,8 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
   a.I = L->inter;
   a.P = n_tokens * top_k;
   a.y_bf16 = y_is_bf16 ? 1 : 0;
+  // Token counts above one decode launch's routing capacity take the grouped path.
+  if (n_tokens > decode_chunk(top_k)) return group_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
   decode_carve(a, workspace);
   return decode_forward(a, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -1,0 +1,696 @@
+// qk_group.cu -- grouped (prefill) path of moe_expert_forward.
+//
+// For token counts where every routed expert sees many tokens, weights are
+// read once per group of tokens instead of once per token tile: the
+// (token, slot) pairs are grouped by expert ("DeepSeekv4 Flash for 1x Spark
+// [REAP25]", "What's actually different": one grouped GEMM per projection),
+// and each projection runs as a grouped GEMM on the 5th-generation tensor
+// cores.
+//
+//   k_grp_count / k_grp_scan / k_grp_scatter
+//       counting sort of the pairs by expert; x rows gathered into expert
+//       order as f16 scaled by a power of two per row (row maximum in
+//       [2^14, 2^15)); the list of token tiles (<= 256 rows of one expert).
+//   k_ggemm<gate/up>  per (token tile, 64 gate + 64 up weight rows):
+//       D[128 x n] = A . B^T on tcgen05 (kind::f16, fp32 accumulator in TMEM);
+//       A = the weight rows dequantized on chip to f16 (interleaved gate/up
+//       rows), B = the token tile; epilogue h = silu(g) * u (fp32).
+//   k_grp_h16         h rows -> f16 with a power-of-two shift per row.
+//   k_ggemm<down>     per (token tile, 128 down rows): d (fp32).
+//   k_grp_combine     y[t] = sum_s w[t][s] d[pair(t, s)] in slot order.
+//
+// Dequantization to f16.  NVFP4: e2m1 x e4m3 is exact in f16 and scale_2 is
+// applied in the epilogue.  MXFP4: each weight row is scaled relative to
+// its largest e8m0 code c_ref, A = e2m1 * 2^(c - c_ref + 8) (exact in f16 for
+// c >= c_ref - 31; smaller blocks lose low bits or flush to 0), and the
+// epilogue multiplies the row by 2^(c_ref - 135).
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "qk_common.cuh"
+#include "qk_tmap.h"
+
+namespace qk {
+
+constexpr int kGM = 128;        // weight rows per tile (tcgen05 M)
+constexpr int kGN = 256;        // token rows per tile (largest tcgen05 N)
+constexpr int kGK = 64;         // reduction per stage (one 128-byte f16 row)
+constexpr int kGS = 3;          // stages
+constexpr int kGDW = 8;         // dequant / epilogue warps
+constexpr int kGThreads = (2 + kGDW) * 32;  // producer warp, MMA warp, dequant warps
+constexpr int kGNBox = 4;       // token-box heights 32, 64, 128, 256
+
+struct GroupWs {
+  int* counts;      // [E] pairs per expert
+  int* offsets;     // [E + 1] first sorted row of each expert
+  int* fill;        // [E] scatter cursors
+  int* tile_e;      // [F] expert of token tile f
+  int* tile_row0;   // [F] first sorted row of token tile f
+  int* tile_n;      // [F] rows in token tile f
+  int* n_tiles;     // [1] token tiles
+  int* inv;         // [P] pair -> sorted row
+  int* xshift;      // [P] per sorted row: x scaled by 2^-xshift
+  int* hshift;      // [P] per sorted row: h scaled by 2^-hshift
+  __half* xperm;    // [P][H] f16
+  float* hperm;     // [P][I] fp32
+  __half* h16;      // [P][I] f16
+  float* dperm;     // [P][H] fp32
+  unsigned long long* n_flush;  // [1] MXFP4 blocks flushed by the relative scaling
+  size_t zero_bytes;            // bytes zeroed from `counts` on every call
+};
+
+}  // namespace qk
+
+namespace qk {
+
+// ------------------------------------------------------- grouping kernels --
+__global__ void k_grp_count(const int32_t* __restrict__ ids, int P, int E, int* __restrict__ counts) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= P) return;
+  const int e = ids[p];
+  if (e < 0 || e >= E) {
+    set_status(QK_ERR_INVALID_ARG);
+    return;
+  }
+  atomicAdd(&counts[e], 1);
+}
+
+// One block: exclusive scans of the per-expert pair counts and token-tile
+// counts; writes the token-tile list.
+constexpr int kScanThreads = 1024;
+__global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, int E) {
+  __shared__ int s_pairs[kScanThreads / 32], s_tiles[kScanThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (E + kScanThreads - 1) / kScanThreads;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+  int np = 0, nt = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int c = W.counts[e];
+    np += c;
+    nt += (c + kGN - 1) / kGN;
+  }
+  int ip = np, it = nt;  // inclusive scans within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, ip, o), b = __shfl_up_sync(0xffffffffu, it, o);
+    if (lane >= o) {
+      ip += a;
+      it += b;
+    }
+  }
+  if (lane == 31) {
+    s_pairs[warp] = ip;
+    s_tiles[warp] = it;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int a = s_pairs[lane], b = s_tiles[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, a, o), y = __shfl_up_sync(0xffffffffu, b, o);
+      if (lane >= o) {
+        a += x;
+        b += y;
+      }
+    }
+    s_pairs[lane] = a;
+    s_tiles[lane] = b;
+  }
+  __syncthreads();
+  int row = ip - np + (warp ? s_pairs[warp - 1] : 0);
+  int tile = it - nt + (warp ? s_tiles[warp - 1] : 0);
+  for (int e = e0; e < e1; ++e) {
+    const int c = W.counts[e];
+    W.offsets[e] = row;
+    W.fill[e] = 0;
+    for (int r = 0; r < c; r += kGN, ++tile) {
+      W.tile_e[tile] = e;
+      W.tile_row0[tile] = row + r;
+      W.tile_n[tile] = min(kGN, c - r);
+    }
+    row += c;
+  }
+  if (tid == kScanThreads - 1) {
+    W.offsets[E] = row;
+    *W.n_tiles = tile;
+  }
+}
+
+// One block per token: the row maximum, then the row in f16 (scaled by
+// 2^-shift) at the sorted position of each of the token's pairs.
+constexpr int kRowThreads = 128;
+__device__ __forceinline__ int block_shift(float m, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  float r = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
+  __syncthreads();
+  return clamp_shift(f16_shift_for(r));
+}
+
+__global__ void __launch_bounds__(kRowThreads) k_grp_scatter(GroupWs W, const uint16_t* __restrict__ x,
+                                                             const int32_t* __restrict__ ids, int k, int E,
+                                                             int H) {
+  __shared__ float red[kRowThreads / 32];
+  __shared__ int pos[8];
+  const int t = blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+  const int nv = H / 8;
+  float m = 0.f;
+  for (int j = threadIdx.x; j < nv; j += kRowThreads) {
+    const uint4 v = __ldg(src + j);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(wv[q] & 0xFFFFu)), fabsf(bf16_bits_to_f32(wv[q] >> 16))));
+  }
+  const int shift = block_shift(m, red);
+  if (threadIdx.x < k) {
+    const int p = t * k + threadIdx.x;
+    const int e = ids[p];
+    int r = -1;
+    if (e >= 0 && e < E) {
+      r = W.offsets[e] + atomicAdd(&W.fill[e], 1);
+      W.xshift[r] = shift;
+    }
+    W.inv[p] = r;
+    pos[threadIdx.x] = r;
+  }
+  __syncthreads();
+  const float sc = pow2f(-shift);
+  for (int j = threadIdx.x; j < nv; j += kRowThreads) {
+    const uint4 v = __ldg(src + j);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      o[q] = pack_f16x2(bf16_bits_to_f32(wv[q] & 0xFFFFu) * sc, bf16_bits_to_f32(wv[q] >> 16) * sc);
+    for (int s = 0; s < k; ++s)
+      if (pos[s] >= 0) reinterpret_cast<uint4*>(W.xperm + (size_t)pos[s] * H)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// One block per sorted row: h (fp32) -> f16 with its own power-of-two shift.
+__global__ void __launch_bounds__(kRowThreads) k_grp_h16(GroupWs W, int E, int I) {
+  __shared__ float red[kRowThreads / 32];
+  const int r = blockIdx.x;
+  if (r >= W.offsets[E]) return;  // block-uniform
+  const float4* src = reinterpret_cast<const float4*>(W.hperm + (size_t)r * I);
+  const int nv = I / 4;
+  float m = 0.f;
+  for (int j = threadIdx.x; j < nv; j += kRowThreads) {
+    const float4 v = __ldcg(src + j);
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+  const int shift = block_shift(m, red);
+  if (threadIdx.x == 0) W.hshift[r] = shift;
+  const float sc = pow2f(-shift);
+  for (int j = threadIdx.x; j < nv; j += kRowThreads) {
+    const float4 v = __ldcg(src + j);
+    reinterpret_cast<uint2*>(W.h16 + (size_t)r * I)[j] =
+        make_uint2(pack_f16x2(v.x * sc, v.y * sc), pack_f16x2(v.z * sc, v.w * sc));
+  }
+}
+
+// One block per token: y[t] = sum_s w[t][s] d[pair (t, s)], slots in order.
+__global__ void __launch_bounds__(256) k_grp_combine(GroupWs W, const float* __restrict__ w, int k, int H,
+                                                     void* y, int y_bf16) {
+  const int t = blockIdx.x;
+  int pos[8];
+  float ws[8];
+  for (int s = 0; s < k; ++s) {
+    pos[s] = W.inv[t * k + s];
+    ws[s] = w[t * k + s];
+  }
+  for (int j = threadIdx.x; j < H / 4; j += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < k; ++s) {
+      if (pos[s] < 0) continue;
+      const float4 d = __ldcg(reinterpret_cast<const float4*>(W.dperm + (size_t)pos[s] * H) + j);
+      acc.x = fmaf(ws[s], d.x, acc.x);
+      acc.y = fmaf(ws[s], d.y, acc.y);
+      acc.z = fmaf(ws[s], d.z, acc.z);
+      acc.w = fmaf(ws[s], d.w, acc.w);
+    }
+    if (y_bf16) {
+      __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y) + (size_t)t * H + 4 * j;
+      yb[0] = __float2bfloat16_rn(acc.x);
+      yb[1] = __float2bfloat16_rn(acc.y);
+      yb[2] = __float2bfloat16_rn(acc.z);
+      yb[3] = __float2bfloat16_rn(acc.w);
+    } else {
+      reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + (size_t)t * H)[j] = acc;
+    }
+  }
+}
+
+}  // namespace qk
+
+namespace qk {
+
+// ------------------------------------------------------ the grouped GEMM --
+struct GemmArgs {
+  GroupWs W;
+  qk_weight A, B;      // gate/up phase: gate, up; down phase: down, down
+  int E, K;            // experts, reduction length
+  int rows_per_e;      // weight rows of one expert (gate/up: inter; down: hidden)
+  int MB;              // weight-row tiles per expert (gate/up: inter/64; down: hidden/128)
+  int out_ld;          // output row length (gate/up: inter; down: hidden)
+  int sc_stride;       // bytes per row of the staged tile scales
+  alignas(64) CUtensorMap tqa, tqb;    // packed rows, 2-D bytes {K/2, rows}, box {32, 64}
+  alignas(64) CUtensorMap tb[kGNBox];  // token rows, f16 {K, P}, box {64, 32 << i}, 128-byte swizzle
+};
+
+struct GHead {
+  alignas(8) uint64_t full[kGS];   // packed rows + token rows landed (TMA)
+  alignas(8) uint64_t aready[kGS]; // f16 weight tile written (dequant warps)
+  alignas(8) uint64_t empty[kGS];  // the stage's MMAs completed
+  alignas(8) uint64_t acc_full;    // the tile's accumulator complete
+  alignas(8) uint64_t acc_empty;   // the accumulator read out
+  alignas(8) uint64_t drained;     // every MMA of the block completed (exit)
+  alignas(8) uint64_t cref_full;   // the tile's per-row reference codes written
+  uint32_t tmem;
+  int abort;                       // a wait ran out: every role stops
+  int cref[2][kGM];                // per tile row, by tile parity: largest e8m0 code of the row
+};
+
+constexpr int kGStageA = kGM * kGK * 2;   // 16 KB f16 weight tile
+constexpr int kGStageB = kGN * kGK * 2;   // 32 KB token tile
+constexpr int kGStageR = kGM * kGK / 2;   // 4 KB packed weight rows
+constexpr int kGTmemCols = kGN;
+
+__host__ __device__ inline int g_smem_bytes(int sc_stride) {
+  return 1024 + kGS * (kGStageA + kGStageB + kGStageR) + kGM * sc_stride + (int)sizeof(GHead);
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ int box_index(int n) { return n <= 32 ? 0 : n <= 64 ? 1 : n <= 128 ? 2 : 3; }
+
+// f16x2 broadcast of 2^e (0 below the smallest f16 subnormal).
+__device__ __forceinline__ uint32_t f16x2_pow2(int e) {
+  uint32_t b = 0;
+  if (e >= -14) b = (uint32_t)(e + 15) << 10;
+  else if (e >= -24) b = 1u << (e + 24);
+  return b | (b << 16);
+}
+
+template <int FA, int FB, bool GATEUP>
+__global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ GemmArgs G) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sA = base;
+  uint8_t* sB = sA + kGS * kGStageA;
+  uint8_t* sR = sB + kGS * kGStageB;
+  uint8_t* sS = sR + kGS * kGStageR;
+  GHead& S = *reinterpret_cast<GHead*>(sS + kGM * G.sc_stride);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const GroupWs& W = G.W;
+  const int MB = G.MB, nks = G.K / kGK;
+  const unsigned long long limit = g_wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGS; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.aready[s], kGDW);
+      mbar_init(&S.empty[s], 1);
+    }
+    mbar_init(&S.acc_full, 1);
+    mbar_init(&S.acc_empty, kGDW);
+    mbar_init(&S.drained, 1);
+    mbar_init(&S.cref_full, kGDW);
+    S.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&S.tmem, kGTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem;
+  const int n_tiles = *W.n_tiles * MB;
+  // Bounded wait; the first one that runs out stops every role of the block.
+  auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (*reinterpret_cast<volatile int*>(&S.abort)) return false;
+    if (mbar_wait_bounded(bar, parity, limit)) return true;
+    set_status(QK_ERR_TIMEOUT);
+    *reinterpret_cast<volatile int*>(&S.abort) = 1;
+    return false;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      const uint64_t pw = policy_evict_first(), px = policy_evict_last();
+      int n = 0;
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+        const int f = t / MB, mb = t - f * MB;
+        const int e = W.tile_e[f], row0 = W.tile_row0[f];
+        const int bi = box_index(W.tile_n[f]);
+        const uint32_t bbytes = (uint32_t)(32 << bi) * kGK * 2;
+        const int wrow = e * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128);
+        for (int ks = 0; ks < nks; ++ks, ++n) {
+          const int s = n % kGS;
+          if (n >= kGS && !wait(&S.empty[s], (uint32_t)((n / kGS - 1) & 1))) break;
+          mbar_arrive_expect_tx(&S.full[s], (uint32_t)kGStageR + bbytes);
+          uint8_t* r = sR + s * kGStageR;
+          tma_load_2d(r, &G.tqa, ks * (kGK / 2), wrow, &S.full[s], pw);
+          tma_load_2d(r + kGStageR / 2, GATEUP ? &G.tqb : &G.tqa, ks * (kGK / 2), GATEUP ? wrow : wrow + 64,
+                      &S.full[s], pw);
+          tma_load_2d(sB + s * kGStageB, &G.tb[bi], ks * kGK, row0, &S.full[s], px);
+        }
+        if (*reinterpret_cast<volatile int*>(&S.abort)) break;
+      }
+      // nothing may still be landing when the block exits
+      for (int q = n > kGS ? n - kGS : 0; q < n; ++q)
+        if (!mbar_wait_bounded(&S.full[q % kGS], (uint32_t)((q / kGS) & 1), kDrainLimitNs)) break;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA --
+    if (lane == 0) {
+      int n = 0, i = 0;
+      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+        const int f = t / MB;
+        const int nbox = 32 << box_index(W.tile_n[f]);
+        const uint32_t idesc = umma_idesc_f16(kGM, nbox);
+        if (i > 0 && !wait(&S.acc_empty, (uint32_t)((i - 1) & 1))) break;
+        tc_fence_after();
+        for (int ks = 0; ks < nks; ++ks, ++n) {
+          const int s = n % kGS;
+          const uint32_t ph = (uint32_t)((n / kGS) & 1);
+          if (!wait(&S.aready[s], ph) || !wait(&S.full[s], ph)) break;
+          tc_fence_after();
+          const uint64_t da = umma_desc_k_sw128(sA + s * kGStageA);
+          const uint64_t db = umma_desc_k_sw128(sB + s * kGStageB);
+#pragma unroll
+          for (int kk = 0; kk < kGK / 16; ++kk)  // 16 elements = 32 bytes = 2 descriptor units
+            umma_f16(tmem, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0 ? 1u : 0u);
+          umma_commit(&S.empty[s]);
+        }
+        if (*reinterpret_cast<volatile int*>(&S.abort)) break;
+        umma_commit(&S.acc_full);
+      }
+      // every MMA issued here completes before the accumulator is freed
+      umma_commit(&S.drained);
+      mbar_wait_bounded(&S.drained, 0, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------- dequant and epilogue --
+    const int dt = threadIdx.x - 64;  // 0 .. 255
+    const int r = dt >> 1, hh = dt & 1;
+    // GATEUP: tile row r = gate row r/2 (even r) or up row r/2 (odd r)
+    const bool rowB = GATEUP && (r & 1);
+    const int fr = rowB ? FB : FA;
+    const qk_weight& WR = rowB ? G.B : G.A;
+    const int wr_in_tile = GATEUP ? (r >> 1) : r;
+    const int sc_len = fr == QK_FMT_MXFP4 ? G.K / 32 : G.K / 16;
+    int n = 0, i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      const int f = t / MB, mb = t - f * MB;
+      const int e = W.tile_e[f], row0 = W.tile_row0[f], nrow = W.tile_n[f];
+      const int wrow = e * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128) + wr_in_tile;
+      // ---- the tile's scale rows, and (MXFP4) their largest code
+      uint8_t* srow = sS + r * G.sc_stride;
+      const uint8_t* gsrc = WR.scales + (size_t)wrow * sc_len;
+      uint32_t m4 = 0, ff = 0;  // byte-wise maxima; any 0xFF code
+      if (sc_len % 32 == 0) {    // two threads per row, 16-byte pieces
+        for (int b = hh * 16; b < sc_len; b += 32) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(gsrc + b));
+          *reinterpret_cast<uint4*>(srow + b) = v;
+          m4 = __vmaxu4(m4, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
+          ff |= __vcmpeq4(v.x, 0xFFFFFFFFu) | __vcmpeq4(v.y, 0xFFFFFFFFu) | __vcmpeq4(v.z, 0xFFFFFFFFu) |
+                __vcmpeq4(v.w, 0xFFFFFFFFu);
+        }
+      } else {
+        for (int b = hh; b < sc_len; b += 2) {
+          const uint32_t c = gsrc[b];
+          srow[b] = (uint8_t)c;
+          m4 = max(m4, c);
+          ff |= c == 255u ? 1u : 0u;
+        }
+      }
+      int cmax = (int)max(max(m4 & 0xFFu, (m4 >> 8) & 0xFFu), max((m4 >> 16) & 0xFFu, m4 >> 24));
+      if (fr == QK_FMT_MXFP4 && ff) set_status(QK_ERR_NAN_SCALE);
+      cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));  // the row's two halves
+      const int cref = fr == QK_FMT_MXFP4 ? min(cmax, 254) : 0;  // MXFP4 rows: relative to the row's max
+      if (hh == 0) S.cref[i & 1][r] = cref;
+      __syncwarp();
+      if (lane == 0) mbar_arrive_one(&S.cref_full);
+      // ---- dequantize every stage of the tile
+      for (int ks = 0; ks < nks; ++ks, ++n) {
+        const int s = n % kGS;
+        if (!__all_sync(0xffffffffu, wait(&S.full[s], (uint32_t)((n / kGS) & 1)))) break;
+        const uint8_t* raw = sR + s * kGStageR + (GATEUP ? (rowB ? kGStageR / 2 : 0) + (r >> 1) * 32 : r * 32) + hh * 16;
+        const uint4 q = *reinterpret_cast<const uint4*>(raw);
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+        uint32_t h2[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          h2[4 * j + 0] = e2m1x2_to_f16x2<0>(qw[j]);
+          h2[4 * j + 1] = e2m1x2_to_f16x2<1>(qw[j]);
+          h2[4 * j + 2] = e2m1x2_to_f16x2<2>(qw[j]);
+          h2[4 * j + 3] = e2m1x2_to_f16x2<3>(qw[j]);
+        }
+        if (fr == QK_FMT_MXFP4) {  // one 32-block: e2m1 * 2^(c - cref + 8)
+          const int c = srow[ks * 2 + hh];
+          const uint32_t sc = f16x2_pow2(c - cref + 8);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            uint32_t d;
+            asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h2[j]), "r"(sc));
+            h2[j] = d;
+          }
+        } else {  // two 16-blocks: e2m1 * e4m3
+          const uint32_t c2 = (uint32_t)srow[ks * 4 + 2 * hh] | ((uint32_t)srow[ks * 4 + 2 * hh + 1] << 8);
+          const uint32_t s01 = e4m3x2_to_f16x2<0>(c2);
+          const uint32_t s0 = __byte_perm(s01, s01, 0x1010), s1 = __byte_perm(s01, s01, 0x3232);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            uint32_t d;
+            asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h2[j]), "r"(j < 8 ? s0 : s1));
+            h2[j] = d;
+          }
+        }
+        uint8_t* arow = sA + s * kGStageA + r * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = 4 * hh + j;
+          *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) =
+              make_uint4(h2[4 * j], h2[4 * j + 1], h2[4 * j + 2], h2[4 * j + 3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_one(&S.aready[s]);
+      }
+      // ---- epilogue: TMEM -> registers -> h (gate/up) or d (down)
+      if (!__all_sync(0xffffffffu, wait(&S.acc_full, (uint32_t)(i & 1)) && wait(&S.cref_full, (uint32_t)(i & 1))))
+        break;
+      tc_fence_after();
+      const int quad = warp & 3;              // TMEM lanes 32 quad .. 32 quad + 31
+      const int chalf = (warp - 2) >> 2;      // which half of the columns
+      const int nbox = 32 << box_index(nrow);
+      const int c_lo = nbox == 32 ? (chalf ? nbox : 0) : chalf * (nbox / 2);
+      const int c_hi = nbox == 32 ? (chalf ? nbox : nbox) : c_lo + nbox / 2;
+      const int feat = quad * 32 + lane;       // tile row of this thread
+      // this thread's tile row: MXFP4 rows were scaled by 2^(135 - cref) on chip
+      const bool frow_b = GATEUP && (feat & 1);
+      const int frow_fmt = frow_b ? FB : FA;
+      const float post = frow_fmt == QK_FMT_MXFP4 ? ldexpf(1.f, S.cref[i & 1][feat] - 135)
+                                                  : (frow_b ? G.B.scale_2[e] : G.A.scale_2[e]);
+      for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+        if (GATEUP) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float mine = __uint_as_float(v[j]) * post;
+            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+            const int col = c0 + j;
+            if (!(lane & 1) && col < nrow) {
+              const int row = row0 + col;
+              const float sx = pow2f(W.xshift[row]);
+              const float g = mine * sx, u = other * sx;
+              W.hperm[(size_t)row * G.out_ld + mb * 64 + (feat >> 1)] = silu_mul(g, u);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int col = c0 + j;
+            if (col < nrow) {
+              const int row = row0 + col;
+              W.dperm[(size_t)row * G.out_ld + mb * 128 + feat] =
+                  __uint_as_float(v[j]) * post * pow2f(W.hshift[row]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_one(&S.acc_empty);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_free(tmem, kGTmemCols);
+  }
+}
+
+}  // namespace qk
+
+namespace qk {
+
+// ================================================================= host ==
+struct GWsLayout {
+  size_t counts, offsets, fill, tile_e, tile_row0, tile_n, n_tiles, n_flush, zero_end;
+  size_t inv, xshift, hshift, xperm, hperm, h16, dperm, total;
+};
+
+static int g_max_tiles(int P, int E) { return P / kGN + E + 1; }
+
+static GWsLayout g_layout(int T, int k, int E, int H, int I) {
+  const size_t P = (size_t)T * k, F = (size_t)g_max_tiles((int)P, E);
+  GWsLayout L;
+  size_t o = 0;
+  L.counts = o; o += (size_t)E * 4;          // zeroed on every call: counts .. n_flush
+  L.n_tiles = o; o += 8;
+  L.n_flush = o; o += 8;
+  L.zero_end = o;
+  o = align256(o);
+  L.offsets = o; o += align256((size_t)(E + 1) * 4);
+  L.fill = o; o += align256((size_t)E * 4);
+  L.tile_e = o; o += align256(F * 4);
+  L.tile_row0 = o; o += align256(F * 4);
+  L.tile_n = o; o += align256(F * 4);
+  L.inv = o; o += align256(P * 4);
+  L.xshift = o; o += align256(P * 4);
+  L.hshift = o; o += align256(P * 4);
+  L.xperm = o; o += align256(P * H * 2);
+  L.hperm = o; o += align256(P * I * 4);
+  L.h16 = o; o += align256(P * I * 2);
+  L.dperm = o; o += align256(P * H * 4);
+  L.total = o;
+  return L;
+}
+
+size_t group_workspace_bytes(int T, int k, int E, int H, int I) { return g_layout(T, k, E, H, I).total; }
+
+static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I) {
+  const GWsLayout L = g_layout(T, k, E, H, I);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  GroupWs W;
+  W.counts = reinterpret_cast<int*>(p + L.counts);
+  W.n_tiles = reinterpret_cast<int*>(p + L.n_tiles);
+  W.n_flush = reinterpret_cast<unsigned long long*>(p + L.n_flush);
+  W.zero_bytes = L.zero_end - L.counts;
+  W.offsets = reinterpret_cast<int*>(p + L.offsets);
+  W.fill = reinterpret_cast<int*>(p + L.fill);
+  W.tile_e = reinterpret_cast<int*>(p + L.tile_e);
+  W.tile_row0 = reinterpret_cast<int*>(p + L.tile_row0);
+  W.tile_n = reinterpret_cast<int*>(p + L.tile_n);
+  W.inv = reinterpret_cast<int*>(p + L.inv);
+  W.xshift = reinterpret_cast<int*>(p + L.xshift);
+  W.hshift = reinterpret_cast<int*>(p + L.hshift);
+  W.xperm = reinterpret_cast<__half*>(p + L.xperm);
+  W.hperm = reinterpret_cast<float*>(p + L.hperm);
+  W.h16 = reinterpret_cast<__half*>(p + L.h16);
+  W.dperm = reinterpret_cast<float*>(p + L.dperm);
+  return W;
+}
+
+// Packed rows [rows][K/2] bytes, boxes {32 bytes, 64 rows}.
+static bool g_map_packed(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
+  const uint64_t dims[2] = {(uint64_t)K / 2, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)K / 2};
+  const uint32_t box[2] = {(uint32_t)kGK / 2, 64};
+  return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Token rows [P][K] f16, boxes {64 elements, 32 << i rows}, 128-byte swizzle.
+static bool g_map_tokens(CUtensorMap (&m)[kGNBox], const __half* x, int64_t P, int K) {
+  const uint64_t dims[2] = {(uint64_t)K, (uint64_t)P};
+  const uint64_t strides[1] = {(uint64_t)K * 2};
+  for (int i = 0; i < kGNBox; ++i) {
+    const uint32_t box[2] = {(uint32_t)kGK, (uint32_t)(32 << i)};
+    if (!tmap_get(&m[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  }
+  return true;
+}
+
+template <int FA, int FB, bool GATEUP>
+static qk_status g_launch(const GemmArgs& A, cudaStream_t st) {
+  auto kern = k_ggemm<FA, FB, GATEUP>;
+  const int smem = g_smem_bytes(A.sc_stride);
+  if (smem > max_smem_optin()) return QK_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return QK_ERR_CUDA;
+  kern<<<num_sms(), kGThreads, smem, st>>>(A);
+  return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+}
+
+template <bool GATEUP>
+static qk_status g_dispatch(const GemmArgs& A, cudaStream_t st) {
+  constexpr int MX = QK_FMT_MXFP4, NV = QK_FMT_NVFP4;
+  const int fa = A.A.fmt, fb = A.B.fmt;
+  if (fa == MX && fb == MX) return g_launch<MX, MX, GATEUP>(A, st);
+  if (fa == MX) return g_launch<MX, NV, GATEUP>(A, st);
+  if (fb == MX) return g_launch<NV, MX, GATEUP>(A, st);
+  return g_launch<NV, NV, GATEUP>(A, st);
+}
+
+qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
+  const int T = a.T, k = a.k, E = a.E, H = a.H, I = a.I, P = a.P;
+  GroupWs W = g_carve(workspace, T, k, E, H, I);
+  if (cudaMemsetAsync(W.counts, 0, W.zero_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
+  k_grp_count<<<(P + 255) / 256, 256, 0, st>>>(a.ids, P, E, W.counts);
+  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, E);
+  k_grp_scatter<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H);
+  if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
+
+  GemmArgs g1 = {};
+  g1.W = W;
+  g1.A = a.gate;
+  g1.B = a.up;
+  g1.E = E;
+  g1.K = H;
+  g1.rows_per_e = I;
+  g1.MB = I / 64;
+  g1.out_ld = I;
+  g1.sc_stride = (a.gate.fmt == QK_FMT_NVFP4 || a.up.fmt == QK_FMT_NVFP4) ? H / 16 : H / 32;
+  if (!g_map_packed(&g1.tqa, a.gate.q, (int64_t)E * I, H) || !g_map_packed(&g1.tqb, a.up.q, (int64_t)E * I, H) ||
+      !g_map_tokens(g1.tb, W.xperm, P, H))
+    return QK_ERR_CUDA;
+  qk_status rc = g_dispatch<true>(g1, st);
+  if (rc != QK_OK) return rc;
+
+  k_grp_h16<<<P, kRowThreads, 0, st>>>(W, E, I);
+  GemmArgs g2 = {};
+  g2.W = W;
+  g2.A = a.down;
+  g2.B = a.down;
+  g2.E = E;
+  g2.K = I;
+  g2.rows_per_e = H;
+  g2.MB = H / 128;
+  g2.out_ld = H;
+  g2.sc_stride = a.down.fmt == QK_FMT_NVFP4 ? I / 16 : I / 32;
+  if (!g_map_packed(&g2.tqa, a.down.q, (int64_t)E * H, I) || !g_map_tokens(g2.tb, W.h16, P, I)) return QK_ERR_CUDA;
+  g2.tqb = g2.tqa;
+  rc = g_dispatch<false>(g2, st);
+  if (rc != QK_OK) return rc;
+  k_grp_combine<<<T, 256, 0, st>>>(W, a.w, k, H, a.y, a.y_bf16);
+  return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+}
+
+}  // namespace qk
