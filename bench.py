@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--cpu-sample-s", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=150.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=20,
+                    help="timed repetitions of the 2048-token prefill layer (0: skip)")
     return ap.parse_args()
 
 
@@ -343,7 +345,84 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 3 * K,
         "clocks": clocks.summary(),
     }
+    if args.prefill_steps > 0:
+        del layers, lays
+        torch.cuda.empty_cache()
+        out["prefill"] = run_prefill(args, rank, world, dev)
+        out["gpu_launches"] += 7 * args.prefill_steps
     return out
+
+
+def run_prefill(args, rank, world, dev):
+    """The 2048-token Zipf prefill layer through moe_expert_forward (grouped
+    path): tokens/s, HBM fraction on the touched experts' bytes, tensor rate."""
+    import torch
+    import torch.distributed as dist
+
+    import block_quantized_expert_mxfp4_b200 as qk
+    from block_quantized_expert_mxfp4_b200 import synth, workload
+
+    wl = synth.WORKLOADS["prefill"]
+    T, k = wl.T, wl.k
+    layer = workload.make_layer(wl, seed=rank, layer=0)
+    lay = layer.c()
+    x = synth.activations(rank, T, wl.H).to(dev)
+    lg = synth.zipf_logits(rank, T, wl.E, k).to(dev)
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    qk.moe_route_topk(lg, k, ids, w)
+    y = torch.empty((T, wl.H), dtype=torch.float32, device=dev)
+    wsp = torch.empty(qk.moe_expert_workspace_size(lay, T, k), dtype=torch.uint8, device=dev)
+    touched = int(torch.unique(ids).numel())
+    wbytes = touched * layer.expert_bytes()
+    flops = 2 * 3 * wl.H * wl.I * T * k
+    s = torch.cuda.Stream(device=dev)
+    for _ in range(3):
+        qk.moe_expert_forward(lay, x, ids, w, y, wsp)
+    torch.cuda.synchronize()
+    if qk.qk_last_device_status() != qk.QK_OK:
+        raise RuntimeError("device status after prefill warm-up")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            qk.moe_expert_forward(lay, x, ids, w, y, wsp, stream=s)
+    torch.cuda.synchronize()
+    K = args.prefill_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(s)
+        for _ in range(K):
+            g.replay()
+        e1.record(s)
+        torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1) / 1e3 / K], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t = float(t.item())
+    if qk.qk_last_device_status() != qk.QK_OK:
+        raise RuntimeError("device status after prefill")
+    peak, peak_kind = peaks()
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tpeak, tkind = float(json.load(f)["bf16_tflops"]), "measured (bf16; f16 runs at the same rate)"
+    except Exception:
+        tpeak, tkind = 1590.0, "fallback"
+    return {
+        "workload": "prefill MoE layer: 2048 tokens, 256 experts, top-6 Zipf(s=1) routing, hidden 4096, "
+                    "intermediate 2048, MXFP4 gate/up/down, bf16 N(0,1) activations",
+        "tokens_per_s": round(T * world / t, 1), "ms_per_layer": round(t * 1e3, 4), "steps": K,
+        "experts_touched": touched,
+        "hbm": {"bytes_per_layer": wbytes, "achieved_gbs": round(wbytes / t / 1e9, 1), "peak_gbs": peak,
+                "peak_kind": peak_kind, "frac": round(wbytes / t / 1e9 / peak, 4)},
+        "tensor": {"flop_per_layer": flops, "achieved_tflops": round(flops / t / 1e12, 1),
+                   "peak_tflops": tpeak, "peak_kind": tkind, "frac": round(flops / t / 1e12 / tpeak, 4)},
+        "path": "group/permute, tcgen05 kind::f16 grouped GEMMs (gate/up+SwiGLU, down), combine",
+    }
 
 
 def main():

@@ -15,10 +15,10 @@ from helpers import MX, NV, assert_parity, oracle_moe
 pytestmark = pytest.mark.gpu
 
 
-def _forward(layer, x, ids, w):
+def _forward(layer, x, ids, w, y_dtype=torch.float32):
     lay = layer.c()
     T, k = ids.shape
-    y = torch.full((T, x.shape[1]), float("nan"), dtype=torch.float32, device="cuda")
+    y = torch.full((T, x.shape[1]), float("nan"), dtype=y_dtype, device="cuda")
     ws = torch.empty(qk.moe_expert_workspace_size(lay, T, k), dtype=torch.uint8, device="cuda")
     qk.moe_expert_forward(lay, x, ids, w, y, ws)
     assert qk.qk_last_device_status() == qk.QK_OK
@@ -70,3 +70,31 @@ def test_prefill_zipf_sampled_tokens():
     pick = sorted(pick)
     yo = oracle_moe(wl, 0, 0, x[pick], oids[pick], ow[pick].astype(np.float32).astype(np.float64))
     assert_parity(y.cpu().numpy()[pick], yo, what="prefill sampled tokens")
+
+
+@pytest.mark.parametrize("fmts", [(NV, NV, NV), (MX, NV, NV), (NV, MX, MX)])
+def test_grouped_path_formats(fmts):
+    """48 tokens x top-4 = 192 pairs (grouped path), NVFP4 and mixed projections."""
+    wl = synth.Workload("mid", 16, 4, 1024, 512, 48, 118, 127)
+    layer = workload.make_layer(wl, 5, 0, fmts)
+    x = synth.activations(5, wl.T, wl.H)
+    lg = synth.router_logits(5, wl.T, wl.E)
+    oids, ow = oracle.route_topk(lg, wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
+    yo = oracle_moe(wl, 5, 0, x, oids, ow.astype(np.float32).astype(np.float64), fmts)
+    assert_parity(y.cpu().numpy(), yo, what=f"grouped {fmts}")
+
+
+def test_grouped_path_bf16_output_and_skewed_groups():
+    """Tiny layer, 200 tokens all routed to experts 1 and 6 (groups of 200:
+    a full and a partial token tile each); bf16 y."""
+    wl = synth.WORKLOADS["tiny"]
+    layer = workload.make_layer(wl, 6, 0)
+    T = 200
+    x = synth.activations(6, T, wl.H)
+    ids = np.array([[1, 6]] * T, np.int32)
+    w = np.tile(np.array([[0.6, 0.4]]), (T, 1))
+    y = _forward(layer, x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).float().cuda(),
+                 torch.bfloat16)
+    yo = oracle_moe(wl, 6, 0, x, ids, w.astype(np.float32).astype(np.float64))
+    assert_parity(y.float().cpu().numpy(), yo, what="grouped bf16 y")
