@@ -36,9 +36,13 @@ namespace qk {
 constexpr int kGM = 128;        // weight rows per tile (tcgen05 M)
 constexpr int kGN = 256;        // token rows per tile (largest tcgen05 N)
 constexpr int kGK = 64;         // reduction per stage (one 128-byte f16 row)
-constexpr int kGS = 3;          // stages
+constexpr int kGRS = 3;         // packed-weight stages (16 KB: four reduction steps of 128 rows)
+constexpr int kGRK = 4;         // reduction steps per packed-weight stage
+constexpr int kGAS = 3;         // f16 weight-tile stages (16 KB)
+constexpr int kGBS = 3;         // token-tile stages (32 KB: 256 / n reduction steps of n tokens)
 constexpr int kGDW = 8;         // dequant / epilogue warps
-constexpr int kGThreads = (2 + kGDW) * 32;  // producer warp, MMA warp, dequant warps
+constexpr int kGEW = 4;         // epilogue warps (one per TMEM lane quadrant)
+constexpr int kGThreads = (3 + kGDW + kGEW) * 32;  // weight producer, MMA, token producer, dequant, epilogue
 constexpr int kGNBox = 4;       // token-box heights 32, 64, 128, 256
 
 struct GroupWs {
@@ -261,30 +265,33 @@ struct GemmArgs {
   int MB;              // weight-row tiles per expert (gate/up: inter/64; down: hidden/128)
   int out_ld;          // output row length (gate/up: inter; down: hidden)
   int sc_stride;       // bytes per row of the staged tile scales
-  alignas(64) CUtensorMap tqa, tqb;    // packed rows, 2-D bytes {K/2, rows}, box {32, 64}
+  alignas(64) CUtensorMap tqa, tqb;    // packed rows, 2-D bytes {K/2, rows}, box {128, 64}, 128B swizzle
   alignas(64) CUtensorMap tb[kGNBox];  // token rows, f16 {K, P}, box {64, 32 << i}, 128-byte swizzle
 };
 
 struct GHead {
-  alignas(8) uint64_t full[kGS];   // packed rows + token rows landed (TMA)
-  alignas(8) uint64_t aready[kGS]; // f16 weight tile written (dequant warps)
-  alignas(8) uint64_t empty[kGS];  // the stage's MMAs completed
-  alignas(8) uint64_t acc_full;    // the tile's accumulator complete
-  alignas(8) uint64_t acc_empty;   // the accumulator read out
-  alignas(8) uint64_t drained;     // every MMA of the block completed (exit)
-  alignas(8) uint64_t cref_full;   // the tile's per-row reference codes written
+  alignas(8) uint64_t rfull[kGRS];   // packed weight rows landed (TMA)
+  alignas(8) uint64_t rempty[kGRS];  // packed rows consumed (dequant warps)
+  alignas(8) uint64_t afull[kGAS];   // f16 weight tile written (dequant warps)
+  alignas(8) uint64_t aempty[kGAS];  // f16 weight tile's MMAs completed
+  alignas(8) uint64_t bfull[kGBS];   // token rows landed (TMA)
+  alignas(8) uint64_t bempty[kGBS];  // token stage's MMAs completed
+  alignas(8) uint64_t acc_full[2];   // accumulator buffer complete (by tile parity)
+  alignas(8) uint64_t acc_empty[2];  // accumulator buffer read out
+  alignas(8) uint64_t drained;       // every MMA of the block completed (exit)
+  alignas(8) uint64_t cref_full[4];  // the tile's per-row reference codes written (tile % 4)
   uint32_t tmem;
-  int abort;                       // a wait ran out: every role stops
-  int cref[2][kGM];                // per tile row, by tile parity: largest e8m0 code of the row
+  int abort;                         // a wait ran out: every role stops
+  int cref[4][kGM];                  // per tile row (tile % 4): largest e8m0 code of the row
 };
 
 constexpr int kGStageA = kGM * kGK * 2;   // 16 KB f16 weight tile
-constexpr int kGStageB = kGN * kGK * 2;   // 32 KB token tile
-constexpr int kGStageR = kGM * kGK / 2;   // 4 KB packed weight rows
-constexpr int kGTmemCols = kGN;
+constexpr int kGStageB = kGN * kGK * 2;   // 32 KB of token rows
+constexpr int kGStageR = kGM * kGK / 2 * kGRK;  // 16 KB packed weight rows (two 64-row boxes)
+constexpr int kGTmemCols = 2 * kGN;  // two accumulator buffers
 
 __host__ __device__ inline int g_smem_bytes(int sc_stride) {
-  return 1024 + kGS * (kGStageA + kGStageB + kGStageR) + kGM * sc_stride + (int)sizeof(GHead);
+  return 1024 + kGAS * kGStageA + kGBS * kGStageB + kGRS * kGStageR + kGM * sc_stride + (int)sizeof(GHead);
 }
 
 __device__ __forceinline__ uint64_t policy_evict_last() {
@@ -307,10 +314,10 @@ template <int FA, int FB, bool GATEUP>
 __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ GemmArgs G) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* sA = base;
-  uint8_t* sB = sA + kGS * kGStageA;
-  uint8_t* sR = sB + kGS * kGStageB;
-  uint8_t* sS = sR + kGS * kGStageR;
+  uint8_t* sA = base;                      // kGAS f16 weight tiles (1024-aligned)
+  uint8_t* sB = sA + kGAS * kGStageA;      // kGBS token stages
+  uint8_t* sR = sB + kGBS * kGStageB;      // kGRS packed-row stages
+  uint8_t* sS = sR + kGRS * kGStageR;      // the tile's scale rows
   GHead& S = *reinterpret_cast<GHead*>(sS + kGM * G.sc_stride);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const GroupWs& W = G.W;
@@ -318,15 +325,24 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
   const unsigned long long limit = g_wait_limit_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kGS; ++s) {
-      mbar_init(&S.full[s], 1);
-      mbar_init(&S.aready[s], kGDW);
-      mbar_init(&S.empty[s], 1);
+    for (int s = 0; s < kGRS; ++s) {
+      mbar_init(&S.rfull[s], 1);
+      mbar_init(&S.rempty[s], kGDW);
     }
-    mbar_init(&S.acc_full, 1);
-    mbar_init(&S.acc_empty, kGDW);
+    for (int s = 0; s < kGAS; ++s) {
+      mbar_init(&S.afull[s], kGDW);
+      mbar_init(&S.aempty[s], 1);
+    }
+    for (int s = 0; s < kGBS; ++s) {
+      mbar_init(&S.bfull[s], 1);
+      mbar_init(&S.bempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.acc_full[b], 1);
+      mbar_init(&S.acc_empty[b], kGEW);
+    }
     mbar_init(&S.drained, 1);
-    mbar_init(&S.cref_full, kGDW);
+    for (int b = 0; b < 4; ++b) mbar_init(&S.cref_full[b], kGDW);
     S.abort = 0;
     fence_mbar_init();
   }
@@ -344,68 +360,89 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
     *reinterpret_cast<volatile int*>(&S.abort) = 1;
     return false;
   };
+  auto aborted = [&]() { return *reinterpret_cast<volatile int*>(&S.abort) != 0; };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer --
-    if (lane == 0) {
-      const uint64_t pw = policy_evict_first(), px = policy_evict_last();
+  if (warp == 0 || warp == 2) {
+    // ----------------------------------------------------------- producers --
+    // warp 0: packed weight rows, kGRK reduction steps per stage (one 8 KB box
+    // per 64-row half); warp 2: token rows, 32 KB per stage (256 / n steps of
+    // an n-row tile).
+    if (warp == 0 && lane == 0) {
+      const uint64_t pw = policy_evict_first();
       int n = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+      for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x) {
         const int f = t / MB, mb = t - f * MB;
-        const int e = W.tile_e[f], row0 = W.tile_row0[f];
-        const int bi = box_index(W.tile_n[f]);
-        const uint32_t bbytes = (uint32_t)(32 << bi) * kGK * 2;
-        const int wrow = e * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128);
-        for (int ks = 0; ks < nks; ++ks, ++n) {
-          const int s = n % kGS;
-          if (n >= kGS && !wait(&S.empty[s], (uint32_t)((n / kGS - 1) & 1))) break;
-          mbar_arrive_expect_tx(&S.full[s], (uint32_t)kGStageR + bbytes);
+        const int wrow = W.tile_e[f] * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128);
+        for (int k0 = 0; k0 < nks; k0 += kGRK, ++n) {
+          const int s = n % kGRS;
+          if (n >= kGRS && !wait(&S.rempty[s], (uint32_t)((n / kGRS - 1) & 1))) break;
+          mbar_arrive_expect_tx(&S.rfull[s], (uint32_t)kGStageR);
           uint8_t* r = sR + s * kGStageR;
-          tma_load_2d(r, &G.tqa, ks * (kGK / 2), wrow, &S.full[s], pw);
-          tma_load_2d(r + kGStageR / 2, GATEUP ? &G.tqb : &G.tqa, ks * (kGK / 2), GATEUP ? wrow : wrow + 64,
-                      &S.full[s], pw);
-          tma_load_2d(sB + s * kGStageB, &G.tb[bi], ks * kGK, row0, &S.full[s], px);
+          tma_load_2d(r, &G.tqa, k0 * (kGK / 2), wrow, &S.rfull[s], pw);
+          tma_load_2d(r + kGStageR / 2, GATEUP ? &G.tqb : &G.tqa, k0 * (kGK / 2), GATEUP ? wrow : wrow + 64,
+                      &S.rfull[s], pw);
         }
-        if (*reinterpret_cast<volatile int*>(&S.abort)) break;
       }
-      // nothing may still be landing when the block exits
-      for (int q = n > kGS ? n - kGS : 0; q < n; ++q)
-        if (!mbar_wait_bounded(&S.full[q % kGS], (uint32_t)((q / kGS) & 1), kDrainLimitNs)) break;
+      for (int q = n > kGRS ? n - kGRS : 0; q < n; ++q)  // nothing may still be landing at exit
+        if (!mbar_wait_bounded(&S.rfull[q % kGRS], (uint32_t)((q / kGRS) & 1), kDrainLimitNs)) break;
+    } else if (warp == 2 && lane == 0) {
+      const uint64_t px = policy_evict_last();
+      int n = 0;
+      for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x) {
+        const int f = t / MB;
+        const int row0 = W.tile_row0[f], bi = box_index(W.tile_n[f]);
+        const int nbox = 32 << bi, kpb = kGN / nbox;  // reduction steps per token stage
+        for (int k0 = 0; k0 < nks; k0 += kpb, ++n) {
+          const int s = n % kGBS, nsub = min(kpb, nks - k0);
+          if (n >= kGBS && !wait(&S.bempty[s], (uint32_t)((n / kGBS - 1) & 1))) break;
+          mbar_arrive_expect_tx(&S.bfull[s], (uint32_t)(nsub * nbox * kGK * 2));
+          for (int j = 0; j < nsub; ++j)
+            tma_load_2d(sB + s * kGStageB + j * nbox * kGK * 2, &G.tb[bi], (k0 + j) * kGK, row0, &S.bfull[s], px);
+        }
+      }
+      for (int q = n > kGBS ? n - kGBS : 0; q < n; ++q)
+        if (!mbar_wait_bounded(&S.bfull[q % kGBS], (uint32_t)((q / kGBS) & 1), kDrainLimitNs)) break;
     }
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA --
     if (lane == 0) {
-      int n = 0, i = 0;
-      for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      int na = 0, nb = 0, i = 0;
+      for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x, ++i) {
         const int f = t / MB;
-        const int nbox = 32 << box_index(W.tile_n[f]);
+        const int nbox = 32 << box_index(W.tile_n[f]), kpb = kGN / nbox;
         const uint32_t idesc = umma_idesc_f16(kGM, nbox);
-        if (i > 0 && !wait(&S.acc_empty, (uint32_t)((i - 1) & 1))) break;
+        const int ab = i & 1;  // accumulator buffer
+        if (i >= 2 && !wait(&S.acc_empty[ab], (uint32_t)((i / 2 - 1) & 1))) break;
         tc_fence_after();
-        for (int ks = 0; ks < nks; ++ks, ++n) {
-          const int s = n % kGS;
-          const uint32_t ph = (uint32_t)((n / kGS) & 1);
-          if (!wait(&S.aready[s], ph) || !wait(&S.full[s], ph)) break;
-          tc_fence_after();
-          const uint64_t da = umma_desc_k_sw128(sA + s * kGStageA);
-          const uint64_t db = umma_desc_k_sw128(sB + s * kGStageB);
+        const uint32_t tacc = tmem + (uint32_t)(ab * kGN);
+        for (int k0 = 0; k0 < nks && !aborted(); k0 += kpb, ++nb) {
+          const int sb = nb % kGBS, nsub = min(kpb, nks - k0);
+          if (!wait(&S.bfull[sb], (uint32_t)((nb / kGBS) & 1))) break;
+          for (int j = 0; j < nsub; ++j, ++na) {
+            const int sa = na % kGAS;
+            if (!wait(&S.afull[sa], (uint32_t)((na / kGAS) & 1))) break;
+            tc_fence_after();
+            const uint64_t da = umma_desc_k_sw128(sA + sa * kGStageA);
+            const uint64_t db = umma_desc_k_sw128(sB + sb * kGStageB + j * nbox * kGK * 2);
 #pragma unroll
-          for (int kk = 0; kk < kGK / 16; ++kk)  // 16 elements = 32 bytes = 2 descriptor units
-            umma_f16(tmem, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0 ? 1u : 0u);
-          umma_commit(&S.empty[s]);
+            for (int kk = 0; kk < kGK / 16; ++kk)  // 16 elements = 32 bytes = 2 descriptor units
+              umma_f16(tacc, da + 2 * kk, db + 2 * kk, idesc, (k0 + j + kk) != 0 ? 1u : 0u);
+            umma_commit(&S.aempty[sa]);
+          }
+          umma_commit(&S.bempty[sb]);
         }
-        if (*reinterpret_cast<volatile int*>(&S.abort)) break;
-        umma_commit(&S.acc_full);
+        if (aborted()) break;
+        umma_commit(&S.acc_full[ab]);
       }
       // every MMA issued here completes before the accumulator is freed
       umma_commit(&S.drained);
       mbar_wait_bounded(&S.drained, 0, kDrainLimitNs);
     }
     __syncwarp();
-  } else {
-    // --------------------------------------------- dequant and epilogue --
-    const int dt = threadIdx.x - 64;  // 0 .. 255
+  } else if (warp < 3 + kGDW) {
+    // ------------------------------------------------------------ dequant --
+    const int dt = threadIdx.x - 96;  // 0 .. 255
     const int r = dt >> 1, hh = dt & 1;
     // GATEUP: tile row r = gate row r/2 (even r) or up row r/2 (odd r)
     const bool rowB = GATEUP && (r & 1);
@@ -413,10 +450,10 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
     const qk_weight& WR = rowB ? G.B : G.A;
     const int wr_in_tile = GATEUP ? (r >> 1) : r;
     const int sc_len = fr == QK_FMT_MXFP4 ? G.K / 32 : G.K / 16;
-    int n = 0, i = 0;
+    int n = 0, nr = 0, i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
       const int f = t / MB, mb = t - f * MB;
-      const int e = W.tile_e[f], row0 = W.tile_row0[f], nrow = W.tile_n[f];
+      const int e = W.tile_e[f];
       const int wrow = e * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128) + wr_in_tile;
       // ---- the tile's scale rows, and (MXFP4) their largest code
       uint8_t* srow = sS + r * G.sc_stride;
@@ -442,15 +479,32 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
       if (fr == QK_FMT_MXFP4 && ff) set_status(QK_ERR_NAN_SCALE);
       cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));  // the row's two halves
       const int cref = fr == QK_FMT_MXFP4 ? min(cmax, 254) : 0;  // MXFP4 rows: relative to the row's max
-      if (hh == 0) S.cref[i & 1][r] = cref;
+      if (hh == 0) S.cref[i & 3][r] = cref;
       __syncwarp();
-      if (lane == 0) mbar_arrive_one(&S.cref_full);
-      // ---- dequantize every stage of the tile
+      if (lane == 0) mbar_arrive_one(&S.cref_full[i & 3]);
+      // ---- dequantize every reduction step of the tile.  Packed stage layout:
+      // two boxes of 64 rows x 128 bytes (kGRK steps), 128-byte swizzle.
+      // GATEUP: box 0 = the gate rows, box 1 = the up rows; else rows 0-63, 64-127.
+      const int brow = GATEUP ? (r >> 1) : (r & 63);
+      const int bofs = (GATEUP ? (rowB ? 1 : 0) : (r >> 6)) * (kGStageR / 2) + brow * 128;
+      bool ok = true;
       for (int ks = 0; ks < nks; ++ks, ++n) {
-        const int s = n % kGS;
-        if (!__all_sync(0xffffffffu, wait(&S.full[s], (uint32_t)((n / kGS) & 1)))) break;
-        const uint8_t* raw = sR + s * kGStageR + (GATEUP ? (rowB ? kGStageR / 2 : 0) + (r >> 1) * 32 : r * 32) + hh * 16;
+        const int sub = ks % kGRK, s = nr % kGRS, sa = n % kGAS;
+        if (sub == 0 && !__all_sync(0xffffffffu, wait(&S.rfull[s], (uint32_t)((nr / kGRS) & 1)))) {
+          ok = false;
+          break;
+        }
+        const uint8_t* raw = sR + s * kGStageR + bofs + (((sub * 2 + hh) ^ (brow & 7)) << 4);
         const uint4 q = *reinterpret_cast<const uint4*>(raw);
+        if (sub == kGRK - 1 || ks == nks - 1) {  // the stage's packed rows are all in registers
+          __syncwarp();
+          if (lane == 0) mbar_arrive_one(&S.rempty[s]);
+          ++nr;
+        }
+        if (n >= kGAS && !__all_sync(0xffffffffu, wait(&S.aempty[sa], (uint32_t)((n / kGAS - 1) & 1)))) {
+          ok = false;
+          break;
+        }
         const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
         uint32_t h2[16];
 #pragma unroll
@@ -480,7 +534,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
             h2[j] = d;
           }
         }
-        uint8_t* arow = sA + s * kGStageA + r * 128;
+        uint8_t* arow = sA + sa * kGStageA + r * 128;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int c = 4 * hh + j;
@@ -489,54 +543,60 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
         }
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_one(&S.aready[s]);
+        if (lane == 0) mbar_arrive_one(&S.afull[sa]);
       }
-      // ---- epilogue: TMEM -> registers -> h (gate/up) or d (down)
-      if (!__all_sync(0xffffffffu, wait(&S.acc_full, (uint32_t)(i & 1)) && wait(&S.cref_full, (uint32_t)(i & 1))))
+      if (!ok) break;
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue --
+    // TMEM -> registers -> h (gate/up: SwiGLU of the interleaved gate/up rows)
+    // or d (down), overlapping the next tile's dequantization and MMAs.
+    const int quad = warp & 3;         // TMEM lanes 32 quad .. 32 quad + 31
+    const int feat = quad * 32 + lane;  // tile row of this thread
+    const bool frow_b = GATEUP && (feat & 1);
+    const int frow_fmt = frow_b ? FB : FA;
+    int i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      const int f = t / MB, mb = t - f * MB;
+      const int e = W.tile_e[f], row0 = W.tile_row0[f], nrow = W.tile_n[f];
+      const int ab = i & 1;
+      if (!__all_sync(0xffffffffu, wait(&S.acc_full[ab], (uint32_t)((i / 2) & 1)) &&
+                                       wait(&S.cref_full[i & 3], (uint32_t)((i / 4) & 1))))
         break;
       tc_fence_after();
-      const int quad = warp & 3;              // TMEM lanes 32 quad .. 32 quad + 31
-      const int chalf = (warp - 2) >> 2;      // which half of the columns
       const int nbox = 32 << box_index(nrow);
-      const int c_lo = nbox == 32 ? (chalf ? nbox : 0) : chalf * (nbox / 2);
-      const int c_hi = nbox == 32 ? (chalf ? nbox : nbox) : c_lo + nbox / 2;
-      const int feat = quad * 32 + lane;       // tile row of this thread
-      // this thread's tile row: MXFP4 rows were scaled by 2^(135 - cref) on chip
-      const bool frow_b = GATEUP && (feat & 1);
-      const int frow_fmt = frow_b ? FB : FA;
-      const float post = frow_fmt == QK_FMT_MXFP4 ? ldexpf(1.f, S.cref[i & 1][feat] - 135)
+      // MXFP4 rows were scaled by 2^(135 - cref) on chip; NVFP4 rows carry scale_2
+      const float post = frow_fmt == QK_FMT_MXFP4 ? ldexpf(1.f, S.cref[i & 3][feat] - 135)
                                                   : (frow_b ? G.B.scale_2[e] : G.A.scale_2[e]);
-      for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
+      const int* rshift = GATEUP ? W.xshift : W.hshift;
+      for (int c0 = 0; c0 < nbox && c0 < nrow; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+        tmem_ld32(tmem + (uint32_t)(ab * kGN) + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+        // the 32 columns' row shifts, one load per lane, broadcast by shuffles
+        const int sh_l = c0 + lane < nrow ? rshift[row0 + c0 + lane] : 0;
         if (GATEUP) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float mine = __uint_as_float(v[j]) * post;
             const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+            const float sx = pow2f(__shfl_sync(0xffffffffu, sh_l, j));
             const int col = c0 + j;
-            if (!(lane & 1) && col < nrow) {
-              const int row = row0 + col;
-              const float sx = pow2f(W.xshift[row]);
-              const float g = mine * sx, u = other * sx;
-              W.hperm[(size_t)row * G.out_ld + mb * 64 + (feat >> 1)] = silu_mul(g, u);
-            }
+            if (!(lane & 1) && col < nrow)
+              W.hperm[(size_t)(row0 + col) * G.out_ld + mb * 64 + (feat >> 1)] = silu_mul(mine * sx, other * sx);
           }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
+            const float sx = pow2f(__shfl_sync(0xffffffffu, sh_l, j));
             const int col = c0 + j;
-            if (col < nrow) {
-              const int row = row0 + col;
-              W.dperm[(size_t)row * G.out_ld + mb * 128 + feat] =
-                  __uint_as_float(v[j]) * post * pow2f(W.hshift[row]);
-            }
+            if (col < nrow)
+              W.dperm[(size_t)(row0 + col) * G.out_ld + mb * 128 + feat] = __uint_as_float(v[j]) * post * sx;
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_one(&S.acc_empty);
+      if (lane == 0) mbar_arrive_one(&S.acc_empty[ab]);
     }
   }
   __syncthreads();
@@ -608,12 +668,12 @@ static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I) {
   return W;
 }
 
-// Packed rows [rows][K/2] bytes, boxes {32 bytes, 64 rows}.
+// Packed rows [rows][K/2] bytes, boxes {128 bytes = kGRK reduction steps, 64 rows}, 128-byte swizzle.
 static bool g_map_packed(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
   const uint64_t dims[2] = {(uint64_t)K / 2, (uint64_t)rows};
   const uint64_t strides[1] = {(uint64_t)K / 2};
-  const uint32_t box[2] = {(uint32_t)kGK / 2, 64};
-  return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  const uint32_t box[2] = {(uint32_t)(kGK / 2 * kGRK), 64};
+  return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Token rows [P][K] f16, boxes {64 elements, 32 << i rows}, 128-byte swizzle.
