@@ -450,24 +450,43 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
     const qk_weight& WR = rowB ? G.B : G.A;
     const int wr_in_tile = GATEUP ? (r >> 1) : r;
     const int sc_len = fr == QK_FMT_MXFP4 ? G.K / 32 : G.K / 16;
+    // The next tile's scale rows are loaded into registers while this tile is
+    // dequantized (two threads per row, 16-byte pieces).
+    constexpr int kScV = 8;
+    const int nvq = sc_len % 32 == 0 ? sc_len / 32 : 0;
+    const bool vec = nvq > 0 && nvq <= kScV;
+    auto scale_row = [&](int tt) {
+      const int f = tt / MB, mb = tt - f * MB;
+      const int wrow = W.tile_e[f] * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128) + wr_in_tile;
+      return WR.scales + (size_t)wrow * sc_len;
+    };
+    uint4 pre[kScV];
+    auto prefetch = [&](int tt) {
+      if (!vec || tt >= n_tiles) return;
+      const uint8_t* g = scale_row(tt) + hh * 16;
+#pragma unroll
+      for (int q = 0; q < kScV; ++q)
+        if (q < nvq) pre[q] = __ldg(reinterpret_cast<const uint4*>(g + q * 32));
+    };
+    prefetch(blockIdx.x);
     int n = 0, nr = 0, i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
-      const int f = t / MB, mb = t - f * MB;
-      const int e = W.tile_e[f];
-      const int wrow = e * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128) + wr_in_tile;
       // ---- the tile's scale rows, and (MXFP4) their largest code
       uint8_t* srow = sS + r * G.sc_stride;
-      const uint8_t* gsrc = WR.scales + (size_t)wrow * sc_len;
       uint32_t m4 = 0, ff = 0;  // byte-wise maxima; any 0xFF code
-      if (sc_len % 32 == 0) {    // two threads per row, 16-byte pieces
-        for (int b = hh * 16; b < sc_len; b += 32) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(gsrc + b));
-          *reinterpret_cast<uint4*>(srow + b) = v;
+      if (vec) {
+#pragma unroll
+        for (int q = 0; q < kScV; ++q) {
+          if (q >= nvq) break;
+          const uint4 v = pre[q];
+          *reinterpret_cast<uint4*>(srow + hh * 16 + q * 32) = v;
           m4 = __vmaxu4(m4, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
           ff |= __vcmpeq4(v.x, 0xFFFFFFFFu) | __vcmpeq4(v.y, 0xFFFFFFFFu) | __vcmpeq4(v.z, 0xFFFFFFFFu) |
                 __vcmpeq4(v.w, 0xFFFFFFFFu);
         }
+        prefetch(t + gridDim.x);
       } else {
+        const uint8_t* gsrc = scale_row(t);
         for (int b = hh; b < sc_len; b += 2) {
           const uint32_t c = gsrc[b];
           srow[b] = (uint8_t)c;
@@ -575,14 +594,22 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
         // the 32 columns' row shifts, one load per lane, broadcast by shuffles
         const int sh_l = c0 + lane < nrow ? rshift[row0 + c0 + lane] : 0;
         if (GATEUP) {
+          // lane pair (gate, up) of one feature: the even lane finishes column
+          // j, the odd lane column j + 1, after swapping one value each
+          const bool odd = lane & 1;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float mine = __uint_as_float(v[j]) * post;
-            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-            const float sx = pow2f(__shfl_sync(0xffffffffu, sh_l, j));
-            const int col = c0 + j;
-            if (!(lane & 1) && col < nrow)
-              W.hperm[(size_t)(row0 + col) * G.out_ld + mb * 64 + (feat >> 1)] = silu_mul(mine * sx, other * sx);
+          for (int j = 0; j < 32; j += 2) {
+            const float a0 = __uint_as_float(v[j]) * post, a1 = __uint_as_float(v[j + 1]) * post;
+            const float give = odd ? a0 : a1;  // even lane sends its column j+1, odd lane its column j
+            const float got = __shfl_xor_sync(0xffffffffu, give, 1);
+            const float g = odd ? got : a0, u = odd ? a1 : got;  // even: (g_j, u_j); odd: (g_j+1, u_j+1)
+            const int col = c0 + j + (odd ? 1 : 0);
+            const float sx = pow2f(__shfl_sync(0xffffffffu, sh_l, j + (odd ? 1 : 0)));
+            if (col < nrow) {
+              const float gs = g * sx;
+              W.hperm[(size_t)(row0 + col) * G.out_ld + mb * 64 + (feat >> 1)] =
+                  __fdividef(gs, 1.0f + __expf(-gs)) * (u * sx);
+            }
           }
         } else {
 #pragma unroll
