@@ -52,6 +52,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=20,
                     help="timed repetitions of the 2048-token prefill layer (0: skip)")
+    ap.add_argument("--prefill-experts", type=int, default=0,
+                    help="profiling only: fewer experts in the prefill layer (0: the workload's 256)")
+    ap.add_argument("--prefill-tokens", type=int, default=0,
+                    help="profiling only: fewer prefill tokens (0: the workload's 2048)")
     return ap.parse_args()
 
 
@@ -363,6 +367,9 @@ def run_prefill(args, rank, world, dev):
     from block_quantized_expert_mxfp4_b200 import synth, workload
 
     wl = synth.WORKLOADS["prefill"]
+    if args.prefill_experts or args.prefill_tokens:
+        import dataclasses
+        wl = dataclasses.replace(wl, E=args.prefill_experts or wl.E, T=args.prefill_tokens or wl.T)
     T, k = wl.T, wl.k
     layer = workload.make_layer(wl, seed=rank, layer=0)
     lay = layer.c()
@@ -413,7 +420,7 @@ def run_prefill(args, rank, world, dev):
     except Exception:
         tpeak, tkind = 1590.0, "fallback"
     return {
-        "workload": "prefill MoE layer: 2048 tokens, 256 experts, top-6 Zipf(s=1) routing, hidden 4096, "
+        "workload": f"prefill MoE layer: {T} tokens, {wl.E} experts, top-6 Zipf(s=1) routing, hidden 4096, "
                     "intermediate 2048, MXFP4 gate/up/down, bf16 N(0,1) activations",
         "tokens_per_s": round(T * world / t, 1), "ms_per_layer": round(t * 1e3, 4), "steps": K,
         "experts_touched": touched,
