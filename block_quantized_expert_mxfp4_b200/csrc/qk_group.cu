@@ -264,7 +264,7 @@ struct GemmArgs {
   int rows_per_e;      // weight rows of one expert (gate/up: inter; down: hidden)
   int MB;              // weight-row tiles per expert (gate/up: inter/64; down: hidden/128)
   int out_ld;          // output row length (gate/up: inter; down: hidden)
-  int sc_stride;       // bytes per row of the staged tile scales
+  int sc_stride;       // bytes per row of the staged tile scales (row length + 4: rows on distinct banks)
   alignas(64) CUtensorMap tqa, tqb;    // packed rows, 2-D bytes {K/2, rows}, box {128, 64}, 128B swizzle
   alignas(64) CUtensorMap tb[kGNBox];  // token rows, f16 {K, P}, box {64, 32 << i}, 128-byte swizzle
 };
@@ -282,7 +282,7 @@ struct GHead {
   alignas(8) uint64_t cref_full[4];  // the tile's per-row reference codes written (tile % 4)
   uint32_t tmem;
   int abort;                         // a wait ran out: every role stops
-  int cref[4][kGM];                  // per tile row (tile % 4): largest e8m0 code of the row
+  uint8_t cref[4][kGM];              // per tile row (tile % 4): largest e8m0 code of the row
 };
 
 constexpr int kGStageA = kGM * kGK * 2;   // 16 KB f16 weight tile
@@ -479,7 +479,11 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
         for (int q = 0; q < kScV; ++q) {
           if (q >= nvq) break;
           const uint4 v = pre[q];
-          *reinterpret_cast<uint4*>(srow + hh * 16 + q * 32) = v;
+          uint32_t* d = reinterpret_cast<uint32_t*>(srow + hh * 16 + q * 32);  // 4-byte aligned rows
+          d[0] = v.x;
+          d[1] = v.y;
+          d[2] = v.z;
+          d[3] = v.w;
           m4 = __vmaxu4(m4, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
           ff |= __vcmpeq4(v.x, 0xFFFFFFFFu) | __vcmpeq4(v.y, 0xFFFFFFFFu) | __vcmpeq4(v.z, 0xFFFFFFFFu) |
                 __vcmpeq4(v.w, 0xFFFFFFFFu);
@@ -498,7 +502,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
       if (fr == QK_FMT_MXFP4 && ff) set_status(QK_ERR_NAN_SCALE);
       cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));  // the row's two halves
       const int cref = fr == QK_FMT_MXFP4 ? min(cmax, 254) : 0;  // MXFP4 rows: relative to the row's max
-      if (hh == 0) S.cref[i & 3][r] = cref;
+      if (hh == 0) S.cref[i & 3][r] = (uint8_t)cref;
       __syncwarp();
       if (lane == 0) mbar_arrive_one(&S.cref_full[i & 3]);
       // ---- dequantize every reduction step of the tile.  Packed stage layout:
@@ -754,7 +758,7 @@ qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
   g1.rows_per_e = I;
   g1.MB = I / 64;
   g1.out_ld = I;
-  g1.sc_stride = (a.gate.fmt == QK_FMT_NVFP4 || a.up.fmt == QK_FMT_NVFP4) ? H / 16 : H / 32;
+  g1.sc_stride = ((a.gate.fmt == QK_FMT_NVFP4 || a.up.fmt == QK_FMT_NVFP4) ? H / 16 : H / 32) + 4;
   if (!g_map_packed(&g1.tqa, a.gate.q, (int64_t)E * I, H) || !g_map_packed(&g1.tqb, a.up.q, (int64_t)E * I, H) ||
       !g_map_tokens(g1.tb, W.xperm, P, H))
     return QK_ERR_CUDA;
@@ -771,7 +775,7 @@ qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
   g2.rows_per_e = H;
   g2.MB = H / 128;
   g2.out_ld = H;
-  g2.sc_stride = a.down.fmt == QK_FMT_NVFP4 ? I / 16 : I / 32;
+  g2.sc_stride = (a.down.fmt == QK_FMT_NVFP4 ? I / 16 : I / 32) + 4;
   if (!g_map_packed(&g2.tqa, a.down.q, (int64_t)E * H, I) || !g_map_tokens(g2.tb, W.h16, P, I)) return QK_ERR_CUDA;
   g2.tqb = g2.tqa;
   rc = g_dispatch<false>(g2, st);
