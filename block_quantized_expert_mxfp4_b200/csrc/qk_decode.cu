@@ -196,6 +196,8 @@ struct DGeo {
   int fast;         // every row of the call is staged once (rows <= xcap)
   int D;            // stages per warp
   int off_rings, off_scales, off_act;  // from the 1024-aligned base
+  int off_raw;      // k_down, every pair row staged at once: the fp32 h rows as copied
+  int raw;          // bytes of that area (0: h is read with plain loads)
   int smem;         // total dynamic shared memory (with alignment slack)
 };
 
@@ -221,7 +223,8 @@ constexpr int kDHead = (int)((sizeof(DHead) + 127) / 128 * 128);
 
 __host__ __device__ inline int up_to(int x, int a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline DGeo make_dgeo(int K, int Kc, int fa, int fb, int xcap, int D, bool tmap_ok) {
+__host__ __device__ inline DGeo make_dgeo(int K, int Kc, int fa, int fb, int xcap, int D, bool tmap_ok,
+                                          int raw = 0) {
   DGeo g;
   g.K = K;
   g.Kc = Kc;
@@ -244,7 +247,12 @@ __host__ __device__ inline DGeo make_dgeo(int K, int Kc, int fa, int fb, int xca
   g.off_rings = up_to(kDHead, 1024);
   g.off_scales = g.off_rings + kDW * D * g.nib_stage;
   g.off_act = up_to(g.off_scales + kDW * D * g.sc_stage, 16);
-  g.smem = g.off_act + xcap * g.act_stride * 2 + 1024;  // + slack to align the base
+  // k_down stages h before its weight stream starts: the raw rows borrow the
+  // rings when they fit there
+  const bool in_rings = raw <= kDW * D * g.nib_stage;
+  g.off_raw = in_rings ? g.off_rings : up_to(g.off_act + xcap * g.act_stride * 2, 16);
+  g.raw = raw;
+  g.smem = up_to(g.off_act + xcap * g.act_stride * 2, 16) + (in_rings ? 0 : raw) + 1024;  // + alignment slack
   return g;
 }
 
@@ -516,6 +524,34 @@ __device__ __forceinline__ void stage_h(const DecodeArgs& a, DHead& S, __half* a
     reinterpret_cast<uint2*>(act + (size_t)row * stride)[q] =
         make_uint2(pack_f16x2(v.x * sc, v.y * sc), pack_f16x2(v.z * sc, v.w * sc));
   }
+}
+
+// Every pair row at once (pairs 0 .. nrows-1, contiguous in h): one round of
+// cp.async into the raw area, then maxima and conversion from shared memory.
+__device__ __forceinline__ void stage_h_raw(const DecodeArgs& a, DHead& S, __half* act, int stride, int nrows,
+                                            float* raw) {
+  const int nvec = a.I / 4;
+  const int total = nrows * nvec;
+  for (int j = threadIdx.x; j < total; j += kDW * 32) cp_async16_nohint(raw + 4 * j, a.h + 4 * j);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  if (threadIdx.x < kXCap) S.amax_bits[threadIdx.x] = 0u;
+  asm volatile("cp.async.wait_group 0;" ::: "memory");  // the h group only: ring copies come later
+  __syncthreads();
+  const bool uniform = nvec % 32 == 0;  // a warp's 32 vectors lie in one row
+  for (int j = threadIdx.x; j < total; j += kDW * 32) {
+    const float4 v = *reinterpret_cast<const float4*>(raw + 4 * j);
+    row_max(S, j / nvec, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))), uniform);
+  }
+  rows_shift(S, nrows);
+  for (int j = threadIdx.x; j < total; j += kDW * 32) {
+    const int row = j / nvec, q = j - row * nvec;
+    const float4 v = *reinterpret_cast<const float4*>(raw + 4 * j);
+    const float sc = pow2f(-S.shift[row]);
+    reinterpret_cast<uint2*>(act + (size_t)row * stride)[q] =
+        make_uint2(pack_f16x2(v.x * sc, v.y * sc), pack_f16x2(v.z * sc, v.w * sc));
+  }
+  // the raw area may be the rings: order these accesses before the copies into them
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ------------------------------------------------------------ the kernel --
@@ -810,7 +846,8 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
         pdl_wait();  // h and hmax come from k_gateup
         waited_pdl = true;
       }
-      stage_h(a, S, act, G.act_stride, seg_rows, fast);
+      if (fast && G.raw) stage_h_raw(a, S, act, G.act_stride, seg_rows, reinterpret_cast<float*>(smem + G.off_raw));
+      else stage_h(a, S, act, G.act_stride, seg_rows, fast);
       for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (done + i) % G.D);
     }
     __syncthreads();
@@ -898,14 +935,14 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
 // ================================================================= host ==
 // Largest chunk (<= 1024, dividing K, >= 128) whose rings of at least 3 stages
 // per warp fit in shared memory (else 2 stages), ring depth up to kMaxD.
-static DGeo plan_geo(int K, int fa, int fb, int xcap, bool tmap_ok) {
+static DGeo plan_geo(int K, int fa, int fb, int xcap, bool tmap_ok, int raw) {
   const int cap = max_smem_optin();
-  DGeo two = make_dgeo(K, 128, fa, fb, xcap, 2, tmap_ok);
+  DGeo two = make_dgeo(K, 128, fa, fb, xcap, 2, tmap_ok, raw);
   two.smem = 0;
   for (int Kc = 1024; Kc >= 128; Kc >>= 1) {
     if (K % Kc) continue;
     for (int D = kMaxD; D >= 2; --D) {
-      const DGeo g = make_dgeo(K, Kc, fa, fb, xcap, D, tmap_ok);
+      const DGeo g = make_dgeo(K, Kc, fa, fb, xcap, D, tmap_ok, raw);
       if (g.smem > cap) continue;
       if (D >= 3) return g;
       if (!two.smem) two = g;
@@ -948,13 +985,17 @@ static qk_status go(DArgs& P, cudaStream_t st, bool pdl) {
 
 // Geometry of one kernel: tensor-map mode when the maps encode, else rows by cp.async.
 static DGeo plan_kernel(int K, int fa, int fb, int rows, CUtensorMap* ta, CUtensorMap* tb,
-                        const uint8_t* qa, const uint8_t* qb, int64_t n_rows, int box_rows) {
+                        const uint8_t* qa, const uint8_t* qb, int64_t n_rows, int box_rows, bool raw_h) {
   const int xcap = std::min(rows, kXCap);
-  DGeo G = plan_geo(K, fa, fb, xcap, true);
+  // k_down with every pair row staged at once copies h raw (fp32) first, when it fits
+  const int raw = raw_h && rows <= kXCap ? rows * K * 4 : 0;
+  DGeo G = plan_geo(K, fa, fb, xcap, true, raw);
+  if (!G.smem && raw) G = plan_geo(K, fa, fb, xcap, true, 0);
+  const int raw_used = G.raw;
   if (G.smem && G.tmap) {
     bool ok = encode_rows(ta, qa, n_rows, K, box_rows, G.nseg);
     if (ok && tb) ok = encode_rows(tb, qb, n_rows, K, box_rows, G.nseg);
-    if (!ok) G = plan_geo(K, fa, fb, xcap, false);
+    if (!ok) G = plan_geo(K, fa, fb, xcap, false, raw_used);
   }
   G.fast = rows <= kXCap ? 1 : 0;
   return G;
@@ -965,14 +1006,14 @@ qk_status decode_forward(DecodeArgs args, cudaStream_t st) {
   P1.a = args;
   P1.RT = args.I / 8;
   P1.G = plan_kernel(args.H, args.gate.fmt, args.up.fmt, args.T, &P1.tqa, &P1.tqb, args.gate.q,
-                     args.up.q, (int64_t)args.E * args.I, 8);
+                     args.up.q, (int64_t)args.E * args.I, 8, false);
   if (!P1.G.smem) return QK_ERR_UNSUPPORTED;
   P1.U_max = args.P * P1.RT;  // virtual experts <= pairs
   DArgs P2 = {};
   P2.a = args;
   P2.RT = args.H / 16;
   P2.G = plan_kernel(args.I, args.down.fmt, args.down.fmt, args.P, &P2.tqa, nullptr, args.down.q,
-                     nullptr, (int64_t)args.E * args.H, 16);
+                     nullptr, (int64_t)args.E * args.H, 16, true);
   if (!P2.G.smem) return QK_ERR_UNSUPPORTED;
   P2.U_max = args.P * P2.RT;
   constexpr int MX = QK_FMT_MXFP4, NV = QK_FMT_NVFP4;
