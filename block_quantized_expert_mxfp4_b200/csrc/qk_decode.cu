@@ -619,14 +619,52 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
   const unsigned long long limit = g_wait_limit_ns;
   const int vpr = G.Kc / 32;  // 16-byte vectors per packed chunk row
   // Chunk c into stage `slot`.
-  auto issue = [&](int c, int slot) {
+  // This lane's scale pieces of a chunk (the same for every chunk): source
+  // offsets from the A / B scale slice, destination offsets in the stage.
+  constexpr int kMaxPc = 4;
+  int pc_src[kMaxPc], pc_dst[kMaxPc];
+  bool pc_b[kMaxPc];
+  int npc = 0;
+  {
+    const int pa = G.sca / G.sc_vec, pb = G.scb / G.sc_vec;  // pieces per row
+    for (int idx = lane; idx < 8 * (pa + pb) && npc < kMaxPc; idx += 32, ++npc) {
+      const bool isb = idx >= 8 * pa;
+      const int k2 = isb ? idx - 8 * pa : idx;
+      const int pr = isb ? pb : pa;
+      const int row = k2 / pr, pc = k2 - row * pr;
+      pc_b[npc] = isb;
+      pc_src[npc] = row * (isb ? G.scb_g : G.sca_g) + pc * G.sc_vec;
+      pc_dst[npc] = (isb ? 8 * G.sca + row * G.scb : row * G.sca) + pc * G.sc_vec;
+    }
+  }
+  // Position of a chunk: unit u = v * RT + r, chunk kc of the unit.
+  struct Cur {
+    int u, kc, v, r;
+  };
+  auto cur_at = [&](int c) -> Cur {
+    Cur q;
+    q.u = c / nk;
+    q.kc = c - q.u * nk;
+    q.v = q.u / RT;
+    q.r = q.u - q.v * RT;
+    return q;
+  };
+  auto cur_next = [&](Cur& q) {
+    if (++q.kc == nk) {
+      q.kc = 0;
+      ++q.u;
+      if (++q.r == RT) {
+        q.r = 0;
+        ++q.v;
+      }
+    }
+  };
+  auto issue = [&](const Cur& q, int slot) {
     uint8_t* st = nring + (size_t)slot * G.nib_stage;
     uint8_t* sd = sring + (size_t)slot * G.sc_stage;
     uint64_t* bar = &full[slot];
-    const int u = c / nk;
-    const int kc = c - u * nk;
-    const int v = u / RT, r = u - v * RT;
-    const int e = S.R.v_expert[v];
+    const int kc = q.kc, r = q.r;
+    const int e = S.R.v_expert[q.v];
     const int64_t rowA0 = (int64_t)e * rows_per_e + (GATEUP ? r * 8 : r * 16);
     const int64_t rowB0 = GATEUP ? rowA0 : rowA0 + 8;
     if (!G.tmap) {
@@ -641,15 +679,11 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     }
     const uint8_t* sa = WA.scales + rowA0 * G.sca_g + (size_t)kc * G.sca;
     const uint8_t* sb = WB.scales + rowB0 * G.scb_g + (size_t)kc * G.scb;
-    const int pa = G.sca / G.sc_vec, pb = G.scb / G.sc_vec;  // pieces per row
-    for (int idx = lane; idx < 8 * (pa + pb); idx += 32) {
-      const bool isb = idx >= 8 * pa;
-      const int k2 = isb ? idx - 8 * pa : idx;
-      const int pr = isb ? pb : pa;
-      const int row = k2 / pr, pc = k2 - row * pr;
-      const uint8_t* src = isb ? sb + (size_t)row * G.scb_g + pc * G.sc_vec
-                               : sa + (size_t)row * G.sca_g + pc * G.sc_vec;
-      uint8_t* dst = sd + (isb ? 8 * G.sca + row * G.scb : row * G.sca) + pc * G.sc_vec;
+#pragma unroll
+    for (int q2 = 0; q2 < kMaxPc; ++q2) {
+      if (q2 >= npc) break;
+      const uint8_t* src = (pc_b[q2] ? sb : sa) + pc_src[q2];
+      uint8_t* dst = sd + pc_dst[q2];
       if (G.sc_vec == 16) cp_async16(dst, src, pol);
       else cp_async4(dst, src);
     }
@@ -837,9 +871,19 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     // ---- k_gateup: x copies (their own cp.async group), weight prefetch (D-1
     // chunks), then the conversion of x.  k_down: h first (it is in L2 and must
     // not queue behind the weight stream), then the weight prefetch.
+    // issue cursor (chunk w0 + issued) and ring slots of issue and consumption
+    Cur icur = cur_at(w0);
+    int islot = done % G.D;
+    int issued = 0;
+    auto issue_next = [&]() {
+      issue(icur, islot);
+      cur_next(icur);
+      if (++islot == G.D) islot = 0;
+      ++issued;
+    };
     if (GATEUP) {
       if (!fast) stage_x_issue(a, S, act, G.act_stride, seg_rows, false);
-      for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (done + i) % G.D);
+      for (int i = 0; i < G.D - 1 && i < wn; ++i) issue_next();
       stage_x_finish(a, S, act, G.act_stride, seg_rows);
     } else {
       if (!waited_pdl) {
@@ -848,7 +892,7 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
       }
       if (fast && G.raw) stage_h_raw(a, S, act, G.act_stride, seg_rows, reinterpret_cast<float*>(smem + G.off_raw));
       else stage_h(a, S, act, G.act_stride, seg_rows, fast);
-      for (int i = 0; i < G.D - 1 && i < wn; ++i) issue(w0 + i, (done + i) % G.D);
+      for (int i = 0; i < G.D - 1 && i < wn; ++i) issue_next();
     }
     __syncthreads();
 
@@ -868,11 +912,13 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
         }
       }
     };
+    Cur ccur = cur_at(w0);  // consumption cursor
+    int slot = done % G.D;
+    uint32_t phase = (uint32_t)((done / G.D) & 1);
     for (int i = 0; i < wn; ++i) {
       // keep D-1 chunks in flight: issue chunk i+D-1, then wait for chunk i
-      if (i + G.D - 1 < wn) issue(w0 + i + G.D - 1, (done + G.D - 1) % G.D);
-      const int slot = done % G.D;
-      const bool landed = mbar_wait_bounded(&full[slot], (uint32_t)((done / G.D) & 1), limit);
+      if (issued < wn) issue_next();
+      const bool landed = mbar_wait_bounded(&full[slot], phase, limit);
       if (__any_sync(0xffffffffu, !landed)) {
         // the copies did not land in time: report, drain what this warp has in
         // flight, and stop the block at the end of the segment
@@ -885,9 +931,7 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
         dead = true;
         break;
       }
-      const int cc = w0 + i;
-      const int u = cc / nk;
-      const int kc = cc - u * nk;
+      const int u = ccur.u, kc = ccur.kc, v = ccur.v;
       if (u != cur_u) {
         if (cur_u >= 0) close();
         cur_u = u;
@@ -895,13 +939,17 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
         acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
       }
       kc_last = kc;
-      const int v = u / RT;
       const int n = S.R.v_n[v];
       const int row = S.col_row[(v - seg_v0) * kTileN + (g < n ? g : 0)];
       const __half* xrow = act + (size_t)row * G.act_stride + 8 * t + (size_t)kc * G.Kc;
       chunk_mma<FA, FB, GATEUP>(acc, nring + (size_t)slot * G.nib_stage, sring + (size_t)slot * G.sc_stage,
                                 G, xrow, lane, bad);
       ++done;
+      cur_next(ccur);
+      if (++slot == G.D) {
+        slot = 0;
+        phase ^= 1u;
+      }
       __syncwarp();  // every lane is done with this stage before it is refilled
     }
     if (dead) {
