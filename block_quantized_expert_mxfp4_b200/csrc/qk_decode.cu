@@ -598,6 +598,9 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
   }
   if (threadIdx.x == 0) S.dead = 0;
   if (GATEUP && fast) stage_x_issue(a, S, act, G.act_stride, a.T, true);  // x does not depend on the routing
+  // k_gateup may start while the router that writes ids and w is finishing
+  // (programmatic dependent launch): wait for it before reading them
+  if (GATEUP) pdl_wait();
   build_route(a.ids, a.P, a.E, S.R);  // ends with a block barrier
   const int n_v = S.R.n_v;
   const int U = n_v * RT;
@@ -1067,10 +1070,12 @@ qk_status decode_forward(DecodeArgs args, cudaStream_t st) {
   constexpr int MX = QK_FMT_MXFP4, NV = QK_FMT_NVFP4;
   const int fg = args.gate.fmt, fu = args.up.fmt, fd = args.down.fmt;
   qk_status rc;
-  if (fg == MX && fu == MX) rc = go<MX, MX, true>(P1, st, false);
-  else if (fg == MX) rc = go<MX, NV, true>(P1, st, false);
-  else if (fu == MX) rc = go<NV, MX, true>(P1, st, false);
-  else rc = go<NV, NV, true>(P1, st, false);
+  // k_gateup overlaps its prologue with the end of the previous kernel only
+  // when that kernel allows it (the router does); otherwise it waits as usual
+  if (fg == MX && fu == MX) rc = go<MX, MX, true>(P1, st, true);
+  else if (fg == MX) rc = go<MX, NV, true>(P1, st, true);
+  else if (fu == MX) rc = go<NV, MX, true>(P1, st, true);
+  else rc = go<NV, NV, true>(P1, st, true);
   if (rc != QK_OK) return rc;
   return fd == MX ? go<MX, MX, false>(P2, st, true) : go<NV, NV, false>(P2, st, true);
 }

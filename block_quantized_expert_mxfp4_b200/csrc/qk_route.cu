@@ -21,6 +21,9 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route(const float* __restr
                                                             int E, int k, int32_t* __restrict__ ids,
                                                             float* __restrict__ w) {
   extern __shared__ float srow[];
+  // the expert FFN launched next may start its own prologue now; it waits
+  // for this grid's completion before it reads ids and w
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kRouteWarps + warp;
   if (t >= T) return;
