@@ -640,7 +640,22 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
       pc_dst[npc] = (isb ? 8 * G.sca + row * G.scb : row * G.sca) + pc * G.sc_vec;
     }
   }
-  // Position of a chunk: unit u = v * RT + r, chunk kc of the unit.
+  // Unit order.  Expert-major (u = v * RT + r) in general.  k_down with every
+  // pair row staged orders its units row-tile-major (u = r * n_v + v): a
+  // block then holds every expert's unit of most of its row tiles, so the
+  // row-tile combines are spread over the blocks instead of all falling to
+  // the blocks that hold the last expert.
+  const bool rmajor = !GATEUP && fast;
+  auto unit_vr = [&](int u, int& v, int& r) {
+    if (rmajor) {
+      r = u / n_v;
+      v = u - r * n_v;
+    } else {
+      v = u / RT;
+      r = u - v * RT;
+    }
+  };
+  // Position of a chunk: unit u (expert slot v, row tile r), chunk kc of the unit.
   struct Cur {
     int u, kc, v, r;
   };
@@ -648,15 +663,19 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     Cur q;
     q.u = c / nk;
     q.kc = c - q.u * nk;
-    q.v = q.u / RT;
-    q.r = q.u - q.v * RT;
+    unit_vr(q.u, q.v, q.r);
     return q;
   };
   auto cur_next = [&](Cur& q) {
     if (++q.kc == nk) {
       q.kc = 0;
       ++q.u;
-      if (++q.r == RT) {
+      if (rmajor) {
+        if (++q.v == n_v) {
+          q.v = 0;
+          ++q.r;
+        }
+      } else if (++q.r == RT) {
         q.r = 0;
         ++q.v;
       }
@@ -750,7 +769,8 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     bool last = false;
     int r = 0;
     if (lane < npend) {
-      r = pend % RT;
+      int v_unused;
+      unit_vr(pend, v_unused, r);
       last = atom_add_acq_rel(a.cnt + r, 1u) + 1u == (uint32_t)n_v;
     }
     unsigned m = __ballot_sync(0xffffffffu, last);
@@ -765,7 +785,8 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
 
   // A finished unit: scale, then SwiGLU into h (k_gateup) or the unit result (k_down).
   auto finalize = [&](int u, float4 f, int seg_v0) {
-    const int v = u / RT, r = u - v * RT;
+    int v, r;
+    unit_vr(u, v, r);
     const int e = S.R.v_expert[v], n = S.R.v_n[v];
     const float s2a = WA.fmt == QK_FMT_NVFP4 ? WA.scale_2[e] : 1.f;
     const float s2b = WB.fmt == QK_FMT_NVFP4 ? WB.scale_2[e] : 1.f;
@@ -802,7 +823,8 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
         }
       }
     } else {
-      reinterpret_cast<float4*>(a.ures)[(size_t)u * 32 + lane] = make_float4(fv[0], fv[1], fv[2], fv[3]);
+      // stored expert-major whatever the processing order (the combine reads v * RT + r)
+      reinterpret_cast<float4*>(a.ures)[((size_t)v * RT + r) * 32 + lane] = make_float4(fv[0], fv[1], fv[2], fv[3]);
       if (lane == npend) pend = u;
       if (++npend == 32) flush();
     }
