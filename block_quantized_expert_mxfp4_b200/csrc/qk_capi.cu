@@ -39,7 +39,7 @@ static int decode_chunk(int top_k) { return kMaxPairs / top_k; }
 size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_t top_k) {
   if (layer_ok(L) != QK_OK || n_tokens < 0 || top_k < 1 || top_k > 8) return 0;
   if (n_tokens > decode_chunk(top_k))
-    return group_workspace_bytes(n_tokens, top_k, L->gate.n_experts, L->hidden, L->inter);
+    return group_workspace_bytes(L, n_tokens, top_k);
   return decode_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
 }
 

@@ -119,6 +119,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int c0,
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)),
+      "l"(policy)
+      : "memory");
+}
+
 // Bring a tensor map (kernel-parameter space) into the descriptor cache.
 __device__ __forceinline__ void tmap_prefetch(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
@@ -261,6 +271,46 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t desc_a, uint6
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
       "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
+// Block-scaled MMA (kind::mxf8f6f4): operand formats 0 = e4m3, 5 = e2m1 (in
+// shared memory one element per byte position: sixteen 4-bit values in the
+// low 8 bytes of each 16-byte chunk), one ue8m0 scale per 32 elements of K
+// for every row of A and of B, fp32 accumulator, K = 32 per instruction.
+// Fields: B scale id (bits 4-5), A format (7-9), B format (10-12), K-major
+// A and B, N >> 3 (17-22), scale type ue8m0 (bit 23), M >> 4 (24-28), A
+// scale id (29-30).  The scale ids select the byte of the 32-bit tensor-memory
+// word that holds the scale for this instruction's 32 elements of K.
+__host__ __device__ constexpr uint32_t umma_idesc_mx(int M, int N, int a_fmt, int b_fmt) {
+  return ((uint32_t)a_fmt << 7) | ((uint32_t)b_fmt << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t umma_idesc_sf_ids(uint32_t idesc, int a_id, int b_id) {
+  return idesc | ((uint32_t)b_id << 4) | ((uint32_t)a_id << 29);
+}
+
+// D[tmem] (+)= (A * sA) (B * sB)^T; tsfa / tsfb are the tensor-memory
+// addresses of the scale columns with the byte index in bits 30-31.
+__device__ __forceinline__ void umma_mx(uint32_t tmem_d, uint64_t desc_a, uint64_t desc_b, uint32_t idesc,
+                                        uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(tmem_d),
+      "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb));
+}
+
+// Shared-memory descriptor of a scale-factor atom for tcgen05.cp: 32 rows of
+// 16 bytes, contiguous (no swizzle; 8-row groups 128 bytes apart).
+__device__ __forceinline__ uint64_t umma_desc_sf(const void* smem_atom) {
+  const uint64_t addr = (uint64_t)(smem_u32(smem_atom) >> 4) & 0x3FFFu;
+  return addr | (8ull << 32) | (1ull << 46);
+}
+
+// Copy 32 rows x 128 bits from shared memory into 4 tensor-memory columns of
+// lanes 0-31, replicated into the lanes of all four sub-partitions.  Ordered
+// with the tcgen05.mma instructions the same thread issues.
+__device__ __forceinline__ void utccp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc));
 }
 
 // The mbarrier receives one arrival when every tcgen05 operation this thread

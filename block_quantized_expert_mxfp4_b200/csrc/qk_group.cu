@@ -29,12 +29,12 @@
 #include <algorithm>
 
 #include "qk_common.cuh"
+#include "qk_group.cuh"
 #include "qk_tmap.h"
 
 namespace qk {
 
 constexpr int kGM = 128;        // weight rows per tile (tcgen05 M)
-constexpr int kGN = 256;        // token rows per tile (largest tcgen05 N)
 constexpr int kGK = 64;         // reduction per stage (one 128-byte f16 row)
 constexpr int kGRS = 3;         // packed-weight stages (16 KB: four reduction steps of 128 rows)
 constexpr int kGRK = 4;         // reduction steps per packed-weight stage
@@ -44,25 +44,6 @@ constexpr int kGDW = 8;         // dequant / epilogue warps
 constexpr int kGEW = 4;         // epilogue warps (one per TMEM lane quadrant)
 constexpr int kGThreads = (3 + kGDW + kGEW) * 32;  // weight producer, MMA, token producer, dequant, epilogue
 constexpr int kGNBox = 4;       // token-box heights 32, 64, 128, 256
-
-struct GroupWs {
-  int* counts;      // [E] pairs per expert
-  int* offsets;     // [E + 1] first sorted row of each expert
-  int* fill;        // [E] scatter cursors
-  int* tile_e;      // [F] expert of token tile f
-  int* tile_row0;   // [F] first sorted row of token tile f
-  int* tile_n;      // [F] rows in token tile f
-  int* n_tiles;     // [1] token tiles
-  int* inv;         // [P] pair -> sorted row
-  int* xshift;      // [P] per sorted row: x scaled by 2^-xshift
-  int* hshift;      // [P] per sorted row: h scaled by 2^-hshift
-  __half* xperm;    // [P][H] f16
-  float* hperm;     // [P][I] fp32
-  __half* h16;      // [P][I] f16
-  float* dperm;     // [P][H] fp32
-  unsigned long long* n_flush;  // [1] MXFP4 blocks flushed by the relative scaling
-  size_t zero_bytes;            // bytes zeroed from `counts` on every call
-};
 
 }  // namespace qk
 
@@ -82,8 +63,9 @@ __global__ void k_grp_count(const int32_t* __restrict__ ids, int P, int E, int* 
 
 // One block: exclusive scans of the per-expert pair counts and token-tile
 // counts; writes the token-tile list.
-constexpr int kScanThreads = 1024;
-__global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, int E) {
+// Token tiles hold at most tn rows; with `mx`, also the per-tile expert
+// extent (first tile, tile count) and each expert's first tile.
+__global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, int E, int tn, int mx) {
   __shared__ int s_pairs[kScanThreads / 32], s_tiles[kScanThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (E + kScanThreads - 1) / kScanThreads;
@@ -92,7 +74,7 @@ __global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, int E) {
   for (int e = e0; e < e1; ++e) {
     const int c = W.counts[e];
     np += c;
-    nt += (c + kGN - 1) / kGN;
+    nt += (c + tn - 1) / tn;
   }
   int ip = np, it = nt;  // inclusive scans within the warp
 #pragma unroll
@@ -126,12 +108,18 @@ __global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, int E) {
   int tile = it - nt + (warp ? s_tiles[warp - 1] : 0);
   for (int e = e0; e < e1; ++e) {
     const int c = W.counts[e];
+    const int first = tile, cnt = (c + tn - 1) / tn;
     W.offsets[e] = row;
     W.fill[e] = 0;
-    for (int r = 0; r < c; r += kGN, ++tile) {
+    if (mx) W.exp_tile0[e] = first;
+    for (int r = 0; r < c; r += tn, ++tile) {
       W.tile_e[tile] = e;
       W.tile_row0[tile] = row + r;
-      W.tile_n[tile] = min(kGN, c - r);
+      W.tile_n[tile] = min(tn, c - r);
+      if (mx) {
+        W.tile_first[tile] = first;
+        W.tile_cnt[tile] = cnt;
+      }
     }
     row += c;
   }
@@ -143,7 +131,6 @@ __global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, int E) {
 
 // One block per token: the row maximum, then the row in f16 (scaled by
 // 2^-shift) at the sorted position of each of the token's pairs.
-constexpr int kRowThreads = 128;
 __device__ __forceinline__ int block_shift(float m, float* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -644,14 +631,17 @@ namespace qk {
 // ================================================================= host ==
 struct GWsLayout {
   size_t counts, offsets, fill, tile_e, tile_row0, tile_n, n_tiles, n_flush, zero_end;
-  size_t inv, xshift, hshift, xperm, hperm, h16, dperm, total;
+  size_t inv, dperm, xshift, hshift, xperm, hperm, h16;
+  size_t tile_first, tile_cnt, exp_tile0, rtile, xq, sfx, gu, hq, sfh, total;
 };
 
-static int g_max_tiles(int P, int E) { return P / kGN + E + 1; }
+static int g_max_tiles(int P, int E, int tn) { return P / tn + E + 1; }
 
-static GWsLayout g_layout(int T, int k, int E, int H, int I) {
-  const size_t P = (size_t)T * k, F = (size_t)g_max_tiles((int)P, E);
-  GWsLayout L;
+// Workspace of the grouped path; `mx` selects the MXFP4 block-scaled buffers
+// instead of the f16 ones.
+static GWsLayout g_layout(int T, int k, int E, int H, int I, bool mx) {
+  const size_t P = (size_t)T * k, F = (size_t)g_max_tiles((int)P, E, mx ? kXN : kGN);
+  GWsLayout L = {};
   size_t o = 0;
   L.counts = o; o += (size_t)E * 4;          // zeroed on every call: counts .. n_flush
   L.n_tiles = o; o += 8;
@@ -664,22 +654,38 @@ static GWsLayout g_layout(int T, int k, int E, int H, int I) {
   L.tile_row0 = o; o += align256(F * 4);
   L.tile_n = o; o += align256(F * 4);
   L.inv = o; o += align256(P * 4);
-  L.xshift = o; o += align256(P * 4);
-  L.hshift = o; o += align256(P * 4);
-  L.xperm = o; o += align256(P * H * 2);
-  L.hperm = o; o += align256(P * I * 4);
-  L.h16 = o; o += align256(P * I * 2);
   L.dperm = o; o += align256(P * H * 4);
+  if (mx) {
+    L.tile_first = o; o += align256(F * 4);
+    L.tile_cnt = o; o += align256(F * 4);
+    L.exp_tile0 = o; o += align256((size_t)E * 4);
+    L.rtile = o; o += align256(P * 4);
+    L.xq = o; o += align256(2 * P * H);
+    L.sfx = o; o += align256(F * (H / kXK) * 2 * kSfAtom);
+    L.gu = o; o += align256(P * 2 * I * 4);
+    L.hq = o; o += align256(3 * P * I);
+    L.sfh = o; o += align256(F * (I / kXK) * 2 * kSfAtom);
+  } else {
+    L.xshift = o; o += align256(P * 4);
+    L.hshift = o; o += align256(P * 4);
+    L.xperm = o; o += align256(P * H * 2);
+    L.hperm = o; o += align256(P * I * 4);
+    L.h16 = o; o += align256(P * I * 2);
+  }
   L.total = o;
   return L;
 }
 
-size_t group_workspace_bytes(int T, int k, int E, int H, int I) { return g_layout(T, k, E, H, I).total; }
+static bool g_mx(const qk_moe_layer* L) { return gmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter); }
 
-static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I) {
-  const GWsLayout L = g_layout(T, k, E, H, I);
+size_t group_workspace_bytes(const qk_moe_layer* L, int T, int k) {
+  return g_layout(T, k, L->gate.n_experts, L->hidden, L->inter, g_mx(L)).total;
+}
+
+static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I, bool mx) {
+  const GWsLayout L = g_layout(T, k, E, H, I, mx);
   uint8_t* p = static_cast<uint8_t*>(ws);
-  GroupWs W;
+  GroupWs W = {};
   W.counts = reinterpret_cast<int*>(p + L.counts);
   W.n_tiles = reinterpret_cast<int*>(p + L.n_tiles);
   W.n_flush = reinterpret_cast<unsigned long long*>(p + L.n_flush);
@@ -690,12 +696,24 @@ static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I) {
   W.tile_row0 = reinterpret_cast<int*>(p + L.tile_row0);
   W.tile_n = reinterpret_cast<int*>(p + L.tile_n);
   W.inv = reinterpret_cast<int*>(p + L.inv);
-  W.xshift = reinterpret_cast<int*>(p + L.xshift);
-  W.hshift = reinterpret_cast<int*>(p + L.hshift);
-  W.xperm = reinterpret_cast<__half*>(p + L.xperm);
-  W.hperm = reinterpret_cast<float*>(p + L.hperm);
-  W.h16 = reinterpret_cast<__half*>(p + L.h16);
   W.dperm = reinterpret_cast<float*>(p + L.dperm);
+  if (mx) {
+    W.tile_first = reinterpret_cast<int*>(p + L.tile_first);
+    W.tile_cnt = reinterpret_cast<int*>(p + L.tile_cnt);
+    W.exp_tile0 = reinterpret_cast<int*>(p + L.exp_tile0);
+    W.rtile = reinterpret_cast<int*>(p + L.rtile);
+    W.xq = p + L.xq;
+    W.sfx = p + L.sfx;
+    W.gu = reinterpret_cast<float*>(p + L.gu);
+    W.hq = p + L.hq;
+    W.sfh = p + L.sfh;
+  } else {
+    W.xshift = reinterpret_cast<int*>(p + L.xshift);
+    W.hshift = reinterpret_cast<int*>(p + L.hshift);
+    W.xperm = reinterpret_cast<__half*>(p + L.xperm);
+    W.hperm = reinterpret_cast<float*>(p + L.hperm);
+    W.h16 = reinterpret_cast<__half*>(p + L.h16);
+  }
   return W;
 }
 
@@ -742,10 +760,18 @@ static qk_status g_dispatch(const GemmArgs& A, cudaStream_t st) {
 
 qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
   const int T = a.T, k = a.k, E = a.E, H = a.H, I = a.I, P = a.P;
-  GroupWs W = g_carve(workspace, T, k, E, H, I);
+  const bool mx = gmx_eligible(a.gate, a.up, a.down, H, I);
+  GroupWs W = g_carve(workspace, T, k, E, H, I, mx);
   if (cudaMemsetAsync(W.counts, 0, W.zero_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
   k_grp_count<<<(P + 255) / 256, 256, 0, st>>>(a.ids, P, E, W.counts);
-  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, E);
+  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, E, mx ? kXN : kGN, mx ? 1 : 0);
+  if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
+  if (mx) {
+    const qk_status rc = gmx_forward(a, W, st);
+    if (rc != QK_OK) return rc;
+    k_grp_combine<<<T, 256, 0, st>>>(W, a.w, k, H, a.y, a.y_bf16);
+    return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  }
   k_grp_scatter<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
 

@@ -32,7 +32,7 @@ struct DecodeArgs {
 
 qk_status decode_forward(DecodeArgs args, cudaStream_t st);
 // Grouped (prefill) path: pairs grouped by expert, tcgen05 grouped GEMMs.
-size_t group_workspace_bytes(int T, int k, int E, int H, int I);
+size_t group_workspace_bytes(const qk_moe_layer* L, int T, int k);
 qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
 size_t decode_workspace_bytes(int T, int k, int H, int I);
 void decode_carve(DecodeArgs& a, void* ws);

@@ -14,10 +14,10 @@ namespace qk {
 namespace {
 
 struct Key {
-  int dtype, rank, swizzle;
+  int dtype, rank, swizzle, l2promo;
   const void* base;
-  uint64_t dims[3], strides[2];
-  uint32_t box[3];
+  uint64_t dims[4], strides[3];
+  uint32_t box[4];
   bool operator==(const Key& o) const { return std::memcmp(this, &o, sizeof(Key)) == 0; }
 };
 
@@ -36,12 +36,13 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 }  // namespace
 
 bool tmap_get(CUtensorMap* out, int dtype, int rank, const void* base, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box, int swizzle) {
+              const uint64_t* strides_bytes, const uint32_t* box, int swizzle, int l2promo) {
   Key k;
   std::memset(&k, 0, sizeof(k));
   k.dtype = dtype;
   k.rank = rank;
   k.swizzle = swizzle;
+  k.l2promo = l2promo;
   k.base = base;
   for (int i = 0; i < rank; ++i) {
     k.dims[i] = dims[i];
@@ -63,8 +64,8 @@ bool tmap_get(CUtensorMap* out, int dtype, int rank, const void* base, const uin
       return false;
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   }
-  cuuint64_t d[3], s[2];
-  cuuint32_t b[3], es[3] = {1, 1, 1};
+  cuuint64_t d[4], s[3];
+  cuuint32_t b[4], es[4] = {1, 1, 1, 1};
   for (int i = 0; i < rank; ++i) {
     d[i] = dims[i];
     b[i] = box[i];
@@ -73,7 +74,7 @@ bool tmap_get(CUtensorMap* out, int dtype, int rank, const void* base, const uin
   CUtensorMap m;
   const CUresult r = g_encode(&m, (CUtensorMapDataType)dtype, rank, const_cast<void*>(base), d, s,
                               b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)swizzle,
-                              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                              (CUtensorMapL2promotion)l2promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
   Entry& e = g_cache[g_next];
   g_next = (g_next + 1) % kCache;

@@ -98,3 +98,45 @@ def test_grouped_path_bf16_output_and_skewed_groups():
                  torch.bfloat16)
     yo = oracle_moe(wl, 6, 0, x, ids, w.astype(np.float32).astype(np.float64))
     assert_parity(y.float().cpu().numpy(), yo, what="grouped bf16 y")
+
+
+def test_mx_block_scaled_path():
+    """All-MXFP4 layer with hidden and inter multiples of 512: the grouped
+    path runs on the block-scaled tensor cores (e2m1 weights as stored, x as
+    two e4m3 terms, h as three).  48 tokens x top-4 over 16 experts."""
+    wl = synth.Workload("mid", 16, 4, 1024, 512, 48, 118, 127)
+    layer = workload.make_layer(wl, 8, 0)
+    x = synth.activations(8, wl.T, wl.H)
+    lg = synth.router_logits(8, wl.T, wl.E)
+    oids, ow = oracle.route_topk(lg, wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
+    yo = oracle_moe(wl, 8, 0, x, oids, ow.astype(np.float32).astype(np.float64))
+    assert_parity(y.cpu().numpy(), yo, what="mx block-scaled")
+
+
+def test_mx_path_skewed_groups_wide_exponents():
+    """Block-scaled path, 300 tokens all routed to experts 1 and 6: three
+    token tiles per expert (128, 128, 44 rows), one 512-element K chunk
+    (hidden 512), e8m0 codes spanning 2^-40 .. 2^10, bf16 y."""
+    wl = synth.Workload("wide", 8, 2, 512, 512, 300, 87, 137)
+    layer = workload.make_layer(wl, 9, 0)
+    x = synth.activations(9, wl.T, wl.H)
+    ids = np.array([[1, 6]] * wl.T, np.int32)
+    w = np.tile(np.array([[0.7, 0.3]]), (wl.T, 1))
+    y = _forward(layer, x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).float().cuda(),
+                 torch.bfloat16)
+    yo = oracle_moe(wl, 9, 0, x, ids, w.astype(np.float32).astype(np.float64))
+    assert_parity(y.float().cpu().numpy(), yo, what="mx skewed wide exponents")
+
+
+def test_mx_path_many_small_groups():
+    """Block-scaled path, 96 tokens x top-8 over 64 experts (groups of a few
+    rows: 32-row token boxes), hidden 2048, inter 1024."""
+    wl = synth.Workload("small_groups", 64, 8, 2048, 1024, 96, 118, 127)
+    layer = workload.make_layer(wl, 10, 0)
+    x = synth.activations(10, wl.T, wl.H)
+    lg = synth.router_logits(10, wl.T, wl.E)
+    oids, ow = oracle.route_topk(lg, wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
+    yo = oracle_moe(wl, 10, 0, x, oids, ow.astype(np.float32).astype(np.float64))
+    assert_parity(y.cpu().numpy(), yo, what="mx many small groups")
