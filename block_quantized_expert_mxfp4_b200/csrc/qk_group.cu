@@ -63,9 +63,11 @@ __global__ void k_grp_count(const int32_t* __restrict__ ids, int P, int E, int* 
 
 // One block: exclusive scans of the per-expert pair counts and token-tile
 // counts; writes the token-tile list.
-// Token tiles hold at most tn rows; with `mx`, also the per-tile expert
-// extent (first tile, tile count) and each expert's first tile.
-__global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, int E, int tn, int mx) {
+// One block: the tile list L of tiles of at most tn rows (with `mx`, also
+// each tile's expert extent and each expert's first tile); `first` also
+// writes the experts' first sorted rows and resets the scatter cursors.
+__global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, TileList L, int E, int tn, int mx,
+                                                            int first) {
   __shared__ int s_pairs[kScanThreads / 32], s_tiles[kScanThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (E + kScanThreads - 1) / kScanThreads;
@@ -108,24 +110,26 @@ __global__ void __launch_bounds__(kScanThreads) k_grp_scan(GroupWs W, int E, int
   int tile = it - nt + (warp ? s_tiles[warp - 1] : 0);
   for (int e = e0; e < e1; ++e) {
     const int c = W.counts[e];
-    const int first = tile, cnt = (c + tn - 1) / tn;
-    W.offsets[e] = row;
-    W.fill[e] = 0;
-    if (mx) W.exp_tile0[e] = first;
+    const int t0 = tile, cnt = (c + tn - 1) / tn;
+    if (first) {
+      W.offsets[e] = row;
+      W.fill[e] = 0;
+    }
+    if (mx) L.exp_tile0[e] = t0;
     for (int r = 0; r < c; r += tn, ++tile) {
-      W.tile_e[tile] = e;
-      W.tile_row0[tile] = row + r;
-      W.tile_n[tile] = min(tn, c - r);
+      L.tile_e[tile] = e;
+      L.tile_row0[tile] = row + r;
+      L.tile_n[tile] = min(tn, c - r);
       if (mx) {
-        W.tile_first[tile] = first;
-        W.tile_cnt[tile] = cnt;
+        L.tile_first[tile] = t0;
+        L.tile_cnt[tile] = cnt;
       }
     }
     row += c;
   }
   if (tid == kScanThreads - 1) {
-    W.offsets[E] = row;
-    *W.n_tiles = tile;
+    if (first) W.offsets[E] = row;
+    *L.n_tiles = tile;
   }
 }
 
@@ -338,7 +342,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem;
-  const int n_tiles = *W.n_tiles * MB;
+  const int n_tiles = *W.L1.n_tiles * MB;
   // Bounded wait; the first one that runs out stops every role of the block.
   auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
     if (*reinterpret_cast<volatile int*>(&S.abort)) return false;
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
       int n = 0;
       for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x) {
         const int f = t / MB, mb = t - f * MB;
-        const int wrow = W.tile_e[f] * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128);
+        const int wrow = W.L1.tile_e[f] * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128);
         for (int k0 = 0; k0 < nks; k0 += kGRK, ++n) {
           const int s = n % kGRS;
           if (n >= kGRS && !wait(&S.rempty[s], (uint32_t)((n / kGRS - 1) & 1))) break;
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
       int n = 0;
       for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x) {
         const int f = t / MB;
-        const int row0 = W.tile_row0[f], bi = box_index(W.tile_n[f]);
+        const int row0 = W.L1.tile_row0[f], bi = box_index(W.L1.tile_n[f]);
         const int nbox = 32 << bi, kpb = kGN / nbox;  // reduction steps per token stage
         for (int k0 = 0; k0 < nks; k0 += kpb, ++n) {
           const int s = n % kGBS, nsub = min(kpb, nks - k0);
@@ -397,7 +401,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
       int na = 0, nb = 0, i = 0;
       for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x, ++i) {
         const int f = t / MB;
-        const int nbox = 32 << box_index(W.tile_n[f]), kpb = kGN / nbox;
+        const int nbox = 32 << box_index(W.L1.tile_n[f]), kpb = kGN / nbox;
         const uint32_t idesc = umma_idesc_f16(kGM, nbox);
         const int ab = i & 1;  // accumulator buffer
         if (i >= 2 && !wait(&S.acc_empty[ab], (uint32_t)((i / 2 - 1) & 1))) break;
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
     const bool vec = nvq > 0 && nvq <= kScV;
     auto scale_row = [&](int tt) {
       const int f = tt / MB, mb = tt - f * MB;
-      const int wrow = W.tile_e[f] * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128) + wr_in_tile;
+      const int wrow = W.L1.tile_e[f] * G.rows_per_e + (GATEUP ? mb * 64 : mb * 128) + wr_in_tile;
       return WR.scales + (size_t)wrow * sc_len;
     };
     uint4 pre[kScV];
@@ -568,7 +572,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
     int i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
       const int f = t / MB, mb = t - f * MB;
-      const int e = W.tile_e[f], row0 = W.tile_row0[f], nrow = W.tile_n[f];
+      const int e = W.L1.tile_e[f], row0 = W.L1.tile_row0[f], nrow = W.L1.tile_n[f];
       const int ab = i & 1;
       if (!__all_sync(0xffffffffu, wait(&S.acc_full[ab], (uint32_t)((i / 2) & 1)) &&
                                        wait(&S.cref_full[i & 3], (uint32_t)((i / 4) & 1))))
@@ -630,41 +634,40 @@ namespace qk {
 
 // ================================================================= host ==
 struct GWsLayout {
-  size_t counts, offsets, fill, tile_e, tile_row0, tile_n, n_tiles, n_flush, zero_end;
-  size_t inv, dperm, xshift, hshift, xperm, hperm, h16;
-  size_t tile_first, tile_cnt, exp_tile0, rtile, xq, sfx, gu, hq, sfh, total;
+  size_t counts, n_tiles1, n_tiles2, n_flush, zero_end, offsets, fill, inv, dperm;
+  size_t t1[5], t2[5], exp1, exp2;  // tile_e, tile_row0, tile_n, tile_first, tile_cnt
+  size_t xshift, hshift, xperm, hperm, h16;
+  size_t rtile2, xt, sfx, gu, ht, sfh, total;
 };
-
-static int g_max_tiles(int P, int E, int tn) { return P / tn + E + 1; }
 
 // Workspace of the grouped path; `mx` selects the MXFP4 block-scaled buffers
 // instead of the f16 ones.
 static GWsLayout g_layout(int T, int k, int E, int H, int I, bool mx) {
-  const size_t P = (size_t)T * k, F = (size_t)g_max_tiles((int)P, E, mx ? kXN : kGN);
+  const size_t P = (size_t)T * k;
+  const size_t F1 = (size_t)g_max_tiles((int)P, E, mx ? kXTok1 : kGN), F2 = (size_t)g_max_tiles((int)P, E, kXTok2);
   GWsLayout L = {};
   size_t o = 0;
   L.counts = o; o += (size_t)E * 4;          // zeroed on every call: counts .. n_flush
-  L.n_tiles = o; o += 8;
+  L.n_tiles1 = o; o += 8;
+  L.n_tiles2 = o; o += 8;
   L.n_flush = o; o += 8;
   L.zero_end = o;
   o = align256(o);
   L.offsets = o; o += align256((size_t)(E + 1) * 4);
   L.fill = o; o += align256((size_t)E * 4);
-  L.tile_e = o; o += align256(F * 4);
-  L.tile_row0 = o; o += align256(F * 4);
-  L.tile_n = o; o += align256(F * 4);
   L.inv = o; o += align256(P * 4);
   L.dperm = o; o += align256(P * H * 4);
+  for (int i = 0; i < (mx ? 5 : 3); ++i) { L.t1[i] = o; o += align256(F1 * 4); }
   if (mx) {
-    L.tile_first = o; o += align256(F * 4);
-    L.tile_cnt = o; o += align256(F * 4);
-    L.exp_tile0 = o; o += align256((size_t)E * 4);
-    L.rtile = o; o += align256(P * 4);
-    L.xq = o; o += align256(2 * P * H);
-    L.sfx = o; o += align256(F * (H / kXK) * 2 * kSfAtom);
+    for (int i = 0; i < 5; ++i) { L.t2[i] = o; o += align256(F2 * 4); }
+    L.exp1 = o; o += align256((size_t)E * 4);
+    L.exp2 = o; o += align256((size_t)E * 4);
+    L.rtile2 = o; o += align256(P * 4);
+    L.xt = o; o += align256(F1 * (H / kXK) * kXBlock);
+    L.sfx = o; o += align256(F1 * (H / kXK) * kSfAtom);
     L.gu = o; o += align256(P * 2 * I * 4);
-    L.hq = o; o += align256(3 * P * I);
-    L.sfh = o; o += align256(F * (I / kXK) * 2 * kSfAtom);
+    L.ht = o; o += align256(F2 * (I / kXK) * kXBlock);
+    L.sfh = o; o += align256(F2 * (I / kXK) * kSfAtom);
   } else {
     L.xshift = o; o += align256(P * 4);
     L.hshift = o; o += align256(P * 4);
@@ -682,30 +685,39 @@ size_t group_workspace_bytes(const qk_moe_layer* L, int T, int k) {
   return g_layout(T, k, L->gate.n_experts, L->hidden, L->inter, g_mx(L)).total;
 }
 
+static TileList g_list(uint8_t* p, const size_t (&t)[5], size_t exp, size_t n_tiles, bool mx) {
+  TileList L = {};
+  L.tile_e = reinterpret_cast<int*>(p + t[0]);
+  L.tile_row0 = reinterpret_cast<int*>(p + t[1]);
+  L.tile_n = reinterpret_cast<int*>(p + t[2]);
+  if (mx) {
+    L.tile_first = reinterpret_cast<int*>(p + t[3]);
+    L.tile_cnt = reinterpret_cast<int*>(p + t[4]);
+    L.exp_tile0 = reinterpret_cast<int*>(p + exp);
+  }
+  L.n_tiles = reinterpret_cast<int*>(p + n_tiles);
+  return L;
+}
+
 static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I, bool mx) {
   const GWsLayout L = g_layout(T, k, E, H, I, mx);
   uint8_t* p = static_cast<uint8_t*>(ws);
   GroupWs W = {};
   W.counts = reinterpret_cast<int*>(p + L.counts);
-  W.n_tiles = reinterpret_cast<int*>(p + L.n_tiles);
   W.n_flush = reinterpret_cast<unsigned long long*>(p + L.n_flush);
   W.zero_bytes = L.zero_end - L.counts;
   W.offsets = reinterpret_cast<int*>(p + L.offsets);
   W.fill = reinterpret_cast<int*>(p + L.fill);
-  W.tile_e = reinterpret_cast<int*>(p + L.tile_e);
-  W.tile_row0 = reinterpret_cast<int*>(p + L.tile_row0);
-  W.tile_n = reinterpret_cast<int*>(p + L.tile_n);
   W.inv = reinterpret_cast<int*>(p + L.inv);
   W.dperm = reinterpret_cast<float*>(p + L.dperm);
+  W.L1 = g_list(p, L.t1, L.exp1, L.n_tiles1, mx);
   if (mx) {
-    W.tile_first = reinterpret_cast<int*>(p + L.tile_first);
-    W.tile_cnt = reinterpret_cast<int*>(p + L.tile_cnt);
-    W.exp_tile0 = reinterpret_cast<int*>(p + L.exp_tile0);
-    W.rtile = reinterpret_cast<int*>(p + L.rtile);
-    W.xq = p + L.xq;
+    W.L2 = g_list(p, L.t2, L.exp2, L.n_tiles2, true);
+    W.rtile2 = reinterpret_cast<int*>(p + L.rtile2);
+    W.xt = p + L.xt;
     W.sfx = p + L.sfx;
     W.gu = reinterpret_cast<float*>(p + L.gu);
-    W.hq = p + L.hq;
+    W.ht = p + L.ht;
     W.sfh = p + L.sfh;
   } else {
     W.xshift = reinterpret_cast<int*>(p + L.xshift);
@@ -764,7 +776,8 @@ qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
   GroupWs W = g_carve(workspace, T, k, E, H, I, mx);
   if (cudaMemsetAsync(W.counts, 0, W.zero_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
   k_grp_count<<<(P + 255) / 256, 256, 0, st>>>(a.ids, P, E, W.counts);
-  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, E, mx ? kXN : kGN, mx ? 1 : 0);
+  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L1, E, mx ? kXTok1 : kGN, mx ? 1 : 0, 1);
+  if (mx) k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L2, E, kXTok2, 1, 0);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
   if (mx) {
     const qk_status rc = gmx_forward(a, W, st);

@@ -9,20 +9,31 @@
 namespace qk {
 
 constexpr int kGN = 256;          // f16 path: token rows per tile (largest tcgen05 N)
-constexpr int kXN = 80;           // MXFP4 path: token rows per tile (terms x rows <= 240 MMA columns)
-constexpr int kXK = 128;          // MXFP4 path: reduction per stage (four 32-element scale blocks)
+constexpr int kXK = 128;          // MXFP4 path: reduction per step (four 32-element scale blocks)
+constexpr int kXTok1 = 64;        // MXFP4 path: tokens per gate/up tile (2 terms x 16 per TMEM lane quadrant)
+constexpr int kXTok2 = 40;        // MXFP4 path: tokens per down tile (3 terms x 10 per quadrant)
 constexpr int kSfAtom = 512;      // scale-factor atom: 128 rows x 4 blocks, tensor-memory copy layout
+constexpr int kXBlock = 128 * kXK;  // one reduction step of a token tile: 128 rows x 128 e4m3 (16 KB)
 constexpr int kScanThreads = 1024;
 constexpr int kRowThreads = 128;
+
+// Token tiles (<= tn rows of one expert's sorted rows).
+struct TileList {
+  int* tile_e;      // [F] expert of token tile f
+  int* tile_row0;   // [F] first sorted row of token tile f
+  int* tile_n;      // [F] rows in token tile f
+  int* tile_first;  // [F] first token tile of the expert of tile f (MXFP4 path)
+  int* tile_cnt;    // [F] token tiles of the expert of tile f (MXFP4 path)
+  int* exp_tile0;   // [E] first token tile of expert e (MXFP4 path)
+  int* n_tiles;     // [1] token tiles
+};
 
 struct GroupWs {
   int* counts;      // [E] pairs per expert
   int* offsets;     // [E + 1] first sorted row of each expert
   int* fill;        // [E] scatter cursors
-  int* tile_e;      // [F] expert of token tile f
-  int* tile_row0;   // [F] first sorted row of token tile f
-  int* tile_n;      // [F] rows in token tile f
-  int* n_tiles;     // [1] token tiles
+  TileList L1;      // f16 path: tiles of kGN rows; MXFP4 path: gate/up tiles of kXTok1 rows
+  TileList L2;      // MXFP4 path: down tiles of kXTok2 rows
   int* inv;         // [P] pair -> sorted row
   float* dperm;     // [P][H] fp32 down-projection result of each sorted row
   unsigned long long* n_flush;  // [1] MXFP4 blocks flushed by the relative scaling (f16 path)
@@ -33,16 +44,16 @@ struct GroupWs {
   __half* xperm;    // [P][H] f16
   float* hperm;     // [P][I] fp32
   __half* h16;      // [P][I] f16
-  // MXFP4 block-scaled path
-  int* tile_first;  // [F] first token tile of the expert of tile f
-  int* tile_cnt;    // [F] token tiles of the expert of tile f
-  int* exp_tile0;   // [E] first token tile of expert e
-  int* rtile;       // [P] per sorted row: (token tile << 8) | row within the tile
-  uint8_t* xq;      // [2][P][H] e4m3 terms of x (x = t0 * 2^s0 + t1 * 2^s1 per 32-block)
-  uint8_t* sfx;     // [F][H / 128][2][512] ue8m0 block scales of the stacked x terms, atom layout
+  // MXFP4 block-scaled path.  A token tile's operand per reduction step is a
+  // 128-row block (the tcgen05 A operand, 128-byte swizzled): row
+  // 32 q + n_t t + i holds term t of the tile's token n_t q + i (n_t = 16
+  // tokens per quadrant for x, 10 for h), and its 512-byte scale atom.
+  int* rtile2;      // [P] per sorted row: (down tile << 8) | row within it
+  uint8_t* xt;      // [F1][H / 128] blocks of the x terms (x = t0 2^s0 + t1 2^s1 per 32-block)
+  uint8_t* sfx;     // [F1][H / 128][512] ue8m0 scales of the x terms, atom layout
   float* gu;        // [P][2 I] fp32 gate (first I) and up (last I) projections
-  uint8_t* hq;      // [3][P][I] e4m3 terms of h = silu(gate) * up
-  uint8_t* sfh;     // [F][I / 128][2][512] ue8m0 block scales of the stacked h terms, atom layout
+  uint8_t* ht;      // [F2][I / 128] blocks of the 3 e4m3 terms of h = silu(gate) * up
+  uint8_t* sfh;     // [F2][I / 128][512] ue8m0 scales of the h terms, atom layout
 };
 
 // The MXFP4 block-scaled path takes a layer when all three projections are
@@ -51,7 +62,9 @@ struct GroupWs {
 bool gmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
 
 // x split, gate/up GEMM, h split, down GEMM of the MXFP4 path (the counting
-// sort has run; the combine follows).
+// sort and both tile lists are done; the combine follows).
 qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st);
+
+inline int g_max_tiles(int P, int E, int tn) { return P / tn + E + 1; }
 
 }  // namespace qk
