@@ -428,7 +428,8 @@ def run_prefill(args, rank, world, dev):
                 "peak_kind": peak_kind, "frac": round(wbytes / t / 1e9 / peak, 4)},
         "tensor": {"flop_per_layer": flops, "achieved_tflops": round(flops / t / 1e12, 1),
                    "peak_tflops": tpeak, "peak_kind": tkind, "frac": round(flops / t / 1e12 / tpeak, 4)},
-        "path": "group/permute, tcgen05 kind::f16 grouped GEMMs (gate/up+SwiGLU, down), combine",
+        "path": "counting sort by expert; x as 2 exact e4m3 terms; block-scaled tcgen05 grouped GEMMs "
+                "(e2m1 weights + e8m0 scales as stored): gate/up, SwiGLU + 3-term h split, down; combine",
     }
 
 

@@ -92,11 +92,17 @@ typedef struct qk_moe_layer {
  *  x_bf16    [T][hidden] bf16.        topk_ids [T][top_k] int32 in [0, E).
  *  topk_w    [T][top_k] fp32.         y        [T][hidden] fp32 (y_is_bf16=0) or bf16.
  *  act_quant QK_ACT_NONE.             workspace >= moe_expert_workspace_size(), 256-B aligned.
- * Shapes: hidden and inter multiples of 128; 1 <= top_k <= 8.  The decode
- * path (nibbles and scales decoded in registers, tensor-core m16n8k16
- * products, fp32 accumulation) takes up to floor(128/top_k) tokens per launch;
- * larger counts run as consecutive launches over slices of that many tokens,
- * in order, on `stream`.  T = 0 returns QK_OK and launches nothing.
+ * Shapes: hidden and inter multiples of 128; 1 <= top_k <= 8.  Up to
+ * floor(128/top_k) tokens run the decode kernels (nibbles and scales decoded
+ * in registers, tensor-core m16n8k16 products, fp32 accumulation).  More
+ * tokens run the grouped path ([REAP25] "What's actually different": one
+ * grouped GEMM per projection): the pairs are sorted by expert and each
+ * projection is a grouped tcgen05 GEMM -- on the block-scaled tensor cores
+ * with the e2m1 weights and e8m0 scales as stored and the activations as
+ * exact e4m3 terms when all three projections are MXFP4, hidden and inter
+ * are multiples of 512, q is 32-byte and scales 16-byte aligned; otherwise
+ * with the weights expanded to f16 on chip.  All kernels run in order on
+ * `stream`.  T = 0 returns QK_OK and launches nothing.
  * Errors: QK_ERR_INVALID_ARG (shapes, pointers, formats), QK_ERR_WORKSPACE,
  * QK_ERR_UNSUPPORTED (act_quant), QK_ERR_CUDA; device: QK_ERR_NAN_SCALE,
  * QK_ERR_INVALID_ARG (id out of range: that pair contributes nothing),
