@@ -137,7 +137,7 @@ def kernel_source_hash() -> str:
     """Hash of the decode kernels' sources (the kernel file and the headers it includes)."""
     from block_quantized_expert_mxfp4_b200 import build as b
     h = hashlib.sha256()
-    for n in ("qk_decode.cu", "qk_device.cuh", "qk_common.cuh", "qk_internal.h", "qk_tmap.h"):
+    for n in ("qk_decode.cu", "qk_route_table.cuh", "qk_device.cuh", "qk_common.cuh", "qk_internal.h", "qk_tmap.h"):
         h.update(open(os.path.join(b.CSRC, n), "rb").read())
     return h.hexdigest()[:16]
 

@@ -145,3 +145,58 @@ def test_large_activation_magnitudes():
     yo = oracle_moe(wl, 0, 0, x, ids, w.astype(np.float32).astype(np.float64))
     for t in range(2):
         assert_parity(y[t].cpu().numpy(), yo[t], what=f"scaled token {t}")
+
+
+# ---- larger decode cases: random routing at mid size, full virtual experts,
+# extreme activation magnitudes, determinism at full size ----
+
+def test_mx_decode_random_routing_mid_size():
+    """5 tokens, top-4 over 16 experts, hidden 1024, inter 1024."""
+    wl = synth.Workload("mxmid", 16, 4, 1024, 1024, 5, 118, 127)
+    y, yo = _e2e(wl, 5, (MX, MX, MX), seed=11)
+    assert_parity(y, yo, what="mx decode mid")
+
+
+def test_mx_decode_full_virtual_experts():
+    """16 tokens all routed to experts 3 and 12 (16 pairs each: two virtual
+    experts of 8 pairs per expert), unequal weights."""
+    wl = synth.Workload("mxhot", 16, 2, 1024, 1024, 16, 118, 127)
+    layer = workload.make_layer(wl, 12, 0)
+    x = synth.activations(12, 16, wl.H)
+    ids = np.array([[3, 12]] * 16, np.int32)
+    w = np.tile(np.array([[0.65, 0.35]]), (16, 1))
+    y = _run(layer, x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).float().cuda())
+    yo = oracle_moe(wl, 12, 0, x, ids, w.astype(np.float32).astype(np.float64))
+    assert_parity(y.cpu().numpy(), yo, what="mx hot experts")
+
+
+def test_mx_decode_extreme_activations():
+    """Token rows scaled by 2^40 and 2^-40: the per-row power-of-two staging
+    follows each row's own range."""
+    wl = synth.Workload("mxext", 16, 2, 1024, 1024, 2, 118, 127)
+    layer = workload.make_layer(wl, 13, 0)
+    x = synth.activations(13, 2, wl.H).float()
+    x[0] *= 2.0 ** 40
+    x[1] *= 2.0 ** -40
+    x = x.to(torch.bfloat16)
+    ids = np.array([[1, 9], [9, 4]], np.int32)
+    w = np.array([[0.5, 0.5], [0.2, 0.8]])
+    y = _run(layer, x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).float().cuda())
+    yo = oracle_moe(wl, 13, 0, x, ids, w.astype(np.float32).astype(np.float64))
+    for t in range(2):
+        assert_parity(y[t].cpu().numpy(), yo[t], what=f"mx extreme token {t}")
+
+
+def test_mx_decode_deterministic():
+    """MXFP4 at full size: the last unit of each output row tile forms y in
+    slot order, so repeated calls give identical bytes."""
+    wl = synth.WORKLOADS["decode_mx"]
+    layer = workload.make_layer(wl, 0, 0)
+    x = synth.activations(14, 3, wl.H).cuda()
+    lg = synth.router_logits(14, 3, wl.E).cuda()
+    ids = torch.empty((3, 6), dtype=torch.int32, device="cuda")
+    w = torch.empty((3, 6), device="cuda")
+    qk.moe_route_topk(lg, 6, ids, w)
+    a = _run(layer, x, ids, w)
+    b = _run(layer, x, ids, w)
+    assert torch.equal(a.view(torch.int32), b.view(torch.int32))
