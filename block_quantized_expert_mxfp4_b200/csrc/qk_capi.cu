@@ -40,6 +40,8 @@ size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_
   if (layer_ok(L) != QK_OK || n_tokens < 0 || top_k < 1 || top_k > 8) return 0;
   if (n_tokens > decode_chunk(top_k))
     return group_workspace_bytes(L, n_tokens, top_k);
+  if (dmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter))
+    return dmx_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
   return decode_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
 }
 
@@ -73,6 +75,9 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
   a.y_bf16 = y_is_bf16 ? 1 : 0;
   // Token counts above one decode launch's routing capacity take the grouped path.
   if (n_tokens > decode_chunk(top_k)) return group_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
+  // All-MXFP4 layers: weights straight to the block-scaled tensor cores.
+  if (dmx_eligible(a.gate, a.up, a.down, a.H, a.I))
+    return dmx_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
   decode_carve(a, workspace);
   return decode_forward(a, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -34,6 +34,10 @@ qk_status decode_forward(DecodeArgs args, cudaStream_t st);
 // Grouped (prefill) path: pairs grouped by expert, tcgen05 grouped GEMMs.
 size_t group_workspace_bytes(const qk_moe_layer* L, int T, int k);
 qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
+// Decode path for all-MXFP4 layers on the block-scaled tensor cores.
+bool dmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
+size_t dmx_workspace_bytes(int T, int k, int H, int I);
+qk_status dmx_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
 size_t decode_workspace_bytes(int T, int k, int H, int I);
 void decode_carve(DecodeArgs& a, void* ws);
 

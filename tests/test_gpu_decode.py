@@ -78,10 +78,12 @@ def test_nv_converted_equals_mx_output_closely():
     w = torch.full((4, 6), 1 / 6, device="cuda")
     a = _run(mx, x, ids, w).cpu().numpy()
     b = _run(nv, x, ids, w).cpu().numpy()
-    # Both paths accumulate in fp32 but associate differently (MXFP4 scales each
-    # block's partial, NVFP4 folds the scale into the f16 operand), so they agree
-    # to fp32 rounding, not bit for bit.
-    assert_parity(b, a, tol=1e-4, cos=0.9999999, what="nv vs mx")
+    # The conversion is lossless, so both layers hold the same weights.  The
+    # MXFP4 layer runs on the block-scaled tensor cores (x exact as two e4m3
+    # terms, h to 2^-12 as three); the NVFP4 layer on the f16 path (h rounded
+    # to f16 after a row shift, 2^-11).  They differ by at most the two paths'
+    # own errors against the exact result (about 2e-4 and 2e-5 measured).
+    assert_parity(b, a, tol=5e-4, cos=0.9999999, what="nv vs mx")
 
 
 @pytest.mark.parametrize("fmts", [(MX, NV, MX), (NV, MX, NV), (NV, NV, MX)])
@@ -151,10 +153,12 @@ def test_large_activation_magnitudes():
 # extreme activation magnitudes, determinism at full size ----
 
 def test_mx_decode_random_routing_mid_size():
-    """5 tokens, top-4 over 16 experts, hidden 1024, inter 1024."""
+    """5 tokens, top-4 over 16 experts, hidden 1024, inter 1024 (the
+    block-scaled decode path)."""
     wl = synth.Workload("mxmid", 16, 4, 1024, 1024, 5, 118, 127)
     y, yo = _e2e(wl, 5, (MX, MX, MX), seed=11)
-    assert_parity(y, yo, what="mx decode mid")
+    e, _ = assert_parity(y, yo, what="mx decode mid")
+    assert e < 1e-4  # x exact as two e4m3 terms, h to 2^-12 as three
 
 
 def test_mx_decode_full_virtual_experts():
@@ -171,8 +175,8 @@ def test_mx_decode_full_virtual_experts():
 
 
 def test_mx_decode_extreme_activations():
-    """Token rows scaled by 2^40 and 2^-40: the per-row power-of-two staging
-    follows each row's own range."""
+    """Token rows scaled by 2^40 and 2^-40: the per-32 ue8m0 scales of the
+    activation terms follow each block's own range."""
     wl = synth.Workload("mxext", 16, 2, 1024, 1024, 2, 118, 127)
     layer = workload.make_layer(wl, 13, 0)
     x = synth.activations(13, 2, wl.H).float()
