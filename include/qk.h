@@ -123,7 +123,8 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
  * embedded in a runtime that owns every device allocation).
  *  Arguments as moe_expert_forward.  The call needs
  *  moe_expert_workspace_size(L, n_tokens, top_k) <= 4 MiB (hidden 4096,
- *  inter 2048: up to 28 pairs per launch); larger requests return
+ *  inter 2048: up to 42 pairs per launch for an all-MXFP4 layer on the
+ *  block-scaled decode kernels, 28 for other layers); larger requests return
  *  QK_ERR_WORKSPACE and launch nothing.  Nothing in the array has to start at
  *  zero.  The array is shared by every call on a device: calls that overlap on
  *  the GPU (other streams, other host threads) race on it and must not be

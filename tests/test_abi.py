@@ -59,6 +59,35 @@ def test_workspace_query_and_shape_validation():
     assert L.moe_expert_workspace_size(ctypes.byref(nv), 1, 6) == 0
 
 
+def test_workspace_query_follows_the_path_choice():
+    """All-MXFP4 layers with 32-byte aligned weights take the block-scaled
+    decode and grouped paths (their own workspace layouts); the same layer
+    with misaligned weights, or in NVFP4, takes the f16 paths, whose
+    workspace depends on the shapes only."""
+    L = qk.load()
+    mx = _fake_layer()
+    nv = _fake_layer(fmts=(2, 2, 2))
+    mis = _fake_layer()
+    mis.gate.q = mis.gate.q + 16  # 16-byte aligned, not 32: no block-scaled path
+    for T in (1, 16, 100):         # decode (<= 21 tokens at top-6) and grouped
+        a, b, c = (L.moe_expert_workspace_size(ctypes.byref(x), T, 6) for x in (mx, nv, mis))
+        assert a > 0 and b > 0
+        assert c == b and a != b, (T, a, b, c)
+
+
+def test_noalloc_limit_in_pairs():
+    """4 MiB of fixed scratch: at hidden 4096, inter 2048 the block-scaled
+    MXFP4 decode needs 96 KiB per pair (42 pairs fit), the f16 decode more
+    (28 pairs)."""
+    L = qk.load()
+    mx, nv = _fake_layer(), _fake_layer(fmts=(2, 2, 2))
+    cap = 4 << 20
+    q = lambda lay, T, k: L.moe_expert_workspace_size(ctypes.byref(lay), T, k)
+    assert q(mx, 7, 6) <= cap < q(mx, 8, 6)        # 42 pairs fit, 48 do not
+    assert q(mx, 21, 2) <= cap < q(mx, 22, 2)      # 42 / 44
+    assert q(nv, 14, 2) <= cap < q(nv, 15, 2)      # 28 / 30
+
+
 def test_forward_argument_errors_are_synchronous():
     L = qk.load()
     lay = _fake_layer()
