@@ -274,9 +274,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
     if (*reinterpret_cast<volatile int*>(&S.abort)) return false;
     if (mbar_wait_bounded(bar, parity, limit)) return true;
     set_status(QK_ERR_TIMEOUT);
-    if (atomicExch(&S.abort, 1) == 0 && lane == 0)
-      printf("k_gmx<%d> timeout: block %d warp %d barrier byte %d parity %u tiles %d\n", GATEUP ? 1 : 0,
-             (int)blockIdx.x, warp, (int)((uint8_t*)bar - (uint8_t*)&S), parity, n_tiles);
+    *reinterpret_cast<volatile int*>(&S.abort) = 1;
     return false;
   };
   auto aborted = [&]() { return *reinterpret_cast<volatile int*>(&S.abort) != 0; };
