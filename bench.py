@@ -157,6 +157,17 @@ def recorded_traffic():
 
 
 # -------------------------------------------------------------- CPU oracle --
+def max_over_ranks(seconds: float, world: int, dev) -> float:
+    """The job's time: the largest of the ranks' device times (every rank
+    calls this at the same point; world 1 returns its own)."""
+    import torch
+    t = torch.tensor([seconds], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def oracle_sample(seconds: float, max_steps: int = 1 << 30):
     """Time the CPU oracle on (token, expert) pairs of the decode workload.
     Returns (bytes, seconds, steps, threads)."""
@@ -291,10 +302,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status {qk.status_string(st)}")
     elapsed = ev0.elapsed_time(ev1) / 1e3
     ffn_s = statistics.fmean(ffn_ms) / 1e3
-    t_max = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    elapsed_max = float(t_max.item())
+    elapsed_max = max_over_ranks(elapsed, world, dev)
     total_bytes = bytes_per_step * K * world
     value = total_bytes / elapsed_max / 1e9
 
@@ -321,10 +329,7 @@ def run_ours(args, rank, world, local_rank):
             yh.copy_(ys[l], non_blocking=True)
         e1.record(s)
         torch.cuda.synchronize()
-    e2e_t = torch.tensor([e0.elapsed_time(e1) / 1e3], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = bytes_per_step * E2 * world / float(e2e_t.item()) / 1e9
+    e2e_value = bytes_per_step * E2 * world / max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev) / 1e9
 
     peak, peak_kind = peaks()
     achieved = bytes_per_step / ffn_s / 1e9
@@ -409,10 +414,7 @@ def run_prefill(args, rank, world, dev):
             g.replay()
         e1.record(s)
         torch.cuda.synchronize()
-    t = torch.tensor([e0.elapsed_time(e1) / 1e3 / K], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    t = float(t.item())
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / K, world, dev)
     if qk.qk_last_device_status() != qk.QK_OK:
         raise RuntimeError("device status after prefill")
     peak, peak_kind = peaks()
