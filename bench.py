@@ -23,6 +23,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import re
 import os
 import statistics
 import sys
@@ -133,13 +134,23 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank lines: what the compiler sees
+    (string literals in these files hold no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(l.rstrip() for l in text.splitlines() if l.strip())
+
+
 def kernel_source_hash() -> str:
-    """Hash of the decode kernels' sources (the kernel file and the headers it includes)."""
+    """Hash of the decode kernels' code (the kernel file and the headers it
+    includes, comments excluded): a recorded DRAM traffic figure stays valid
+    while the code it was measured on is unchanged."""
     from block_quantized_expert_mxfp4_b200 import build as b
     h = hashlib.sha256()
     for n in ("qk_dmx.cu", "qk_route_table.cuh", "qk_device.cuh", "qk_common.cuh", "qk_group.cuh", "qk_internal.h",
               "qk_tmap.h"):
-        h.update(open(os.path.join(b.CSRC, n), "rb").read())
+        h.update(_code_only(open(os.path.join(b.CSRC, n)).read()).encode())
     return h.hexdigest()[:16]
 
 

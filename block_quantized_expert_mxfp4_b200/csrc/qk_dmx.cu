@@ -47,8 +47,8 @@ constexpr int kDKc = kDSteps * kXK;      // 1024 elements of K per unit
 constexpr int kDWS = 3;                  // weight stages
 constexpr int kDStageW = kDN * kXK;      // 16 KB (unpacked), 8 KB of packed weights
 constexpr int kDRows = 24;               // A rows per step block (terms x pairs <= 24)
-constexpr int kDABlock = kDRows * kXK;   // 4 KB
-constexpr int kDAUnit = kDSteps * kDABlock;  // 32 KB per unit
+constexpr int kDABlock = kDRows * kXK;   // 3 KB
+constexpr int kDAUnit = kDSteps * kDABlock;  // 24 KB per unit
 constexpr int kDThreads = 8 * 32;    // warp 0 weights, 1 MMA, 2 weight scales, 4 epilogue, 3 and 5-7 A builders
 constexpr int kDBuild = 4;           // A builder warps
 constexpr int kDTmemCols = 256;          // one 128-column accumulator; scales from 128
@@ -73,8 +73,8 @@ struct DmxHead {
   alignas(8) uint64_t aempty[2];
   alignas(8) uint64_t sfull[2];      // four steps' weight scale atoms written
   alignas(8) uint64_t sempty[2];
-  alignas(8) uint64_t acc_full[2];
-  alignas(8) uint64_t acc_empty[2];
+  alignas(8) uint64_t acc_full[2];   // [0]: the accumulator holds a finished unit
+  alignas(8) uint64_t acc_empty[2];  // [0]: the epilogue has read it ([1] unused)
   alignas(8) uint64_t drained;
   uint32_t tmem;
   int abort;
