@@ -469,7 +469,7 @@ def main():
         line = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
                 "n_gpus": 1, "steps": steps, "warmup": 0,
                 "ms_per_step": round(secs / max(steps, 1) * 1e3, 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 dequantized weights)",
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64 (exact dequantized weights)",
                 "data": "synthetic (seeded)",
                 "config": {"workload": WORKLOAD_DESC, "parallelism": "host cores"},
                 "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": thr,

@@ -148,7 +148,8 @@ class Layer:
 
 
 def dequant(w: Weight, e: int) -> np.ndarray:
-    out = np.empty((w.N, w.K), dtype=np.float32)
+    """Expert e's dequantized matrix [N][K], exact (float64)."""
+    out = np.empty((w.N, w.K), dtype=np.float64)
     cw = w.c()
     for n in range(w.N):
         _chk(lib().qko_dequant_row(ctypes.byref(cw), e, n, _p(out[n])))

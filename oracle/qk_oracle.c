@@ -87,7 +87,13 @@ static int nibble(const uint8_t* row_q, int32_t k) {
   return (k & 1) ? (b >> 4) : (b & 15);
 }
 
-int qko_dequant_row(const qko_weight* w, int32_t e, int32_t row, float* out) {
+/* The dequantized value is held in fp64, where it is exact for every code of
+ * every format: e2m1 (2 significant bits) x e8m0 (a power of two, 2^-127 ..
+ * 2^127) for MXFP4; e2m1 x e4m3 (4 bits) x an fp32 scale_2 (24 bits) for
+ * NVFP4, at most 30 significant bits and within fp64's exponent range.
+ * Rounding it to fp32 would change general NVFP4 weights (scale_2 not a power
+ * of two) and overflow MXFP4 codes >= 253. */
+int qko_dequant_row(const qko_weight* w, int32_t e, int32_t row, double* out) {
   int64_t r = (int64_t)e * w->rows + row;
   const uint8_t* rq = w->q + r * (w->cols / 2);
   int32_t k;
@@ -96,7 +102,7 @@ int qko_dequant_row(const qko_weight* w, int32_t e, int32_t row, float* out) {
     for (k = 0; k < w->cols; ++k) {
       uint8_t c = rs[k / 32];
       if (c == 255) return QKO_ERR_NAN_SCALE;
-      out[k] = (float)(qko_e2m1_value((uint8_t)nibble(rq, k)) * qko_e8m0_value(c));
+      out[k] = qko_e2m1_value((uint8_t)nibble(rq, k)) * qko_e8m0_value(c);
     }
     return QKO_OK;
   }
@@ -106,7 +112,7 @@ int qko_dequant_row(const qko_weight* w, int32_t e, int32_t row, float* out) {
     for (k = 0; k < w->cols; ++k) {
       uint8_t c = rs[k / 16];
       if ((c & 0x7F) == 0x7F) return QKO_ERR_NAN_SCALE;
-      out[k] = (float)(qko_e2m1_value((uint8_t)nibble(rq, k)) * qko_e4m3_value(c) * s2);
+      out[k] = qko_e2m1_value((uint8_t)nibble(rq, k)) * qko_e4m3_value(c) * s2;
     }
     return QKO_OK;
   }
@@ -193,7 +199,7 @@ static int matvec_rows(const qko_weight* w, int32_t e, const double* x, double* 
   int32_t n;
 #pragma omp parallel
   {
-    float* row = (float*)malloc(sizeof(float) * w->cols);
+    double* row = (double*)malloc(sizeof(double) * w->cols);
 #pragma omp for schedule(static)
     for (n = 0; n < w->rows; ++n) {
       int32_t k;
@@ -203,7 +209,7 @@ static int matvec_rows(const qko_weight* w, int32_t e, const double* x, double* 
         err = QKO_ERR_NAN_SCALE;
         continue;
       }
-      for (k = 0; k < w->cols; ++k) acc += (double)row[k] * x[k];
+      for (k = 0; k < w->cols; ++k) acc += row[k] * x[k];
       out[n] = acc;
     }
     free(row);
@@ -278,20 +284,20 @@ int qko_moe_forward(const qko_layer* L, const uint16_t* x_bf16, int32_t T,
 /* ------------------------------------------------------ FP8 block-128 --
  * Dense FP8 linear (IQ2XXS-Q2K-FP8 page: "FP8 E4M3, block-128, UE8M0
  * scales"): weight [N][K] e4m3 with one power-of-two scale per b x b tile,
- * scales [ceil(N/b)][ceil(K/b)].  dq = fp32(e4m3 * 2^(s-127)). */
+ * scales [ceil(N/b)][ceil(K/b)].  dq = e4m3 * 2^(s-127), exact in fp64. */
 static int fp8_linear_d(const double* x, int32_t M, int32_t K, const uint8_t* w,
                         const uint8_t* ws, int32_t N, int32_t b, double* y) {
   int32_t kb = (K + b - 1) / b, n, err = QKO_OK;
 #pragma omp parallel
   {
-    float* row = (float*)malloc(sizeof(float) * K);
+    double* row = (double*)malloc(sizeof(double) * K);
 #pragma omp for schedule(static)
     for (n = 0; n < N; ++n) {
       int32_t k, mm, bad = 0;
       for (k = 0; k < K; ++k) {
         uint8_t sc = ws[(int64_t)(n / b) * kb + k / b];
         if (sc == 255) bad = 1;
-        row[k] = (float)(qko_e4m3_value(w[(int64_t)n * K + k]) * qko_e8m0_value(sc));
+        row[k] = qko_e4m3_value(w[(int64_t)n * K + k]) * qko_e8m0_value(sc);
       }
       if (bad) {
 #pragma omp atomic write
@@ -300,7 +306,7 @@ static int fp8_linear_d(const double* x, int32_t M, int32_t K, const uint8_t* w,
       for (mm = 0; mm < M; ++mm) {
         double acc = 0.0;
         const double* xr = x + (int64_t)mm * K;
-        for (k = 0; k < K; ++k) acc += (double)row[k] * xr[k];
+        for (k = 0; k < K; ++k) acc += row[k] * xr[k];
         y[(int64_t)mm * N + n] = acc;
       }
     }

@@ -7,8 +7,8 @@
  * are the storage formats themselves.
  *
  * Everything here is the plain definition: decode every code to its value,
- * form fp32 dequantized weights, accumulate dot products in fp64, apply SwiGLU
- * in fp64, and sum the routed experts in slot order.  No blocking, fusion or
+ * form the dequantized weights exactly (fp64), accumulate dot products in
+ * fp64, apply SwiGLU in fp64, and sum the routed experts in slot order.  No blocking, fusion or
  * reordering beyond that.
  *
  * Sources (pages on DeepSeek-V4-Flash quantized checkpoints):
@@ -64,8 +64,8 @@ typedef struct {
   int32_t hidden, inter;
 } qko_layer;
 
-/* Dequantize one row of expert e to fp32. Returns QKO_ERR_NAN_SCALE on a NaN scale. */
-int qko_dequant_row(const qko_weight* w, int32_t e, int32_t row, float* out);
+/* Dequantize one row of expert e, exactly (fp64). Returns QKO_ERR_NAN_SCALE on a NaN scale. */
+int qko_dequant_row(const qko_weight* w, int32_t e, int32_t row, double* out);
 
 /* Scale-only MXFP4 -> NVFP4 conversion of one projection. */
 int qko_convert_mx_to_nv(const uint8_t* e8m0, int32_t E, int32_t N, int32_t K,

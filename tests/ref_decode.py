@@ -23,26 +23,27 @@ def unpack_nibbles(q):
 
 
 def dequant_mx(q, s):
-    """MXFP4 -> fp32 [.., N, K]: e2m1 * 2^(c-127) per 32-block (np.repeat on K)."""
+    """MXFP4 -> float64 [.., N, K]: e2m1 * 2^(c-127) per 32-block (np.repeat on K);
+    exact (2 significant bits times a power of two)."""
     codes = unpack_nibbles(q)
     scale = np.repeat(E8M0[np.asarray(s)], 32, axis=-1)
-    with np.errstate(over="ignore"):  # 6 * 2^127 overflows fp32, as it must
-        return (E2M1[codes] * scale).astype(np.float32)
+    return E2M1[codes] * scale
 
 
 def dequant_nv(q, s, s2):
-    """NVFP4 -> fp32: e2m1 * e4m3 per 16-block * per-expert scale_2."""
+    """NVFP4 -> float64: e2m1 * e4m3 per 16-block * per-expert fp32 scale_2;
+    exact (at most 2 + 4 + 24 significant bits)."""
     codes = unpack_nibbles(q)
     scale = np.repeat(E4M3[np.asarray(s)], 16, axis=-1)
-    s2 = np.asarray(s2, dtype=np.float64).reshape((-1,) + (1,) * (codes.ndim - 1))
-    with np.errstate(over="ignore"):
-        return (E2M1[codes] * scale * s2).astype(np.float32)
+    s2 = np.asarray(s2, dtype=np.float32).astype(np.float64)
+    s2 = s2.reshape((-1,) + (1,) * (codes.ndim - 1))
+    return E2M1[codes] * scale * s2
 
 
 def dequant_fp8(w, s, block=128):
     N, K = w.shape
     scale = np.kron(E8M0[np.asarray(s)], np.ones((block, block)))[:N, :K]
-    return (E4M3[np.asarray(w)] * scale).astype(np.float32)
+    return E4M3[np.asarray(w)] * scale
 
 
 def bf16_to_f64(x):

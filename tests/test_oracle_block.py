@@ -50,7 +50,7 @@ def test_worked_block_nv_view():
     assert [f"{c:02X}" for c in e4.reshape(-1)] == g["nv_e4m3"]
     dq_mx = oracle.dequant(_one_row_layer(q, s.reshape(-1)), 0)
     dq_nv = oracle.dequant(_one_row_layer(q, e4.reshape(-1), oracle.NVFP4, s2), 0)
-    assert np.array_equal(dq_mx.view(np.uint32), dq_nv.view(np.uint32))
+    assert np.array_equal(dq_mx.view(np.uint64), dq_nv.view(np.uint64))
 
 
 def test_worked_block_ffn_dot_through_expert_path():

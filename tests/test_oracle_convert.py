@@ -27,12 +27,12 @@ def test_lossless_when_span_le_17(lo, hi):
     assert bad == 0
     a = dequant_mx(q, s)
     b = dequant_nv(q, e4, s2)
-    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    assert np.array_equal(a.view(np.uint64), b.view(np.uint64))
     # and through the oracle's own dequant
     for e in range(3):
         da = oracle.dequant(oracle.Weight(oracle.MXFP4, q, s), e)
         db = oracle.dequant(oracle.Weight(oracle.NVFP4, q, e4, s2), e)
-        assert np.array_equal(da.view(np.uint32), db.view(np.uint32))
+        assert np.array_equal(da.view(np.uint64), db.view(np.uint64))
 
 
 def test_scale2_is_power_of_two_anchor_at_max():
