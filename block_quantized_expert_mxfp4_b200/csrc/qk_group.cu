@@ -441,6 +441,8 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
     const qk_weight& WR = rowB ? G.B : G.A;
     const int wr_in_tile = GATEUP ? (r >> 1) : r;
     const int sc_len = fr == QK_FMT_MXFP4 ? G.K / 32 : G.K / 16;
+    // NaN scale codes: e8m0 0xFF; e4m3 0x7F and 0xFF (the sign bit set first).
+    const uint32_t nan_or = fr == QK_FMT_MXFP4 ? 0u : 0x80808080u;
     // The next tile's scale rows are loaded into registers while this tile is
     // dequantized (two threads per row, 16-byte pieces).
     constexpr int kScV = 8;
@@ -464,7 +466,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
       // ---- the tile's scale rows, and (MXFP4) their largest code
       uint8_t* srow = sS + r * G.sc_stride;
-      uint32_t m4 = 0, ff = 0;  // byte-wise maxima; any 0xFF code
+      uint32_t m4 = 0, ff = 0;  // byte-wise maxima; any NaN code
       if (vec) {
 #pragma unroll
         for (int q = 0; q < kScV; ++q) {
@@ -476,8 +478,8 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
           d[2] = v.z;
           d[3] = v.w;
           m4 = __vmaxu4(m4, __vmaxu4(__vmaxu4(v.x, v.y), __vmaxu4(v.z, v.w)));
-          ff |= __vcmpeq4(v.x, 0xFFFFFFFFu) | __vcmpeq4(v.y, 0xFFFFFFFFu) | __vcmpeq4(v.z, 0xFFFFFFFFu) |
-                __vcmpeq4(v.w, 0xFFFFFFFFu);
+          ff |= __vcmpeq4(v.x | nan_or, 0xFFFFFFFFu) | __vcmpeq4(v.y | nan_or, 0xFFFFFFFFu) |
+                __vcmpeq4(v.z | nan_or, 0xFFFFFFFFu) | __vcmpeq4(v.w | nan_or, 0xFFFFFFFFu);
         }
         prefetch(t + gridDim.x);
       } else {
@@ -486,11 +488,11 @@ __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ 
           const uint32_t c = gsrc[b];
           srow[b] = (uint8_t)c;
           m4 = max(m4, c);
-          ff |= c == 255u ? 1u : 0u;
+          ff |= (c | (nan_or & 0x80u)) == 255u ? 1u : 0u;
         }
       }
       int cmax = (int)max(max(m4 & 0xFFu, (m4 >> 8) & 0xFFu), max((m4 >> 16) & 0xFFu, m4 >> 24));
-      if (fr == QK_FMT_MXFP4 && ff) set_status(QK_ERR_NAN_SCALE);
+      if (ff) set_status(QK_ERR_NAN_SCALE);
       cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));  // the row's two halves
       const int cref = fr == QK_FMT_MXFP4 ? min(cmax, 254) : 0;  // MXFP4 rows: relative to the row's max
       if (hh == 0) S.cref[i & 3][r] = (uint8_t)cref;

@@ -27,6 +27,11 @@ layer; expert intermediate 2048):
 * ``prefill``    E=256, k=6, H=4096, I=2048, T=2048, MXFP4, Zipf(s=1) routing
 * ``stack43``    43 layers, E=180, k=6, T=8, per-(layer, projection) MXFP4 or
   NVFP4, plus an FP8 E4M3 block-128 shared expert 4096x2048.
+
+General NVFP4 sources (not converted from MXFP4): the same nibble bytes, e4m3
+block-scale codes uniform in ``[NV_CODE_LO, NV_CODE_HI]`` (32 .. 448, every
+mantissa) and a per-expert fp32 ``scale_2`` in [2^-13, 2^-12) with a full
+24-bit significand, so neither scale is a power of two in general.
 """
 from __future__ import annotations
 
@@ -39,7 +44,8 @@ import torch
 __all__ = [
     "WORKLOADS", "Workload", "splitmix64_np", "splitmix64_torch", "tensor_key",
     "random_bytes", "scale_codes", "fp8_codes", "activations", "router_logits",
-    "zipf_logits", "format_choice", "TID",
+    "zipf_logits", "format_choice", "TID", "NV_CODE_LO", "NV_CODE_HI", "nv_scale_2",
+    "nv_expert_bytes", "mx_expert_bytes",
 ]
 
 _C0 = 0x9E3779B97F4A7C15
@@ -92,7 +98,7 @@ class TID:
     """Tensor ids: one independent stream per (layer, projection, kind)."""
 
     GATE, UP, DOWN, SH_GATE, SH_UP, SH_DOWN = range(6)
-    NIBBLES, SCALES = 0, 1
+    NIBBLES, SCALES, NV_SCALES, NV_SCALE_2 = 0, 1, 2, 3
 
     @staticmethod
     def of(layer: int, proj: int, kind: int) -> int:
@@ -235,3 +241,46 @@ def mx_expert_bytes(seed: int, layer: int, proj: int, E_rows: int, K: int, lo: i
         qs.append(random_bytes(seed, tq, nb, device, offset=e * nb).view(E_rows, K // 2))
         ss.append(scale_codes(seed, ts, ns, lo, hi, device, offset=e * ns).view(E_rows, K // 32))
     return torch.stack(qs), torch.stack(ss)
+
+
+NV_CODE_LO, NV_CODE_HI = 0x60, 0x7E  # e4m3 32 .. 448 (0x7F is NaN)
+
+
+def nv_scale_2(seed: int, layer: int, proj: int, n_experts: int) -> np.ndarray:
+    """fp32 ``scale_2`` [n_experts] of a general NVFP4 projection:
+    (2^23 + m) * 2^-36 with m the top 23 bits of word e of the projection's
+    stream, so every value lies in [2^-13, 2^-12) and is an exact fp32."""
+    key = tensor_key(seed, TID.of(layer, proj, TID.NV_SCALE_2))
+    w = _hash_words(key, 0, n_experts, "cpu").numpy().view(np.uint64)
+    m = (w >> np.uint64(41)).astype(np.float64)
+    return ((2.0 ** 23 + m) * 2.0 ** -36).astype(np.float32)
+
+
+def nv_expert_bytes(seed: int, layer: int, proj: int, E_rows: int, K: int,
+                    experts: Optional[Sequence[int]], n_experts: int, device="cpu",
+                    code_lo: int = NV_CODE_LO, code_hi: int = NV_CODE_HI):
+    """A general NVFP4 projection: nibble bytes [e][N][K/2] (the stream of the
+    MXFP4 bytes), e4m3 block-scale codes [e][N][K/16] uniform in
+    ``[code_lo, code_hi]`` and fp32 ``scale_2`` [e].
+
+    ``experts=None`` generates all ``n_experts``; otherwise only the listed ones
+    (same bytes as the full tensor's slices).
+    """
+    if not 0 <= code_lo <= code_hi <= 0x7E:
+        raise ValueError("e4m3 block-scale codes must lie in [0, 0x7E] (0x7F is NaN)")
+    nb = E_rows * K // 2
+    ns = E_rows * K // 16
+    tq = TID.of(layer, proj, TID.NIBBLES)
+    ts = TID.of(layer, proj, TID.NV_SCALES)
+    s2 = torch.from_numpy(nv_scale_2(seed, layer, proj, n_experts))
+    if experts is None:
+        q = random_bytes(seed, tq, n_experts * nb, device).view(n_experts, E_rows, K // 2)
+        s = scale_codes(seed, ts, n_experts * ns, code_lo, code_hi, device).view(
+            n_experts, E_rows, K // 16)
+        return q, s, s2.to(device)
+    qs, ss = [], []
+    for e in experts:
+        qs.append(random_bytes(seed, tq, nb, device, offset=e * nb).view(E_rows, K // 2))
+        ss.append(scale_codes(seed, ts, ns, code_lo, code_hi, device, offset=e * ns).view(
+            E_rows, K // 16))
+    return torch.stack(qs), torch.stack(ss), s2[list(experts)].to(device)

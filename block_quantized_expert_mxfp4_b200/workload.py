@@ -2,9 +2,10 @@
 
 Weights are generated on the GPU by the counter-based generator in ``synth``
 (the host can regenerate any expert's bytes independently); NVFP4 projections
-are produced from MXFP4 ones by the library's own scale-only conversion.  This
-module only allocates and fills tensors and calls the library; it computes
-nothing of the method itself.
+are produced from MXFP4 ones by the library's own scale-only conversion, or,
+for a general NVFP4 source, drawn directly (e4m3 block scales and scale_2 that
+are not powers of two).  This module only allocates and fills tensors and
+calls the library; it computes nothing of the method itself.
 """
 from __future__ import annotations
 
@@ -66,15 +67,29 @@ def to_nvfp4(p: Proj, stream=None) -> Proj:
     return Proj(_lib.QK_FMT_NVFP4, p.q, e4, s2, mx_scales=p.scales)
 
 
+def nv_proj(seed: int, layer: int, proj: int, E: int, rows: int, cols: int, codes,
+            device="cuda") -> Proj:
+    """A general NVFP4 projection; ``codes`` = (lo, hi) of its e4m3 block-scale codes."""
+    q, s, s2 = synth.nv_expert_bytes(seed, layer, proj, rows, cols, None, E, device, *codes)
+    return Proj(_lib.QK_FMT_NVFP4, q, s, s2)
+
+
 def make_layer(wl: synth.Workload, seed: int = 0, layer: int = 0, fmts=None,
-               device="cuda") -> DeviceLayer:
-    """One MoE layer of workload ``wl``; ``fmts`` = (gate, up, down) formats."""
+               device="cuda", nv_codes=None) -> DeviceLayer:
+    """One MoE layer of workload ``wl``; ``fmts`` = (gate, up, down) formats.
+
+    NVFP4 projections are the MXFP4 ones converted when ``nv_codes`` is None,
+    else general NVFP4 sources with e4m3 block-scale codes in ``nv_codes``.
+    """
     shapes = ((wl.I, wl.H), (wl.I, wl.H), (wl.H, wl.I))
     if fmts is None:
         f = _lib.QK_FMT_NVFP4 if wl.fmt == "nv" else _lib.QK_FMT_MXFP4
         fmts = (f, f, f)
     projs: List[Proj] = []
     for pi, ((rows, cols), fmt) in enumerate(zip(shapes, fmts)):
+        if fmt == _lib.QK_FMT_NVFP4 and nv_codes is not None:
+            projs.append(nv_proj(seed, layer, pi, wl.E, rows, cols, nv_codes, device))
+            continue
         p = mx_proj(seed, layer, pi, wl.E, rows, cols, wl.code_lo, wl.code_hi, device)
         projs.append(to_nvfp4(p) if fmt == _lib.QK_FMT_NVFP4 else p)
     return DeviceLayer(*projs)

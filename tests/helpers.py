@@ -14,12 +14,18 @@ TOL_REL = 5e-3      # max|gpu - oracle| / max|oracle|
 TOL_COS = 0.9999
 
 
-def oracle_sublayer(wl, seed, layer, experts, fmts=(MX, MX, MX)):
+def oracle_sublayer(wl, seed, layer, experts, fmts=(MX, MX, MX), nv_codes=None):
     """oracle.Layer holding only `experts` (in that order), bytes regenerated
-    on the host; NVFP4 projections converted by the oracle's own rule."""
+    on the host; NVFP4 projections converted by the oracle's own rule, or, with
+    `nv_codes`, the general NVFP4 source drawn with those block-scale codes."""
     shapes = ((wl.I, wl.H), (wl.I, wl.H), (wl.H, wl.I))
     ws = []
     for pi, ((rows, cols), fmt) in enumerate(zip(shapes, fmts)):
+        if fmt == NV and nv_codes is not None:
+            q, e4, s2 = synth.nv_expert_bytes(seed, layer, pi, rows, cols, list(experts), wl.E,
+                                              "cpu", *nv_codes)
+            ws.append(oracle.Weight(NV, q, e4, s2))
+            continue
         q, s = synth.mx_expert_bytes(seed, layer, pi, rows, cols, wl.code_lo, wl.code_hi,
                                      list(experts), wl.E, "cpu")
         if fmt == NV:
@@ -31,12 +37,12 @@ def oracle_sublayer(wl, seed, layer, experts, fmts=(MX, MX, MX)):
     return oracle.Layer(*ws)
 
 
-def oracle_moe(wl, seed, layer, x_bf16, ids, w, fmts=(MX, MX, MX)):
+def oracle_moe(wl, seed, layer, x_bf16, ids, w, fmts=(MX, MX, MX), nv_codes=None):
     """Oracle y for tokens x with routing (ids, w): experts remapped to a sub-layer."""
     ids = np.asarray(ids)
     experts = sorted(set(int(e) for e in ids.reshape(-1)))
     remap = {e: i for i, e in enumerate(experts)}
-    L = oracle_sublayer(wl, seed, layer, experts, fmts)
+    L = oracle_sublayer(wl, seed, layer, experts, fmts, nv_codes)
     sub = np.vectorize(remap.get)(ids).astype(np.int32)
     return oracle.moe_forward(L, x_bf16, sub, np.asarray(w, dtype=np.float64))
 

@@ -37,6 +37,30 @@ def test_nan_scale_reported():
     assert qk.qk_last_device_status() == qk.QK_ERR_NAN_SCALE
 
 
+def test_nan_e4m3_block_scale_reported_decode():
+    """NVFP4 (a general source): e4m3 0x7F in one block scale, decode path."""
+    layer = workload.make_layer(WL, 3, 0, (2, 2, 2), nv_codes=(0x60, 0x7E))
+    layer.up.scales[2, 7, 5] = 0x7F
+    x = synth.activations(3, WL.T, WL.H)
+    ids = torch.tensor([[2, 1]] * 4, dtype=torch.int32, device="cuda")
+    w = torch.full((4, 2), 0.5, device="cuda")
+    _fwd(layer, x, ids, w)
+    assert qk.qk_last_device_status() == qk.QK_ERR_NAN_SCALE
+
+
+@pytest.mark.parametrize("fmt,code", [(1, 0xFF), (2, 0x7F), (2, 0xFF)])
+def test_nan_scale_reported_grouped(fmt, code):
+    """100 tokens x top-2 (the grouped GEMMs): one NaN scale code in expert
+    2's up projection (e8m0 0xFF; e4m3 0x7F or 0xFF)."""
+    layer = workload.make_layer(WL, 4, 0, (fmt, fmt, fmt), nv_codes=(0x60, 0x7E))
+    layer.up.scales[2, 7, 3] = code
+    x = synth.activations(4, 100, WL.H)
+    ids = torch.tensor([[2, 1]] * 100, dtype=torch.int32, device="cuda")
+    w = torch.full((100, 2), 0.5, device="cuda")
+    _fwd(layer, x, ids, w)
+    assert qk.qk_last_device_status() == qk.QK_ERR_NAN_SCALE
+
+
 def test_out_of_range_id_reported_and_skipped():
     layer, x = _setup(1)
     ids_np = np.array([[1, 4], [8, 2], [3, -1], [0, 7]], np.int32)
