@@ -52,6 +52,39 @@ def test_stack_layer_mixed_formats():
     assert_parity(y.cpu().numpy(), yo, what=f"stack layer 5 {fmts}")
 
 
+@pytest.mark.parametrize("layer_id", [0, 17, 29, 42])
+def test_stack_sampled_layers_with_shared_expert(layer_id):
+    """The 43-layer stack on a seeded sample of its layers: 180 experts,
+    top-6, 8 tokens, the layer's seeded per-projection formats, and the FP8
+    block-128 shared expert added into the same output (y = routed + shared).
+    The oracle regenerates both on the host.  The shared expert's synthetic
+    FP8 weights (codes uniform over all 254 values) make its output about
+    10^6 times the routed one, so each part is checked on its own as well as
+    the sum."""
+    wl = synth.WORKLOADS["stack43"]
+    fmts = tuple(int(f) for f in synth.format_choice(0, wl.layers)[layer_id])
+    layer = workload.make_layer(wl, 0, layer_id, fmts)
+    sh = workload.make_fp8_shared(0, layer_id, wl.H, wl.I)
+    x = synth.activations(0, wl.T, wl.H, stream=layer_id)
+    lg = synth.router_logits(0, wl.T, wl.E, stream=layer_id)
+    oids, ow = oracle.route_topk(lg, wl.k)
+    xd = x.cuda()
+    y = _forward(layer, xd, torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
+    y_routed = y.cpu().numpy().astype(np.float64)
+    ws = torch.empty(qk.fp8_shared_expert_workspace_size(wl.T, wl.H, wl.I), dtype=torch.uint8,
+                     device="cuda")
+    qk.fp8_shared_expert_forward(xd, sh.wg, sh.sg, sh.wu, sh.su, sh.wd, sh.sd, y, ws)
+    assert qk.qk_last_device_status() == qk.QK_OK
+    y_total = y.cpu().numpy().astype(np.float64)
+    ro = oracle_moe(wl, 0, layer_id, x, oids, ow.astype(np.float32).astype(np.float64), fmts)
+    hs = workload.make_fp8_shared(0, layer_id, wl.H, wl.I, device="cpu")
+    so = oracle.fp8_swiglu_ffn(x, hs.wg, hs.sg, hs.wu, hs.su, hs.wd, hs.sd)
+    what = f"stack layer {layer_id} {fmts}"
+    assert_parity(y_routed, ro, what=what + " routed")
+    assert_parity(y_total - y_routed, so, what=what + " shared expert")
+    assert_parity(y_total, ro + so, what=what + " routed + shared")
+
+
 def test_prefill_zipf_sampled_tokens():
     """2048 tokens, Zipf-skewed routing over 256 experts; 12 sampled tokens
     (including ones routed to the most and least loaded experts) against the
