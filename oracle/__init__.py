@@ -18,6 +18,7 @@ _SO = os.path.join(_HERE, "liboracle.so")
 
 QKO_OK, QKO_ERR_INVALID_ARG, QKO_ERR_NAN_SCALE = 0, 1, 4
 MXFP4, NVFP4 = 1, 2
+ACT_NONE, ACT_MXFP4, ACT_E4M3 = 0, 1, 2
 
 
 def build(force: bool = False) -> str:
@@ -59,6 +60,11 @@ def lib():
         L.qko_e4m3_value.argtypes = [ctypes.c_uint8]
         L.qko_e4m3_encode.restype = ctypes.c_uint8
         L.qko_e4m3_encode.argtypes = [f64]
+        L.qko_e2m1_encode.restype = ctypes.c_uint8
+        L.qko_e2m1_encode.argtypes = [f64]
+        L.qko_act_quant.argtypes = [vp, i32, i32, vp, vp, vp]
+        L.qko_moe_forward_aq.argtypes = [ctypes.POINTER(_Layer), vp, i32, vp, vp, i32, i32, vp]
+        L.qko_expert_ffn_aq.argtypes = [ctypes.POINTER(_Layer), i32, vp, i32, vp, vp, vp, vp]
         L.qko_dequant_row.argtypes = [ctypes.POINTER(_Weight), i32, i32, vp]
         L.qko_convert_mx_to_nv.argtypes = [vp, i32, i32, i32, vp, vp, vp]
         L.qko_route_topk.argtypes = [vp, i32, i32, i32, vp, vp]
@@ -176,25 +182,43 @@ def route_topk(logits, k: int):
     return ids, w
 
 
-def moe_forward(layer: Layer, x_bf16, ids, w) -> np.ndarray:
+def moe_forward(layer: Layer, x_bf16, ids, w, aq: int = ACT_NONE) -> np.ndarray:
     x = _np(x_bf16, np.uint16)
     ids = _np(ids, np.int32)
     w = np.ascontiguousarray(np.asarray(w, dtype=np.float64))
     T, k = ids.shape
     y = np.empty((T, layer.hidden), dtype=np.float64)
     cl = layer.c()
-    _chk(lib().qko_moe_forward(ctypes.byref(cl), _p(x), T, _p(ids), _p(w), k, _p(y)))
+    _chk(lib().qko_moe_forward_aq(ctypes.byref(cl), _p(x), T, _p(ids), _p(w), k, aq, _p(y)))
     return y
 
 
-def expert_ffn(layer: Layer, e: int, x_bf16_row):
+def expert_ffn(layer: Layer, e: int, x_bf16_row, aq: int = ACT_NONE):
+    """(g, u, h, d) of expert e on one token; with `aq`, h is the quantized
+    h that the down projection consumes."""
     x = _np(x_bf16_row, np.uint16).reshape(-1)
     I, H = layer.inter, layer.hidden
     g, u, h = (np.empty(I) for _ in range(3))
     d = np.empty(H)
     cl = layer.c()
-    _chk(lib().qko_expert_ffn(ctypes.byref(cl), e, _p(x), _p(g), _p(u), _p(h), _p(d)))
+    _chk(lib().qko_expert_ffn_aq(ctypes.byref(cl), e, _p(x), aq, _p(g), _p(u), _p(h), _p(d)))
     return g, u, h, d
+
+
+def e2m1_encode(v: float) -> int:
+    return lib().qko_e2m1_encode(float(v))
+
+
+def act_quant(v, aq: int):
+    """Quantize a float64 vector (length a multiple of 32) by the OCP MX rule:
+    returns (element codes uint8 [n], e8m0 scale codes uint8 [n/32],
+    dequantized float64 [n])."""
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64).reshape(-1))
+    codes = np.empty(v.size, np.uint8)
+    scales = np.empty(v.size // 32, np.uint8)
+    out = np.empty(v.size, np.float64)
+    _chk(lib().qko_act_quant(_p(v), v.size, aq, _p(codes), _p(scales), _p(out)))
+    return codes, scales, out
 
 
 def fp8_block_linear(x_bf16, w, w_scale, block: int = 128) -> np.ndarray:

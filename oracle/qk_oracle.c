@@ -71,6 +71,22 @@ uint8_t qko_e4m3_encode(double v) {
   return sign | (uint8_t)(((ex + 7) << 3) | m);
 }
 
+/* Cast to e2m1: round to nearest, ties to the even code (mantissa bit 0),
+ * saturating to +-6 (FP4 has no infinity or NaN; OCP Microscaling v1.0
+ * conversions clamp).  Returns the 4-bit code. */
+uint8_t qko_e2m1_encode(double v) {
+  uint8_t sign = signbit(v) ? 8 : 0;
+  double a = fabs(v);
+  int ex, n;
+  if (a >= 6.0) return sign | 7;
+  if (a < 1.0) return sign | (uint8_t)round_half_even(a * 2.0); /* 0, 0.5, 1: codes 0, 1, 2 */
+  frexp(a, &ex);
+  ex -= 1;                                 /* a = f * 2^ex, f in [1,2), ex in {0, 1, 2} */
+  n = (int)round_half_even(ldexp(a, 1 - ex)); /* a / 2^(ex-1) in [2, 4) -> 2, 3 or 4 */
+  if (n == 4) return sign | (uint8_t)((ex + 2) << 1);
+  return sign | (uint8_t)(((ex + 1) << 1) | (n - 2));
+}
+
 double qko_bf16_value(uint16_t bits) {
   uint32_t u = (uint32_t)bits << 16;
   float f;
@@ -190,6 +206,60 @@ int qko_route_topk(const float* logits, int32_t T, int32_t E, int32_t k,
   return QKO_OK;
 }
 
+/* ------------------------------------------------- activation quantization --
+ * The activation-quantized modes: fp4 weights times MXFP4 or E4M3
+ * activations on block-scaled tensor cores, the latter being the expert
+ * numerics DeepSeek-V4-Flash's own config names ("DeepSeekv4 Flash for 1x
+ * Spark [REAP25]", the v0.2.3 update: fp4 weights x dynamic E4M3
+ * activations on the f8f6f4 tensor cores).  The block-scaled MMA takes one
+ * e8m0 scale per 32 activations; the scale rule is the OCP Microscaling v1.0
+ * one (reading adopted; the pages give none): per block of 32,
+ *   X = floor(log2 max|v|) - emax,  emax = 2 (e2m1) or 8 (e4m3),
+ * clamped to the e8m0 range [-127, 127] (X = -127 for an all-zero block), and
+ * each element is cast from v / 2^X with round-to-nearest-even, saturating.
+ * codes: one element code per value (e2m1 in the low nibble, or e4m3);
+ * scales: one e8m0 code per block; out: the dequantized values.  Any of the
+ * three outputs may be NULL.  A non-finite value is an argument error. */
+int qko_act_quant(const double* v, int32_t n, int32_t aq, uint8_t* codes, uint8_t* scales,
+                  double* out) {
+  int32_t b, i;
+  int emax;
+  if (!v || n < 0 || n % 32) return QKO_ERR_INVALID_ARG;
+  if (aq == QKO_ACT_MXFP4) emax = 2;
+  else if (aq == QKO_ACT_E4M3) emax = 8;
+  else return QKO_ERR_INVALID_ARG;
+  for (b = 0; b < n / 32; ++b) {
+    const double* vb = v + (int64_t)b * 32;
+    double amax = 0.0;
+    int X = -127, ex;
+    for (i = 0; i < 32; ++i) {
+      if (isnan(vb[i]) || isinf(vb[i])) return QKO_ERR_INVALID_ARG;
+      if (fabs(vb[i]) > amax) amax = fabs(vb[i]);
+    }
+    if (amax > 0.0) {
+      frexp(amax, &ex);
+      X = (ex - 1) - emax;
+      if (X < -127) X = -127;
+      if (X > 127) X = 127;
+    }
+    if (scales) scales[b] = (uint8_t)(X + 127);
+    for (i = 0; i < 32; ++i) {
+      double q = ldexp(vb[i], -X), val;
+      uint8_t c;
+      if (aq == QKO_ACT_MXFP4) {
+        c = qko_e2m1_encode(q);
+        val = qko_e2m1_value(c);
+      } else {
+        c = qko_e4m3_encode(q);
+        val = qko_e4m3_value(c);
+      }
+      if (codes) codes[(int64_t)b * 32 + i] = c;
+      if (out) out[(int64_t)b * 32 + i] = ldexp(val, X);
+    }
+  }
+  return QKO_OK;
+}
+
 /* ----------------------------------------------------------------- FFN --
  * Routed expert (pages: gate/up/down projections; SwiGLU form not printed,
  * reading adopted: h = silu(gate) * up, silu(g) = g / (1 + exp(-g)), no clamp,
@@ -226,11 +296,16 @@ static int check_layer(const qko_layer* L) {
   return 1;
 }
 
-int qko_expert_ffn(const qko_layer* L, int32_t e, const uint16_t* x_bf16,
-                   double* g, double* u, double* h, double* d) {
-  int32_t I, H, i, err = QKO_OK;
+/* One expert on one token.  With an activation-quantized mode, x is
+ * quantized before gate/up, and h is rounded to fp32 (the precision in which
+ * the GPU takes the same decision) and quantized before down; h then returns
+ * the quantized values down consumes. */
+int qko_expert_ffn_aq(const qko_layer* L, int32_t e, const uint16_t* x_bf16, int32_t aq,
+                      double* g, double* u, double* h, double* d) {
+  int32_t I, H, i, err = QKO_OK, aq_err = QKO_OK;
   double *xg, *gg, *uu, *hh, *dd;
   if (!check_layer(L) || !x_bf16 || e < 0 || e >= L->gate.n_experts) return QKO_ERR_INVALID_ARG;
+  if (aq != QKO_ACT_NONE && aq != QKO_ACT_MXFP4 && aq != QKO_ACT_E4M3) return QKO_ERR_INVALID_ARG;
   I = L->inter;
   H = L->hidden;
   xg = (double*)malloc(sizeof(double) * H);
@@ -239,22 +314,33 @@ int qko_expert_ffn(const qko_layer* L, int32_t e, const uint16_t* x_bf16,
   hh = (double*)malloc(sizeof(double) * I);
   dd = (double*)malloc(sizeof(double) * H);
   for (i = 0; i < H; ++i) xg[i] = qko_bf16_value(x_bf16[i]);
+  if (aq != QKO_ACT_NONE) aq_err |= qko_act_quant(xg, H, aq, NULL, NULL, xg);
   err |= matvec_rows(&L->gate, e, xg, gg);
   err |= matvec_rows(&L->up, e, xg, uu);
   for (i = 0; i < I; ++i) hh[i] = gg[i] / (1.0 + exp(-gg[i])) * uu[i];
+  if (aq != QKO_ACT_NONE && !err) {
+    for (i = 0; i < I; ++i) hh[i] = (double)(float)hh[i];
+    aq_err |= qko_act_quant(hh, I, aq, NULL, NULL, hh);
+  }
   err |= matvec_rows(&L->down, e, hh, dd);
   if (g) memcpy(g, gg, sizeof(double) * I);
   if (u) memcpy(u, uu, sizeof(double) * I);
   if (h) memcpy(h, hh, sizeof(double) * I);
   if (d) memcpy(d, dd, sizeof(double) * H);
   free(xg); free(gg); free(uu); free(hh); free(dd);
-  return err ? QKO_ERR_NAN_SCALE : QKO_OK;
+  if (err) return QKO_ERR_NAN_SCALE;
+  return aq_err ? QKO_ERR_INVALID_ARG : QKO_OK;  /* a non-finite activation */
+}
+
+int qko_expert_ffn(const qko_layer* L, int32_t e, const uint16_t* x_bf16,
+                   double* g, double* u, double* h, double* d) {
+  return qko_expert_ffn_aq(L, e, x_bf16, QKO_ACT_NONE, g, u, h, d);
 }
 
 /* Weighted combine: y[t] = sum over slots s = 0..k-1, in that order, of
  * w[t][s] * d_{t,s}. */
-int qko_moe_forward(const qko_layer* L, const uint16_t* x_bf16, int32_t T,
-                    const int32_t* ids, const double* w, int32_t k, double* y) {
+int qko_moe_forward_aq(const qko_layer* L, const uint16_t* x_bf16, int32_t T,
+                       const int32_t* ids, const double* w, int32_t k, int32_t aq, double* y) {
   int32_t t, s, m, H;
   double* d;
   if (!check_layer(L) || T < 0 || k <= 0 || (T > 0 && (!x_bf16 || !ids || !w || !y)))
@@ -271,14 +357,19 @@ int qko_moe_forward(const qko_layer* L, const uint16_t* x_bf16, int32_t T,
     double* yt = y + (int64_t)t * H;
     for (m = 0; m < H; ++m) yt[m] = 0.0;
     for (s = 0; s < k; ++s) {
-      int err = qko_expert_ffn(L, ids[(int64_t)t * k + s], x_bf16 + (int64_t)t * H, NULL, NULL,
-                               NULL, d);
+      int err = qko_expert_ffn_aq(L, ids[(int64_t)t * k + s], x_bf16 + (int64_t)t * H, aq, NULL,
+                                  NULL, NULL, d);
       if (err) { free(d); return err; }
       for (m = 0; m < H; ++m) yt[m] += w[(int64_t)t * k + s] * d[m];
     }
   }
   free(d);
   return QKO_OK;
+}
+
+int qko_moe_forward(const qko_layer* L, const uint16_t* x_bf16, int32_t T,
+                    const int32_t* ids, const double* w, int32_t k, double* y) {
+  return qko_moe_forward_aq(L, x_bf16, T, ids, w, k, QKO_ACT_NONE, y);
 }
 
 /* ------------------------------------------------------ FP8 block-128 --

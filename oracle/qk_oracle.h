@@ -40,12 +40,14 @@ extern "C" {
 
 enum { QKO_OK = 0, QKO_ERR_INVALID_ARG = 1, QKO_ERR_NAN_SCALE = 4 };
 enum { QKO_FMT_MXFP4 = 1, QKO_FMT_NVFP4 = 2 };
+enum { QKO_ACT_NONE = 0, QKO_ACT_MXFP4 = 1, QKO_ACT_E4M3 = 2 }; /* activation quantization */
 
 /* Element codes. */
 double qko_e2m1_value(uint8_t code);      /* low 4 bits: s|e1 e0|m */
 double qko_e8m0_value(uint8_t code);      /* 2^(c-127); NaN for 255 */
 double qko_e4m3_value(uint8_t code);      /* E4M3FN; NaN for 0x7F/0xFF */
 uint8_t qko_e4m3_encode(double v);        /* round-to-nearest-even, saturate to +-448 */
+uint8_t qko_e2m1_encode(double v);        /* round-to-nearest-even, saturate to +-6 */
 double qko_bf16_value(uint16_t bits);
 
 /* One projection of one layer: nibbles [E][rows][cols/2], scales
@@ -82,6 +84,19 @@ int qko_moe_forward(const qko_layer* L, const uint16_t* x_bf16, int32_t T,
 /* One expert's FFN on one token, with intermediates (any pointer may be NULL). */
 int qko_expert_ffn(const qko_layer* L, int32_t e, const uint16_t* x_bf16,
                    double* g, double* u, double* h, double* d);
+
+/* Activation quantization of n values (n % 32 == 0) to MXFP4 or E4M3 with one
+ * e8m0 scale per 32 (OCP MX scale rule): element codes [n], scale codes
+ * [n/32], dequantized values [n]; any output may be NULL. */
+int qko_act_quant(const double* v, int32_t n, int32_t aq, uint8_t* codes, uint8_t* scales,
+                  double* out);
+
+/* The FFN and the routed sum with activation quantization `aq` (QKO_ACT_*):
+ * x quantized before gate/up, h (rounded to fp32) quantized before down. */
+int qko_expert_ffn_aq(const qko_layer* L, int32_t e, const uint16_t* x_bf16, int32_t aq,
+                      double* g, double* u, double* h, double* d);
+int qko_moe_forward_aq(const qko_layer* L, const uint16_t* x_bf16, int32_t T,
+                       const int32_t* ids, const double* w, int32_t k, int32_t aq, double* y);
 
 /* y[M][N] = x[M][K] . dq(W)^T with W e4m3 [N][K], scales ue8m0 [N/b][K/b]. */
 int qko_fp8_block_linear(const uint16_t* x_bf16, int32_t M, int32_t K,
