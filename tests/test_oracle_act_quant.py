@@ -203,3 +203,37 @@ def test_aq_none_is_the_plain_path():
     ids = np.array([[0, 1], [1, 0]], np.int32)
     w = np.array([[0.5, 0.5], [0.25, 0.75]])
     assert np.array_equal(oracle.moe_forward(L, x, ids, w), oracle.moe_forward(L, x, ids, w, oracle.ACT_NONE))
+
+
+def test_h_is_rounded_to_fp32_before_it_is_quantized():
+    """A constructed expert whose h lies within fp32 rounding of an e2m1 tie.
+    g = 40 and 64 (silu(g) = g exactly in fp64 for g >= 38), u = 1 + 2^-25
+    and 1: h = 40 + 40 * 2^-25 and 64.  The block maximum 64 gives X = 4.
+    fp32(h) = 40 exactly (half an fp32 ulp at 40 is 2^-19 > 40 * 2^-25), and
+    40 / 16 = 2.5 is a tie between 2 and 3 that goes to the even code: 2, so
+    hq = 32.  Without the fp32 rounding h / 16 lies above the tie and gives
+    3 (48).  down row 0 picks hq at that index."""
+    H = I = 64
+    qg, qu, qd = (np.zeros((1, r, c // 2), np.uint8) for r, c in ((I, H), (I, H), (H, I)))
+    sg, su, sd = (np.full((1, r, c // 32), 127, np.uint8) for r, c in ((I, H), (I, H), (H, I)))
+
+    def put(q, s, row, col, code, scale):
+        q[0, row, col // 2] |= code << (4 * (col % 2))
+        s[0, row, col // 32] = scale
+
+    put(qg, sg, 0, 0, 6, 131)   # g_0 = 4 * 2^4 = 64
+    put(qu, su, 0, 0, 2, 127)   # u_0 = 1
+    put(qg, sg, 1, 0, 6, 130)   # g_1 = 4 * 2^3 + 1 * 2^3 = 40
+    put(qg, sg, 1, 32, 2, 130)
+    put(qu, su, 1, 0, 2, 127)   # u_1 = 1 + 0.5 * 2^-24 = 1 + 2^-25
+    put(qu, su, 1, 32, 1, 103)
+    put(qd, sd, 0, 1, 2, 127)   # d_0 = hq_1
+    L = oracle.Layer(oracle.Weight(oracle.MXFP4, qg, sg), oracle.Weight(oracle.MXFP4, qu, su),
+                     oracle.Weight(oracle.MXFP4, qd, sd))
+    x = torch.zeros(H, dtype=torch.bfloat16)
+    x[0] = x[32] = 1.0
+    g, u, h, d = oracle.expert_ffn(L, 0, x, oracle.ACT_MXFP4)
+    assert g[0] == 64 and g[1] == 40 and u[1] == 1 + 2.0 ** -25
+    assert h[0] == 64 and h[1] == 32 and d[0] == 32
+    _, _, h_plain, _ = oracle.expert_ffn(L, 0, x)
+    assert h_plain[1] == 40 + 40 * 2.0 ** -25
