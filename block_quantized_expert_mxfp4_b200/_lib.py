@@ -61,7 +61,7 @@ def load() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     L.moe_expert_workspace_size.restype = sz
-    L.moe_expert_workspace_size.argtypes = [ctypes.POINTER(qk_moe_layer), i32, i32]
+    L.moe_expert_workspace_size.argtypes = [ctypes.POINTER(qk_moe_layer), i32, i32, i32]
     L.moe_expert_forward.restype = i32
     L.moe_expert_forward.argtypes = [ctypes.POINTER(qk_moe_layer), vp, i32, vp, vp, i32, vp, i32,
                                      i32, vp, sz, vp]
@@ -118,8 +118,9 @@ def make_layer(gate: qk_weight, up: qk_weight, down: qk_weight) -> qk_moe_layer:
     return qk_moe_layer(gate, up, down, gate.cols, gate.rows)
 
 
-def moe_expert_workspace_size(layer: qk_moe_layer, n_tokens: int, top_k: int) -> int:
-    return load().moe_expert_workspace_size(ctypes.byref(layer), n_tokens, top_k)
+def moe_expert_workspace_size(layer: qk_moe_layer, n_tokens: int, top_k: int,
+                              act_quant: int = QK_ACT_NONE) -> int:
+    return load().moe_expert_workspace_size(ctypes.byref(layer), n_tokens, top_k, act_quant)
 
 
 def moe_expert_forward(layer: qk_moe_layer, x: torch.Tensor, topk_ids: torch.Tensor,

@@ -2,6 +2,7 @@
 // argument validation, workspace carving, dispatch, and the device status word.
 #include <cuda_runtime.h>
 
+#include "qk_actq.cuh"
 #include "qk_device.cuh"
 #include "qk_internal.h"
 
@@ -36,8 +37,17 @@ extern "C" {
 // pairs; more tokens take the grouped path.
 static int decode_chunk(int top_k) { return kMaxPairs / top_k; }
 
-size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_t top_k) {
+// The activation-quantized modes run on the grouped block-scaled kernels at
+// every token count (all-MXFP4 layers that qualify for them).
+static bool act_quant_ok(const qk_moe_layer* L, int32_t act_quant) {
+  return (act_quant == QK_ACT_MXFP4 || act_quant == QK_ACT_E4M3) &&
+         gmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter);
+}
+
+size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_t top_k, int32_t act_quant) {
   if (layer_ok(L) != QK_OK || n_tokens < 0 || top_k < 1 || top_k > 8) return 0;
+  if (act_quant != QK_ACT_NONE)
+    return act_quant_ok(L, act_quant) ? group_workspace_bytes(L, n_tokens, top_k) : 0;
   if (n_tokens > decode_chunk(top_k))
     return group_workspace_bytes(L, n_tokens, top_k);
   if (dmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter))
@@ -52,10 +62,12 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
   const qk_status lrc = layer_ok(L);
   if (lrc != QK_OK) return lrc;
   if (n_tokens < 0 || top_k < 1 || top_k > 8) return QK_ERR_INVALID_ARG;
-  if (act_quant != QK_ACT_NONE) return QK_ERR_UNSUPPORTED;
+  if (act_quant != QK_ACT_NONE && act_quant != QK_ACT_MXFP4 && act_quant != QK_ACT_E4M3)
+    return QK_ERR_INVALID_ARG;
+  if (act_quant != QK_ACT_NONE && !act_quant_ok(L, act_quant)) return QK_ERR_UNSUPPORTED;
   if (n_tokens == 0) return QK_OK;
   if (!x_bf16 || !topk_ids || !topk_w || !y || !aligned16(x_bf16)) return QK_ERR_INVALID_ARG;
-  const size_t need = moe_expert_workspace_size(L, n_tokens, top_k);
+  const size_t need = moe_expert_workspace_size(L, n_tokens, top_k, act_quant);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return QK_ERR_WORKSPACE;
   DecodeArgs a = {};
@@ -73,7 +85,10 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
   a.I = L->inter;
   a.P = n_tokens * top_k;
   a.y_bf16 = y_is_bf16 ? 1 : 0;
-  // Token counts above one decode launch's routing capacity take the grouped path.
+  // The activation-quantized modes, and token counts above one decode launch's
+  // routing capacity, take the grouped path.
+  if (act_quant != QK_ACT_NONE)
+    return group_forward_act(a, act_quant, workspace, reinterpret_cast<cudaStream_t>(stream));
   if (n_tokens > decode_chunk(top_k)) return group_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
   // All-MXFP4 layers: weights straight to the block-scaled tensor cores.
   if (dmx_eligible(a.gate, a.up, a.down, a.H, a.I))

@@ -43,6 +43,7 @@
 #include <cuda.h>
 #include <cuda_fp8.h>
 
+#include "qk_actq.cuh"
 #include "qk_common.cuh"
 #include "qk_group.cuh"
 #include "qk_tmap.h"
@@ -93,10 +94,12 @@ __device__ __forceinline__ void put_term(uint8_t* blocks, uint8_t* atoms, int f,
 }
 
 // One block per token: its pairs' sorted rows (counting-sort scatter) and
-// tile positions, then x split into two e4m3 terms per 32-block, written into
-// the gate/up tile of each pair.
+// tile positions, then x split into two e4m3 terms per 32-block (QK_ACT_NONE)
+// or quantized to one term (the activation-quantized modes; second term
+// zero), written into the gate/up tile of each pair.
 __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uint16_t* __restrict__ x,
-                                                            const int32_t* __restrict__ ids, int k, int E, int H) {
+                                                            const int32_t* __restrict__ ids, int k, int E, int H,
+                                                            int act_quant) {
   __shared__ int fj[8];
   const int t = blockIdx.x;
   if (threadIdx.x < k) {
@@ -131,8 +134,16 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
       }
     }
     uint32_t q0[8], q1[8];
-    const int c0 = split_term(v, q0);
-    const int c1 = split_term(v, q1);
+    int c0, c1;
+    if (act_quant == QK_ACT_NONE) {
+      c0 = split_term(v, q0);
+      c1 = split_term(v, q1);
+    } else {
+      c0 = actq_block(v, q0, act_quant == QK_ACT_MXFP4);
+      c1 = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q1[i] = 0u;
+    }
     for (int s = 0; s < k; ++s) {
       const int tj = fj[s];
       if (tj < 0) continue;
@@ -143,8 +154,10 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
 }
 
 // One block per sorted row: h = silu(gate) * up in fp32, split into three
-// e4m3 terms per 32-block, written into the row's down tile.
-__global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, int I) {
+// e4m3 terms per 32-block (QK_ACT_NONE) or quantized to one term (the
+// activation-quantized modes; the other two zero), written into the row's
+// down tile.
+__global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, int I, int act_quant) {
   const int r = blockIdx.x;
   if (r >= W.offsets[E]) return;  // block-uniform
   const int tj = W.rtile2[r], f = tj >> 8, j = tj & 255;
@@ -161,11 +174,21 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, in
       v[4 * q + 2] = __fdividef(g.z, 1.0f + __expf(-g.z)) * u.z;
       v[4 * q + 3] = __fdividef(g.w, 1.0f + __expf(-g.w)) * u.w;
     }
+    if (act_quant == QK_ACT_NONE) {
 #pragma unroll
-    for (int term = 0; term < 3; ++term) {
+      for (int term = 0; term < 3; ++term) {
+        uint32_t q[8];
+        const int c = split_term(v, q);
+        put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, term, b, q, c);
+      }
+    } else {
       uint32_t q[8];
-      const int c = split_term(v, q);
-      put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, term, b, q, c);
+      const int c = actq_block(v, q, act_quant == QK_ACT_MXFP4);
+      put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, 0, b, q, c);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = 0u;
+      put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, 1, b, q, 0);
+      put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, 2, b, q, 0);
     }
   }
 }
@@ -535,8 +558,12 @@ static qk_status x_launch(const GmxArgs& A, cudaStream_t st) {
 }
 
 qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st) {
+  return gmx_forward_act(a, W, QK_ACT_NONE, st);
+}
+
+qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, cudaStream_t st) {
   const int T = a.T, k = a.k, E = a.E, H = a.H, I = a.I;
-  k_gmx_xsplit<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H);
+  k_gmx_xsplit<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H, act_quant);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
 
   GmxArgs g1 = {};
@@ -556,7 +583,7 @@ qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st) {
   qk_status rc = x_launch<true, 2>(g1, st);
   if (rc != QK_OK) return rc;
 
-  k_gmx_hsplit<<<a.P, kRowThreads, 0, st>>>(W, E, I);
+  k_gmx_hsplit<<<a.P, kRowThreads, 0, st>>>(W, E, I, act_quant);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
 
   GmxArgs g2 = {};

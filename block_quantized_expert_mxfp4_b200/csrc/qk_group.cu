@@ -28,6 +28,7 @@
 
 #include <algorithm>
 
+#include "qk_actq.cuh"
 #include "qk_common.cuh"
 #include "qk_group.cuh"
 #include "qk_tmap.h"
@@ -773,8 +774,15 @@ static qk_status g_dispatch(const GemmArgs& A, cudaStream_t st) {
 }
 
 qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
+  return group_forward_act(a, QK_ACT_NONE, workspace, st);
+}
+
+// act_quant other than QK_ACT_NONE runs only on the block-scaled kernels (the
+// caller checks eligibility).
+qk_status group_forward_act(const DecodeArgs& a, int act_quant, void* workspace, cudaStream_t st) {
   const int T = a.T, k = a.k, E = a.E, H = a.H, I = a.I, P = a.P;
   const bool mx = gmx_eligible(a.gate, a.up, a.down, H, I);
+  if (act_quant != QK_ACT_NONE && !mx) return QK_ERR_UNSUPPORTED;
   GroupWs W = g_carve(workspace, T, k, E, H, I, mx);
   if (cudaMemsetAsync(W.counts, 0, W.zero_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
   k_grp_count<<<(P + 255) / 256, 256, 0, st>>>(a.ids, P, E, W.counts);
@@ -782,7 +790,7 @@ qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
   if (mx) k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L2, E, kXTok2, 1, 0);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
   if (mx) {
-    const qk_status rc = gmx_forward(a, W, st);
+    const qk_status rc = gmx_forward_act(a, W, act_quant, st);
     if (rc != QK_OK) return rc;
     k_grp_combine<<<T, 256, 0, st>>>(W, a.w, k, H, a.y, a.y_bf16);
     return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;

@@ -52,7 +52,7 @@ extern "C" qk_status moe_expert_forward_noalloc(const qk_moe_layer* L, const voi
                                                 int32_t y_is_bf16, qk_stream_t stream) {
   if (n_tokens < 0) return QK_ERR_INVALID_ARG;
   // validates the layer and top_k (0 = invalid); the size for >= 1 token
-  const size_t need = moe_expert_workspace_size(L, n_tokens > 0 ? n_tokens : 1, top_k);
+  const size_t need = moe_expert_workspace_size(L, n_tokens > 0 ? n_tokens : 1, top_k, QK_ACT_NONE);
   if (need == 0) return QK_ERR_INVALID_ARG;
   if (n_tokens == 0) return QK_OK;
   if (need > kNoallocScratchBytes) return QK_ERR_WORKSPACE;  // beyond the fixed array

@@ -60,9 +60,20 @@ enum {
 
 enum { QK_FMT_MXFP4 = 1, QK_FMT_NVFP4 = 2 };
 
-/* Activation handling inside moe_expert_forward.  Only QK_ACT_NONE (bf16
- * activations; weights dequantized exactly on chip) is implemented; the
- * others return QK_ERR_UNSUPPORTED. */
+/* Activation handling inside moe_expert_forward.
+ *  QK_ACT_NONE   bf16 activations, used as they are (weights exact on chip,
+ *                activations exact or as exact sums of e4m3 terms).
+ *  QK_ACT_E4M3   W4A8: activations quantized to E4M3 with one e8m0 scale per
+ *                32 ([REAP25] v0.2.3 update: fp4 weights x dynamic E4M3
+ *                activations on block-scaled f8f6f4 tensor cores, the model's
+ *                own expert numerics), x before gate/up and h before down.
+ *  QK_ACT_MXFP4  the same with e2m1 activations (fp4 x fp4).
+ * Scale rule for both (the pages give none; OCP Microscaling v1.0): X =
+ * floor(log2 max|v|) - 8 (e4m3) or - 2 (e2m1) per 32 values, clamped to the
+ * e8m0 range; elements rounded to nearest even, saturating (E4M3 to 448,
+ * e2m1 to 6).  The quantized modes need an all-MXFP4 layer that qualifies for
+ * the block-scaled grouped kernels (see moe_expert_forward) and run on them
+ * at every token count; other layers return QK_ERR_UNSUPPORTED. */
 enum { QK_ACT_NONE = 0, QK_ACT_MXFP4 = 1, QK_ACT_E4M3 = 2 };
 
 /* One projection of one layer, all experts.  Device pointers. */
@@ -91,7 +102,7 @@ typedef struct qk_moe_layer {
  *
  *  x_bf16    [T][hidden] bf16.        topk_ids [T][top_k] int32 in [0, E).
  *  topk_w    [T][top_k] fp32.         y        [T][hidden] fp32 (y_is_bf16=0) or bf16.
- *  act_quant QK_ACT_NONE.             workspace >= moe_expert_workspace_size(), 256-B aligned.
+ *  act_quant QK_ACT_* (above).        workspace >= moe_expert_workspace_size(), 256-B aligned.
  * Shapes: hidden and inter multiples of 128; 1 <= top_k <= 8.  Up to
  * floor(128/top_k) tokens run the decode kernels (nibbles and scales decoded
  * in registers, tensor-core m16n8k16 products, fp32 accumulation).  More
@@ -103,12 +114,18 @@ typedef struct qk_moe_layer {
  * are multiples of 512, q is 32-byte and scales 16-byte aligned; otherwise
  * with the weights expanded to f16 on chip.  All kernels run in order on
  * `stream`.  T = 0 returns QK_OK and launches nothing.
- * Errors: QK_ERR_INVALID_ARG (shapes, pointers, formats), QK_ERR_WORKSPACE,
- * QK_ERR_UNSUPPORTED (act_quant), QK_ERR_CUDA; device: QK_ERR_NAN_SCALE,
+ * Errors: QK_ERR_INVALID_ARG (shapes, pointers, formats, an unknown
+ * act_quant), QK_ERR_WORKSPACE, QK_ERR_UNSUPPORTED (a quantized act_quant on
+ * a layer the block-scaled kernels do not take), QK_ERR_CUDA; device:
+ * QK_ERR_NAN_SCALE,
  * QK_ERR_INVALID_ARG (id out of range: that pair contributes nothing),
  * QK_ERR_TIMEOUT.
+ * moe_expert_workspace_size returns the workspace bytes of the path the same
+ * (layer, n_tokens, top_k, act_quant) call takes, or 0 for arguments the call
+ * would reject (including a quantized act_quant the layer does not take).
  * ---------------------------------------------------------------------- */
-size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_t top_k);
+size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_t top_k,
+                                 int32_t act_quant);
 
 qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t n_tokens,
                              const int32_t* topk_ids, const float* topk_w, int32_t top_k,
@@ -122,7 +139,7 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
  * callers that cannot allocate device memory on the call path (a C caller
  * embedded in a runtime that owns every device allocation).
  *  Arguments as moe_expert_forward.  The call needs
- *  moe_expert_workspace_size(L, n_tokens, top_k) <= 4 MiB (hidden 4096,
+ *  moe_expert_workspace_size(L, n_tokens, top_k, QK_ACT_NONE) <= 4 MiB (hidden 4096,
  *  inter 2048: up to 42 pairs per launch for an all-MXFP4 layer on the
  *  block-scaled decode kernels, 28 for other layers); larger requests return
  *  QK_ERR_WORKSPACE and launch nothing.  Nothing in the array has to start at

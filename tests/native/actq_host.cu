@@ -1,0 +1,17 @@
+// Host build of the library's activation-quantization arithmetic
+// (qk_actq.cuh), for the CPU test that compares it with the oracle.  Test
+// infrastructure only: built into tests/_build by tests/test_actq_host.py.
+#define QK_ACTQ_ARITHMETIC_ONLY
+#include "qk_actq.cuh"
+
+// n values (n % 32 == 0) -> one e4m3 code per value (e4m3 of the e2m1 value
+// in fp4 mode) and one e8m0 code per 32.
+extern "C" void actq_host(const float* v, int n, int fp4, uint8_t* codes, uint8_t* scales) {
+  for (int b = 0; b < n / 32; ++b) {
+    float blk[32];
+    uint32_t q[8];
+    for (int i = 0; i < 32; ++i) blk[i] = v[b * 32 + i];
+    scales[b] = (uint8_t)qk::actq_block(blk, q, fp4);
+    memcpy(codes + b * 32, q, 32);
+  }
+}

@@ -45,18 +45,18 @@ def _fake_layer(H=4096, I=2048, E=256, fmts=(1, 1, 1)):
 def test_workspace_query_and_shape_validation():
     L = qk.load()
     lay = _fake_layer()
-    n1 = L.moe_expert_workspace_size(ctypes.byref(lay), 1, 6)
-    n16 = L.moe_expert_workspace_size(ctypes.byref(lay), 16, 6)
+    n1 = L.moe_expert_workspace_size(ctypes.byref(lay), 1, 6, 0)
+    n16 = L.moe_expert_workspace_size(ctypes.byref(lay), 16, 6, 0)
     assert 0 < n1 < n16
-    assert L.moe_expert_workspace_size(ctypes.byref(lay), 1, 9) == 0        # top_k > 8
-    assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(H=4096 + 64)), 1, 6) == 0
-    assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(fmts=(1, 3, 1))), 1, 6) == 0
+    assert L.moe_expert_workspace_size(ctypes.byref(lay), 1, 9, 0) == 0        # top_k > 8
+    assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(H=4096 + 64)), 1, 6, 0) == 0
+    assert L.moe_expert_workspace_size(ctypes.byref(_fake_layer(fmts=(1, 3, 1))), 1, 6, 0) == 0
     bad = _fake_layer()
     bad.down.rows = 2048
-    assert L.moe_expert_workspace_size(ctypes.byref(bad), 1, 6) == 0
+    assert L.moe_expert_workspace_size(ctypes.byref(bad), 1, 6, 0) == 0
     nv = _fake_layer(fmts=(2, 2, 2))
     nv.up.scale_2 = None
-    assert L.moe_expert_workspace_size(ctypes.byref(nv), 1, 6) == 0
+    assert L.moe_expert_workspace_size(ctypes.byref(nv), 1, 6, 0) == 0
 
 
 def test_workspace_query_follows_the_path_choice():
@@ -70,9 +70,25 @@ def test_workspace_query_follows_the_path_choice():
     mis = _fake_layer()
     mis.gate.q = mis.gate.q + 16  # 16-byte aligned, not 32: no block-scaled path
     for T in (1, 16, 100):         # decode (<= 21 tokens at top-6) and grouped
-        a, b, c = (L.moe_expert_workspace_size(ctypes.byref(x), T, 6) for x in (mx, nv, mis))
+        a, b, c = (L.moe_expert_workspace_size(ctypes.byref(x), T, 6, 0) for x in (mx, nv, mis))
         assert a > 0 and b > 0
         assert c == b and a != b, (T, a, b, c)
+
+
+def test_workspace_query_with_activation_modes():
+    """The quantized modes run the grouped block-scaled kernels at every token
+    count: their workspace is the grouped one (the bf16 query's size above one
+    decode launch), and 0 where the mode is refused."""
+    L = qk.load()
+    q = lambda lay, T, aq: L.moe_expert_workspace_size(ctypes.byref(lay), T, 6, aq)
+    mx, nv, mis = _fake_layer(), _fake_layer(fmts=(2, 2, 2)), _fake_layer()
+    mis.gate.q = mis.gate.q + 16
+    for aq in (qk.QK_ACT_MXFP4, qk.QK_ACT_E4M3):
+        assert q(mx, 100, aq) == q(mx, 100, qk.QK_ACT_NONE) > 0
+        assert q(mx, 1, aq) > 0 and q(mx, 1, aq) != q(mx, 1, qk.QK_ACT_NONE)
+        assert q(mx, 1, aq) < q(mx, 16, aq) < q(mx, 100, aq)
+        assert q(nv, 1, aq) == 0 and q(mis, 1, aq) == 0
+    assert q(mx, 1, 7) == 0
 
 
 def test_noalloc_limit_in_pairs():
@@ -82,7 +98,7 @@ def test_noalloc_limit_in_pairs():
     L = qk.load()
     mx, nv = _fake_layer(), _fake_layer(fmts=(2, 2, 2))
     cap = 4 << 20
-    q = lambda lay, T, k: L.moe_expert_workspace_size(ctypes.byref(lay), T, k)
+    q = lambda lay, T, k: L.moe_expert_workspace_size(ctypes.byref(lay), T, k, 0)
     assert q(mx, 7, 6) <= cap < q(mx, 8, 6)        # 42 pairs fit, 48 do not
     assert q(mx, 21, 2) <= cap < q(mx, 22, 2)      # 42 / 44
     assert q(nv, 14, 2) <= cap < q(nv, 15, 2)      # 28 / 30
@@ -94,9 +110,15 @@ def test_forward_argument_errors_are_synchronous():
     vp = ctypes.c_void_p
     f = L.moe_expert_forward
     p = vp(1 << 24)
-    ws = L.moe_expert_workspace_size(ctypes.byref(lay), 1, 6)
+    ws = L.moe_expert_workspace_size(ctypes.byref(lay), 1, 6, 0)
     assert f(ctypes.byref(lay), p, 0, p, p, 6, p, 0, 0, p, ws, None) == qk.QK_OK  # T = 0
-    assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 1, p, ws, None) == qk.QK_ERR_UNSUPPORTED
+    assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 7, p, ws, None) == qk.QK_ERR_INVALID_ARG  # mode
+    nv = _fake_layer(fmts=(2, 2, 2))
+    for aq in (qk.QK_ACT_MXFP4, qk.QK_ACT_E4M3):
+        # a quantized mode: NVFP4 layers are refused; an all-MXFP4 layer runs
+        # the grouped kernels, whose workspace the bf16-path size does not cover
+        assert f(ctypes.byref(nv), p, 1, p, p, 6, p, 0, aq, p, 1 << 30, None) == qk.QK_ERR_UNSUPPORTED
+        assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, aq, p, ws, None) == qk.QK_ERR_WORKSPACE
     assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 0, p, ws - 1, None) == qk.QK_ERR_WORKSPACE
     assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 0, None, ws, None) == qk.QK_ERR_WORKSPACE
     assert f(ctypes.byref(lay), None, 1, p, p, 6, p, 0, 0, p, ws, None) == qk.QK_ERR_INVALID_ARG
