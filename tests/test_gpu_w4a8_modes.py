@@ -1,0 +1,91 @@
+"""GPU parity of the activation-quantized modes of moe_expert_forward:
+QK_ACT_E4M3 (W4A8: fp4 weights x E4M3 activations, the numerics "DeepSeekv4
+Flash for 1x Spark [REAP25]" (v0.2.3 update) names as the model's own) and
+QK_ACT_MXFP4 (fp4 x fp4), against the oracle run in the same mode.
+
+Both run on the grouped block-scaled kernels at every token count.  x codes
+are unique on both sides (bf16 input); an h code may differ where fp32
+rounding leaves it undetermined, which helpers.assert_parity_act_quant allows
+for before applying the usual bar (max-rel <= 5e-3, cosine >= 0.9999)."""
+import numpy as np
+import pytest
+import torch
+
+import block_quantized_expert_mxfp4_b200 as qk
+import oracle
+from block_quantized_expert_mxfp4_b200 import synth, workload
+from helpers import assert_parity_act_quant, oracle_sublayer
+
+pytestmark = pytest.mark.gpu
+
+MODES = [qk.QK_ACT_E4M3, qk.QK_ACT_MXFP4]
+
+
+def _forward(layer, x, ids, w, aq):
+    lay = layer.c()
+    T, k = ids.shape
+    y = torch.full((T, x.shape[1]), float("nan"), dtype=torch.float32, device="cuda")
+    n = qk.moe_expert_workspace_size(lay, T, k, aq)
+    assert n > 0
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    qk.moe_expert_forward(lay, x, ids, w, y, ws, act_quant=aq)
+    assert qk.qk_last_device_status() == qk.QK_OK
+    return y.cpu().numpy()
+
+
+def _check(wl, seed, x, oids, ow, y, aq, what):
+    experts = sorted(set(int(e) for e in oids.reshape(-1)))
+    remap = {e: i for i, e in enumerate(experts)}
+    L = oracle_sublayer(wl, seed, 0, experts)
+    sub = np.vectorize(remap.get)(oids).astype(np.int32)
+    return assert_parity_act_quant(y, L, x, sub, ow.astype(np.float32).astype(np.float64), aq, what=what)
+
+
+@pytest.mark.parametrize("aq", MODES)
+@pytest.mark.parametrize("T", [1, 4])
+def test_decode_sizes(aq, T):
+    """The decode MoE layer (256 experts, top-6, hidden 4096, intermediate
+    2048, MXFP4) at 1 and 4 tokens."""
+    wl = synth.WORKLOADS["decode_mx"]
+    layer = workload.make_layer(wl, 21, 0)
+    x = synth.activations(21, T, wl.H)
+    oids, ow = oracle.route_topk(synth.router_logits(21, T, wl.E), wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda(), aq)
+    _check(wl, 21, x, oids, ow, y, aq, f"act mode {aq} decode T={T}")
+
+
+@pytest.mark.parametrize("aq", MODES)
+def test_grouped_sizes(aq):
+    """48 tokens x top-4 over 16 experts, hidden 1024, intermediate 512."""
+    wl = synth.Workload("mid", 16, 4, 1024, 512, 48, 118, 127)
+    layer = workload.make_layer(wl, 22, 0)
+    x = synth.activations(22, wl.T, wl.H)
+    oids, ow = oracle.route_topk(synth.router_logits(22, wl.T, wl.E), wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda(), aq)
+    _check(wl, 22, x, oids, ow, y, aq, f"act mode {aq} grouped")
+
+
+def test_w4a8_prefill_zipf_sampled_tokens():
+    """The 2048-token Zipf prefill layer in W4A8; 10 sampled tokens."""
+    wl = synth.WORKLOADS["prefill"]
+    layer = workload.make_layer(wl, 23, 0)
+    x = synth.activations(23, wl.T, wl.H)
+    oids, ow = oracle.route_topk(synth.zipf_logits(23, wl.T, wl.E, wl.k), wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda(),
+                 qk.QK_ACT_E4M3)
+    pick = sorted(int(t) for t in np.random.default_rng(24).choice(wl.T, 10, replace=False))
+    _check(wl, 23, x[pick], oids[pick], ow[pick], y[pick], qk.QK_ACT_E4M3, "w4a8 prefill sampled tokens")
+
+
+@pytest.mark.parametrize("aq", MODES)
+def test_modes_are_deterministic_and_differ_from_bf16(aq):
+    wl = synth.Workload("mid", 16, 4, 1024, 512, 24, 118, 127)
+    layer = workload.make_layer(wl, 25, 0)
+    x = synth.activations(25, wl.T, wl.H).cuda()
+    oids, ow = oracle.route_topk(synth.router_logits(25, wl.T, wl.E), wl.k)
+    ids, w = torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda()
+    a = _forward(layer, x, ids, w, aq)
+    b = _forward(layer, x, ids, w, aq)
+    assert np.array_equal(a.view(np.int32), b.view(np.int32))
+    plain = _forward(layer, x, ids, w, qk.QK_ACT_NONE)
+    assert not np.array_equal(a, plain)
