@@ -67,6 +67,7 @@ def lib():
         L.qko_expert_ffn_aq.argtypes = [ctypes.POINTER(_Layer), i32, vp, i32, vp, vp, vp, vp]
         L.qko_dequant_row.argtypes = [ctypes.POINTER(_Weight), i32, i32, vp]
         L.qko_convert_mx_to_nv.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+        L.qko_convert_nv_to_mx.argtypes = [vp, vp, i32, i32, i32, vp, vp]
         L.qko_route_topk.argtypes = [vp, i32, i32, i32, vp, vp]
         L.qko_moe_forward.argtypes = [ctypes.POINTER(_Layer), vp, i32, vp, vp, i32, vp]
         L.qko_expert_ffn.argtypes = [ctypes.POINTER(_Layer), i32, vp, vp, vp, vp, vp]
@@ -171,6 +172,17 @@ def convert_mx_to_nv(e8m0) -> tuple:
     n_bad = ctypes.c_uint64(0)
     _chk(lib().qko_convert_mx_to_nv(_p(s), E, N, 32 * K32, _p(out), _p(s2), ctypes.byref(n_bad)))
     return out, s2, int(n_bad.value)
+
+
+def convert_nv_to_mx(e4m3, scale_2) -> tuple:
+    """e4m3 [E][N][K/16] + scale_2 [E] -> (e8m0 [E][N][K/32] uint8, n_inexact)."""
+    s = _np(e4m3, np.uint8)
+    s2 = np.ascontiguousarray(_np(scale_2, np.float32).reshape(-1))
+    E, N, K16 = s.shape
+    out = np.empty((E, N, K16 // 2), dtype=np.uint8)
+    n_bad = ctypes.c_uint64(0)
+    _chk(lib().qko_convert_nv_to_mx(_p(s), _p(s2), E, N, 16 * K16, _p(out), ctypes.byref(n_bad)))
+    return out, int(n_bad.value)
 
 
 def route_topk(logits, k: int):

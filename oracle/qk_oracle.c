@@ -175,6 +175,52 @@ int qko_convert_mx_to_nv(const uint8_t* e8m0, int32_t E, int32_t N, int32_t K,
  * Softmax over the E logits in fp64, the k largest probabilities (equal
  * probabilities: lower expert id first), renormalised to sum to 1, slots in
  * that order.  (The pages name 256 experts and top-6 but not the function.) */
+/* NVFP4 -> MXFP4, scales only (the reverse of the conversion above; the pages
+ * define only the forward direction, so the rule is the reading adopted).  A
+ * 32-block's two half scales e4m3(s0) * scale_2 and e4m3(s1) * scale_2 (exact
+ * in fp64) convert exactly when they are equal and a power of two 2^p with
+ * -127 <= p <= 127: code p + 127.  Any other block is counted once in
+ * n_inexact and gets the code whose power of two is nearest in log2 to the
+ * larger magnitude of the two (2^p for a mantissa below sqrt 2, else 2^(p+1);
+ * clamped to codes 0 .. 254; code 0 for two zero scales).  A NaN code or a
+ * non-finite product is QKO_ERR_NAN_SCALE. */
+int qko_convert_nv_to_mx(const uint8_t* e4m3, const float* scale_2, int32_t E, int32_t N, int32_t K,
+                         uint8_t* e8m0, uint64_t* n_inexact) {
+  int64_t e, i, per;
+  uint64_t bad = 0;
+  if (!e4m3 || !scale_2 || !e8m0 || E < 0 || N < 0 || K <= 0 || K % 32) return QKO_ERR_INVALID_ARG;
+  per = (int64_t)N * (K / 32);
+  for (e = 0; e < E; ++e) {
+    double s2 = (double)scale_2[e];
+    for (i = 0; i < per; ++i) {
+      uint8_t c0 = e4m3[(e * per + i) * 2], c1 = e4m3[(e * per + i) * 2 + 1];
+      double a = qko_e4m3_value(c0) * s2, b = qko_e4m3_value(c1) * s2, v, f;
+      int ex, p;
+      if (isnan(a) || isnan(b) || isinf(a) || isinf(b)) return QKO_ERR_NAN_SCALE;
+      if (a == b && a > 0.0) {
+        f = frexp(a, &ex);                 /* a = f * 2^ex, f in [0.5, 1) */
+        if (f == 0.5 && ex - 1 >= -127 && ex - 1 <= 127) {
+          e8m0[e * per + i] = (uint8_t)(ex - 1 + 127);
+          continue;
+        }
+      }
+      ++bad;
+      v = fabs(a) > fabs(b) ? fabs(a) : fabs(b);
+      if (v == 0.0) {
+        e8m0[e * per + i] = 0;
+        continue;
+      }
+      f = frexp(v, &ex);                   /* v = (2f) * 2^(ex-1), 2f in [1, 2) */
+      p = (2.0 * f < sqrt(2.0)) ? ex - 1 : ex;
+      if (p < -127) p = -127;
+      if (p > 127) p = 127;
+      e8m0[e * per + i] = (uint8_t)(p + 127);
+    }
+  }
+  if (n_inexact) *n_inexact = bad;
+  return QKO_OK;
+}
+
 int qko_route_topk(const float* logits, int32_t T, int32_t E, int32_t k,
                    int32_t* ids, double* w) {
   int32_t t, i, s;

@@ -73,6 +73,12 @@ int qko_dequant_row(const qko_weight* w, int32_t e, int32_t row, double* out);
 int qko_convert_mx_to_nv(const uint8_t* e8m0, int32_t E, int32_t N, int32_t K,
                          uint8_t* e4m3, float* scale_2, uint64_t* n_inexact);
 
+/* NVFP4 -> MXFP4, scales only: exact blocks (equal power-of-two half scales)
+ * map to their code, others are counted and take the code nearest in log2 to
+ * the larger half scale. */
+int qko_convert_nv_to_mx(const uint8_t* e4m3, const float* scale_2, int32_t E, int32_t N, int32_t K,
+                         uint8_t* e8m0, uint64_t* n_inexact);
+
 /* Softmax over E logits, top-k, renormalised; fp64 weights. */
 int qko_route_topk(const float* logits, int32_t T, int32_t E, int32_t k,
                    int32_t* ids, double* w);
