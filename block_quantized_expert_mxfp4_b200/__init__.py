@@ -8,5 +8,6 @@ from ._lib import (  # noqa: F401
     fp8_shared_expert_workspace_size, load, make_layer, make_weight, moe_expert_forward,
     moe_expert_forward_noalloc,
     moe_expert_workspace_size, moe_route_topk, qk_debug_set_wait_limit_ns, qk_last_device_status,
-    qk_moe_layer, qk_weight, quant_convert_mxfp4_to_nvfp4, status_string,
+    qk_moe_layer, qk_weight, quant_convert_mxfp4_to_nvfp4, quant_convert_nvfp4_to_mxfp4,
+    status_string,
 )

@@ -25,7 +25,8 @@ QK_ACT_NONE, QK_ACT_MXFP4, QK_ACT_E4M3 = 0, 1, 2
 # exported symbols (kept in sync with include/qk.h; checked by tests/test_abi.py)
 SYMBOLS = (
     "moe_expert_workspace_size", "moe_expert_forward", "moe_route_topk",
-    "quant_convert_mxfp4_to_nvfp4", "fp8_block_linear", "fp8_shared_expert_workspace_size",
+    "quant_convert_mxfp4_to_nvfp4", "quant_convert_nvfp4_to_mxfp4", "fp8_block_linear",
+    "fp8_shared_expert_workspace_size",
     "fp8_shared_expert_forward", "qk_last_device_status", "qk_status_string",
     "qk_debug_set_wait_limit_ns", "moe_expert_forward_noalloc",
 )
@@ -72,6 +73,8 @@ def load() -> ctypes.CDLL:
     L.moe_route_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     L.quant_convert_mxfp4_to_nvfp4.restype = i32
     L.quant_convert_mxfp4_to_nvfp4.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
+    L.quant_convert_nvfp4_to_mxfp4.restype = i32
+    L.quant_convert_nvfp4_to_mxfp4.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
     L.fp8_block_linear.restype = i32
     L.fp8_block_linear.argtypes = [vp, i32, i32, vp, vp, i32, vp, i32, vp]
     L.fp8_shared_expert_workspace_size.restype = sz
@@ -159,6 +162,14 @@ def quant_convert_mxfp4_to_nvfp4(e8m0: torch.Tensor, e4m3: torch.Tensor, scale_2
     _check(load().quant_convert_mxfp4_to_nvfp4(_ptr(e8m0), E, N, 32 * K32, _ptr(e4m3),
                                                _ptr(scale_2), _ptr(n_inexact), _stream(stream)),
            "quant_convert_mxfp4_to_nvfp4")
+
+
+def quant_convert_nvfp4_to_mxfp4(e4m3: torch.Tensor, scale_2: torch.Tensor, e8m0: torch.Tensor,
+                                 n_inexact: torch.Tensor, stream=None) -> None:
+    E, N, K16 = e4m3.shape
+    _check(load().quant_convert_nvfp4_to_mxfp4(_ptr(e4m3), _ptr(scale_2), E, N, 16 * K16, _ptr(e8m0),
+                                               _ptr(n_inexact), _stream(stream)),
+           "quant_convert_nvfp4_to_mxfp4")
 
 
 def fp8_block_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor, y: torch.Tensor,

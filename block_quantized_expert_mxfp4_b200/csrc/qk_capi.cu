@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include "qk_actq.cuh"
+#include "qk_convert_nv.h"
 #include "qk_device.cuh"
 #include "qk_internal.h"
 
@@ -115,6 +116,15 @@ qk_status quant_convert_mxfp4_to_nvfp4(const uint8_t* e8m0, int32_t n_experts, i
   if (!e8m0 || !e4m3 || !scale_2 || !n_inexact) return QK_ERR_INVALID_ARG;
   return convert_launch(e8m0, n_experts, rows, cols, e4m3, scale_2, n_inexact,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+qk_status quant_convert_nvfp4_to_mxfp4(const uint8_t* e4m3, const float* scale_2, int32_t n_experts,
+                                       int32_t rows, int32_t cols, uint8_t* e8m0,
+                                       unsigned long long* n_inexact, qk_stream_t stream) {
+  if (n_experts < 0 || rows < 0 || cols <= 0 || cols % 32) return QK_ERR_INVALID_ARG;
+  if (!e4m3 || !scale_2 || !e8m0 || !n_inexact) return QK_ERR_INVALID_ARG;
+  return convert_nv_launch(e4m3, scale_2, n_experts, rows, cols, e8m0, n_inexact,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 qk_status fp8_block_linear(const void* x_bf16, int32_t M, int32_t K, const uint8_t* w,

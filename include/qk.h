@@ -190,6 +190,24 @@ qk_status quant_convert_mxfp4_to_nvfp4(const uint8_t* e8m0, int32_t n_experts, i
                                        unsigned long long* n_inexact, qk_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * quant_convert_nvfp4_to_mxfp4 -- scale-only NVFP4 -> MXFP4, the reverse of
+ * the conversion above (the pages give only the forward direction; rule
+ * adopted): a 32-block whose half scales e4m3(s0) * scale_2 and
+ * e4m3(s1) * scale_2 are equal and a power of two 2^p (-127 <= p <= 127)
+ * converts exactly to code p + 127.  Any other block counts once in
+ * *n_inexact and takes the code whose power of two is nearest in log2 to the
+ * larger magnitude of the two (code 0 for two zero scales).  The nibbles are
+ * not touched; the reverse of a lossless forward conversion is the identity.
+ *  e4m3 [E][N][K/16], scale_2 [E] fp32 -> e8m0 [E][N][K/32];
+ *  n_inexact: device uint64, overwritten.  K multiple of 32.
+ * Errors: QK_ERR_INVALID_ARG, QK_ERR_CUDA; device: QK_ERR_NAN_SCALE (an e4m3
+ * code 0x7F/0xFF or a non-finite scale product; that block's code is 255).
+ * ---------------------------------------------------------------------- */
+qk_status quant_convert_nvfp4_to_mxfp4(const uint8_t* e4m3, const float* scale_2, int32_t n_experts,
+                                       int32_t rows, int32_t cols, uint8_t* e8m0,
+                                       unsigned long long* n_inexact, qk_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * fp8_block_linear -- y[M][N] = x[M][K] . dq(W)^T, dq = e4m3 * 2^(s-127) per
  * 128x128 tile.  [IQ2-FP8] component table ("FP8 E4M3, block-128, UE8M0
  * scales"); [W4A16-FP8] ("FP8_BLOCK 128x128").

@@ -21,7 +21,7 @@ def _declared():
 def test_library_exports_every_declared_symbol():
     L = qk.load()
     names = _declared()
-    assert len(names) == 11
+    assert len(names) == 12
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(_lib.SYMBOLS)
@@ -128,6 +128,8 @@ def test_forward_argument_errors_are_synchronous():
     assert L.moe_route_topk(p, 4, 8, 9, p, p, None) == qk.QK_ERR_INVALID_ARG  # k > E
     assert L.moe_route_topk(p, 0, 8, 2, p, p, None) == qk.QK_OK
     assert L.quant_convert_mxfp4_to_nvfp4(p, 2, 4, 48, p, p, p, None) == qk.QK_ERR_INVALID_ARG
+    assert L.quant_convert_nvfp4_to_mxfp4(p, p, 2, 4, 48, p, p, None) == qk.QK_ERR_INVALID_ARG
+    assert L.quant_convert_nvfp4_to_mxfp4(None, p, 2, 4, 64, p, p, None) == qk.QK_ERR_INVALID_ARG
     assert L.fp8_block_linear(p, 1, 100, p, p, 16, p, 0, None) == qk.QK_ERR_INVALID_ARG
     assert L.fp8_shared_expert_workspace_size(8, 4096, 2048) > 0
     assert L.fp8_shared_expert_forward(p, 8, 4096, 2048, p, p, p, p, p, p, p, p, 0, None) == \
