@@ -105,6 +105,26 @@ def test_prefill_zipf_sampled_tokens():
     assert_parity(y.cpu().numpy()[pick], yo, what="prefill sampled tokens")
 
 
+def test_prefill_16k_tokens_sampled():
+    """The same prefill layer at 16,384 tokens (Zipf s=1, top-6, 256 experts,
+    MXFP4: 98,304 pairs, past the size where the layer turns tensor-bound);
+    12 sampled tokens, including ones routed to the most and the least loaded
+    experts, against the oracle."""
+    wl = synth.WORKLOADS["prefill"]
+    T = 16384
+    layer = workload.make_layer(wl, 0, 0)
+    x = synth.activations(40, T, wl.H)
+    oids, ow = oracle.route_topk(synth.zipf_logits(40, T, wl.E, wl.k), wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
+    counts = np.bincount(oids.reshape(-1), minlength=wl.E)
+    hot, cold = int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
+    pick = {int(np.nonzero((oids == hot).any(1))[0][0]), int(np.nonzero((oids == cold).any(1))[0][0])}
+    pick |= set(int(t) for t in np.random.default_rng(41).choice(T, 10, replace=False))
+    pick = sorted(pick)
+    yo = oracle_moe(wl, 0, 0, x[pick], oids[pick], ow[pick].astype(np.float32).astype(np.float64))
+    assert_parity(y.cpu().numpy()[pick], yo, what="prefill 16k sampled tokens")
+
+
 @pytest.mark.parametrize("fmts", [(NV, NV, NV), (MX, NV, NV), (NV, MX, MX)])
 def test_grouped_path_formats(fmts):
     """48 tokens x top-4 = 192 pairs (grouped path), NVFP4 and mixed projections."""
