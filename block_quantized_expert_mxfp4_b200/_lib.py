@@ -76,11 +76,12 @@ def load() -> ctypes.CDLL:
     L.quant_convert_nvfp4_to_mxfp4.restype = i32
     L.quant_convert_nvfp4_to_mxfp4.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
     L.fp8_block_linear.restype = i32
-    L.fp8_block_linear.argtypes = [vp, i32, i32, vp, vp, i32, vp, i32, vp]
+    L.fp8_block_linear.argtypes = [vp, i32, i32, vp, vp, i32, i32, vp, i32, vp]
     L.fp8_shared_expert_workspace_size.restype = sz
     L.fp8_shared_expert_workspace_size.argtypes = [i32, i32, i32]
     L.fp8_shared_expert_forward.restype = i32
-    L.fp8_shared_expert_forward.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.fp8_shared_expert_forward.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, sz,
+                                            vp]
     L.qk_last_device_status.restype = i32
     L.qk_last_device_status.argtypes = [vp]
     L.qk_status_string.restype = ctypes.c_char_p
@@ -173,10 +174,10 @@ def quant_convert_nvfp4_to_mxfp4(e4m3: torch.Tensor, scale_2: torch.Tensor, e8m0
 
 
 def fp8_block_linear(x: torch.Tensor, w: torch.Tensor, w_scale: torch.Tensor, y: torch.Tensor,
-                     stream=None) -> None:
+                     stream=None, scale_block: int = 128) -> None:
     M, K = x.shape
     N = w.shape[0]
-    _check(load().fp8_block_linear(_ptr(x), M, K, _ptr(w), _ptr(w_scale), N, _ptr(y),
+    _check(load().fp8_block_linear(_ptr(x), M, K, _ptr(w), _ptr(w_scale), N, scale_block, _ptr(y),
                                    int(y.dtype == torch.bfloat16), _stream(stream)),
            "fp8_block_linear")
 
@@ -185,12 +186,13 @@ def fp8_shared_expert_workspace_size(M: int, hidden: int, inter: int) -> int:
     return load().fp8_shared_expert_workspace_size(M, hidden, inter)
 
 
-def fp8_shared_expert_forward(x, wg, sg, wu, su, wd, sd, y, workspace, stream=None) -> None:
+def fp8_shared_expert_forward(x, wg, sg, wu, su, wd, sd, y, workspace, stream=None,
+                              scale_block: int = 128) -> None:
     M, H = x.shape
     I = wg.shape[0]
     _check(load().fp8_shared_expert_forward(
-        _ptr(x), M, H, I, _ptr(wg), _ptr(sg), _ptr(wu), _ptr(su), _ptr(wd), _ptr(sd), _ptr(y),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+        _ptr(x), M, H, I, _ptr(wg), _ptr(sg), _ptr(wu), _ptr(su), _ptr(wd), _ptr(sd), scale_block,
+        _ptr(y), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
         "fp8_shared_expert_forward")
 
 

@@ -4,6 +4,7 @@
 
 #include "qk_actq.cuh"
 #include "qk_convert_nv.h"
+#include "qk_fp8.h"
 #include "qk_device.cuh"
 #include "qk_internal.h"
 
@@ -128,13 +129,14 @@ qk_status quant_convert_nvfp4_to_mxfp4(const uint8_t* e4m3, const float* scale_2
 }
 
 qk_status fp8_block_linear(const void* x_bf16, int32_t M, int32_t K, const uint8_t* w,
-                           const uint8_t* w_scale, int32_t N, void* y, int32_t y_is_bf16,
-                           qk_stream_t stream) {
+                           const uint8_t* w_scale, int32_t N, int32_t scale_block, void* y,
+                           int32_t y_is_bf16, qk_stream_t stream) {
   if (M < 1 || K < 128 || K % 128 || N < 16 || N % 16) return QK_ERR_INVALID_ARG;
+  if (scale_block != 128 && scale_block != 32) return QK_ERR_INVALID_ARG;
   if (!x_bf16 || !w || !w_scale || !y || !aligned16(x_bf16) || !aligned16(w))
     return QK_ERR_INVALID_ARG;
-  return fp8_linear_launch(x_bf16, M, K, w, w_scale, N, y, y_is_bf16 ? 1 : 0,
-                           reinterpret_cast<cudaStream_t>(stream));
+  return fp8_linear_launch_blk(x_bf16, M, K, w, w_scale, N, y, y_is_bf16 ? 1 : 0, scale_block,
+                               reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fp8_shared_expert_workspace_size(int32_t M, int32_t hidden, int32_t inter) {
@@ -145,9 +147,11 @@ size_t fp8_shared_expert_workspace_size(int32_t M, int32_t hidden, int32_t inter
 qk_status fp8_shared_expert_forward(const void* x_bf16, int32_t M, int32_t hidden, int32_t inter,
                                     const uint8_t* w_gate, const uint8_t* s_gate,
                                     const uint8_t* w_up, const uint8_t* s_up,
-                                    const uint8_t* w_down, const uint8_t* s_down, float* y,
-                                    void* workspace, size_t workspace_bytes, qk_stream_t stream) {
+                                    const uint8_t* w_down, const uint8_t* s_down, int32_t scale_block,
+                                    float* y, void* workspace, size_t workspace_bytes,
+                                    qk_stream_t stream) {
   if (M < 1 || hidden < 128 || inter < 128 || hidden % 128 || inter % 128) return QK_ERR_INVALID_ARG;
+  if (scale_block != 128 && scale_block != 32) return QK_ERR_INVALID_ARG;
   if (!x_bf16 || !w_gate || !s_gate || !w_up || !s_up || !w_down || !s_down || !y)
     return QK_ERR_INVALID_ARG;
   if (!aligned16(x_bf16) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down))
@@ -155,8 +159,8 @@ qk_status fp8_shared_expert_forward(const void* x_bf16, int32_t M, int32_t hidde
   const size_t need = fp8_shared_expert_workspace_size(M, hidden, inter);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return QK_ERR_WORKSPACE;
-  return fp8_ffn_launch(x_bf16, M, hidden, inter, w_gate, s_gate, w_up, s_up, w_down, s_down, y,
-                        workspace, reinterpret_cast<cudaStream_t>(stream));
+  return fp8_ffn_launch_blk(x_bf16, M, hidden, inter, w_gate, s_gate, w_up, s_up, w_down, s_down, y,
+                            workspace, scale_block, reinterpret_cast<cudaStream_t>(stream));
 }
 
 qk_status qk_last_device_status(qk_stream_t stream) {

@@ -1,4 +1,5 @@
-// qk_fp8.cu -- FP8 E4M3 linear layers with one UE8M0 scale per 128x128 tile.
+// qk_fp8.cu -- FP8 E4M3 linear layers with one UE8M0 scale per 128x128 tile
+// (or per 32x32 tile).
 //
 // "DeepSeek-V4-Flash-IQ2XXS-Q2K-FP8-120GB-target", component table: dense
 // linears are FP8 E4M3, block-128, UE8M0 scales; "DeepSeek-V4-Flash-W4A16-FP8"
@@ -10,10 +11,15 @@
 // shared rows; eight warps split the reduction in 128-wide scale chunks.
 // e4m3 -> f16 is exact (hardware e4m3x2 -> f16x2), products run on the
 // tensor cores (m16n8k16, fp32 accumulate), and the tile scale 2^(s-127)
-// multiplies each chunk's fp32 partial.
+// multiplies each chunk's fp32 partial.  With 32x32 tiles ("DeepSeek-V4.1-Flash
+// mixed-Q2 GGUF (IQ2_XXS gate/up + Q2_K down)", "Recipe": DeepSeek-V4.1 stores
+// its FP8 dense weights with 32x32 E8M0 block scales, V4 with 128x128) each
+// 32-wide step of a chunk is scaled by its own tile's code; a 16-row unit
+// lies in one 32-row tile.
 #include <algorithm>
 
 #include "qk_common.cuh"
+#include "qk_fp8.h"
 
 namespace qk {
 
@@ -27,7 +33,8 @@ struct Fp8Args {
   const uint8_t* sa;
   const uint8_t* wb;      // kGateUp: rows 8..15 (up projection)
   const uint8_t* sb;
-  int M, K, N, kb;        // N output rows, kb = ceil(K/128) scale columns
+  int M, K, N, kb;        // N output rows, kb = ceil(K/blk) scale columns
+  int blk;                // scale tile edge: 128 or 32
   void* y;                // kLinear: [M][N] fp32/bf16; kDownAcc: fp32 [M][N] (+=)
   int y_bf16;
   float* hout;            // kGateUp: [M][N]
@@ -128,15 +135,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_fp8(const Fp8Args a) {
       return;
     }
     const int64_t r0 = (int64_t)u * rows_per_unit;
-    const uint8_t* sa_row = a.sa + (r0 / 128) * a.kb;
-    const uint8_t* sb_row = MODE == kGateUp ? a.sb + (r0 / 128) * a.kb : sa_row;
+    const uint8_t* sa_row = a.sa + (r0 / a.blk) * a.kb;
+    const uint8_t* sb_row = MODE == kGateUp ? a.sb + (r0 / a.blk) * a.kb : sa_row;
     for (int tile = 0; tile < ntiles; ++tile) {
       const int nt = min(kTileN, a.M - tile * kTileN);
       if (!stage_once) stage_tile(tile);
       const __half* xrow = act + min(g, a.rows_act - 1) * fp8_act_stride(a.K) + 4 * t;
       const uint8_t* lrow = st + ((mj & 1) * 8 + mr) * RS + (mj >> 1) * 16;
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int c = c0; c < c1; ++c) {
+      for (int c = c0; c < c1 && a.blk == 32; ++c) {
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {  // one 32x32 scale tile per step
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t wa0, wb0, wa1, wb1;
+          ldmatrix_x4(wa0, wb0, wa1, wb1, lrow + c * 128 + jj * 32);
+          const uint2 x0 = *reinterpret_cast<const uint2*>(xrow + c * 128 + jj * 32);
+          const uint2 x1 = *reinterpret_cast<const uint2*>(xrow + c * 128 + jj * 32 + 16);
+          mma_f16_16816(d, e4m3x2_to_f16x2<0>(wa0), e4m3x2_to_f16x2<0>(wb0),
+                        e4m3x2_to_f16x2<1>(wa0), e4m3x2_to_f16x2<1>(wb0), x0.x, x0.y);
+          mma_f16_16816(d, e4m3x2_to_f16x2<0>(wa1), e4m3x2_to_f16x2<0>(wb1),
+                        e4m3x2_to_f16x2<1>(wa1), e4m3x2_to_f16x2<1>(wb1), x1.x, x1.y);
+          const uint32_t ca = __ldg(sa_row + 4 * c + jj), cb = __ldg(sb_row + 4 * c + jj);
+          bad |= (ca == 255u) | (cb == 255u);
+          const float fa = e8m0_to_f32(ca), fb = e8m0_to_f32(cb);
+          acc[0] = fmaf(d[0], fa, acc[0]);
+          acc[1] = fmaf(d[1], fa, acc[1]);
+          acc[2] = fmaf(d[2], fb, acc[2]);
+          acc[3] = fmaf(d[3], fb, acc[3]);
+        }
+      }
+      for (int c = c0; c < c1 && a.blk == 128; ++c) {
         float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -234,6 +262,11 @@ static qk_status fp8_go(Fp8Args& a, int units, size_t budget, cudaStream_t st, b
 
 qk_status fp8_linear_launch(const void* x, int M, int K, const uint8_t* w, const uint8_t* ws, int N,
                             void* y, int y_bf16, cudaStream_t st) {
+  return fp8_linear_launch_blk(x, M, K, w, ws, N, y, y_bf16, 128, st);
+}
+
+qk_status fp8_linear_launch_blk(const void* x, int M, int K, const uint8_t* w, const uint8_t* ws, int N,
+                                void* y, int y_bf16, int blk, cudaStream_t st) {
   Fp8Args a = {};
   a.x = static_cast<const uint16_t*>(x);
   a.wa = w;
@@ -241,7 +274,8 @@ qk_status fp8_linear_launch(const void* x, int M, int K, const uint8_t* w, const
   a.M = M;
   a.K = K;
   a.N = N;
-  a.kb = (K + 127) / 128;
+  a.blk = blk;
+  a.kb = (K + blk - 1) / blk;
   a.y = y;
   a.y_bf16 = y_bf16;
   return fp8_go<kLinear>(a, N / 16, 200 * 1024, st, false);
@@ -254,6 +288,12 @@ size_t fp8_ffn_workspace_bytes(int M, int H, int I) {
 qk_status fp8_ffn_launch(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
                          const uint8_t* wu, const uint8_t* su, const uint8_t* wd, const uint8_t* sd,
                          float* y, void* ws, cudaStream_t st) {
+  return fp8_ffn_launch_blk(x, M, H, I, wg, sg, wu, su, wd, sd, y, ws, 128, st);
+}
+
+qk_status fp8_ffn_launch_blk(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
+                             const uint8_t* wu, const uint8_t* su, const uint8_t* wd, const uint8_t* sd,
+                             float* y, void* ws, int blk, cudaStream_t st) {
   float* h = static_cast<float*>(ws);
   float* hmax = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256((size_t)M * I * 4));
   Fp8Args a = {};
@@ -265,7 +305,8 @@ qk_status fp8_ffn_launch(const void* x, int M, int H, int I, const uint8_t* wg, 
   a.M = M;
   a.K = H;
   a.N = I;
-  a.kb = (H + 127) / 128;
+  a.blk = blk;
+  a.kb = (H + blk - 1) / blk;
   a.hout = h;
   a.hmax_out = hmax;
   qk_status rc = fp8_go<kGateUp>(a, I / 8, 132 * 1024, st, false);
@@ -278,7 +319,8 @@ qk_status fp8_ffn_launch(const void* x, int M, int H, int I, const uint8_t* wg, 
   b.M = M;
   b.K = I;
   b.N = H;
-  b.kb = (I + 127) / 128;
+  b.blk = blk;
+  b.kb = (I + blk - 1) / blk;
   b.y = y;
   return fp8_go<kDownAcc>(b, H / 16, 92 * 1024, st, true);
 }

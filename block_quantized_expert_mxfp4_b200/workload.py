@@ -108,14 +108,15 @@ class Fp8Shared:
         return sum(t.numel() for t in (self.wg, self.sg, self.wu, self.su, self.wd, self.sd))
 
 
-def make_fp8_shared(seed: int, layer: int, H: int, I: int, device="cuda") -> Fp8Shared:
+def make_fp8_shared(seed: int, layer: int, H: int, I: int, device="cuda", block: int = 128) -> Fp8Shared:
     """Shared expert gate/up [I][H], down [H][I]: e4m3 codes uniform over the
-    254 non-NaN codes, UE8M0 tile exponents uniform in 2^-9..2^0."""
+    254 non-NaN codes, UE8M0 exponents uniform in 2^-9..2^0, one per
+    block x block tile (128, or 32 for the V4.1 layout)."""
     out = []
     for pi, (rows, cols) in zip((synth.TID.SH_GATE, synth.TID.SH_UP, synth.TID.SH_DOWN),
                                 ((I, H), (I, H), (H, I))):
         w = synth.fp8_codes(seed, synth.TID.of(layer, pi, 0), rows * cols, device).view(rows, cols)
-        s = synth.scale_codes(seed, synth.TID.of(layer, pi, 1), (rows // 128) * (cols // 128),
-                              118, 127, device).view(rows // 128, cols // 128)
+        s = synth.scale_codes(seed, synth.TID.of(layer, pi, 1), (rows // block) * (cols // block),
+                              118, 127, device).view(rows // block, cols // block)
         out += [w, s]
     return Fp8Shared(*out)

@@ -10,6 +10,8 @@
  *               "What's actually different" and the v0.2.3 update.
  *  [IQ2-FP8]    "DeepSeek-V4-Flash-IQ2XXS-Q2K-FP8-120GB-target", component table.
  *  [W4A16-FP8]  "DeepSeek-V4-Flash-W4A16-FP8", "Architecture & precision".
+ *  [V41-Q2]     "DeepSeek-V4.1-Flash mixed-Q2 GGUF (IQ2_XXS gate/up + Q2_K
+ *               down)", "Recipe".
  *
  * Storage formats (the byte layouts are the interface):
  *  MXFP4   nibbles  uint8 [E][rows][cols/2]  element 2i = low nibble of byte i
@@ -209,24 +211,28 @@ qk_status quant_convert_nvfp4_to_mxfp4(const uint8_t* e4m3, const float* scale_2
 
 /* ------------------------------------------------------------------------
  * fp8_block_linear -- y[M][N] = x[M][K] . dq(W)^T, dq = e4m3 * 2^(s-127) per
- * 128x128 tile.  [IQ2-FP8] component table ("FP8 E4M3, block-128, UE8M0
- * scales"); [W4A16-FP8] ("FP8_BLOCK 128x128").
- *  x bf16 [M][K]; w e4m3 [N][K]; w_scale ue8m0 [ceil(N/128)][ceil(K/128)];
- *  y fp32 or bf16 [M][N].  N multiple of 16, K multiple of 128, M >= 1.
+ * B x B tile, B = scale_block.  [IQ2-FP8] component table ("FP8 E4M3,
+ * block-128, UE8M0 scales"); [W4A16-FP8] ("FP8_BLOCK 128x128"); [V41-Q2]
+ * "Recipe": DeepSeek-V4.1's FP8 dense weights carry 32x32 E8M0 block
+ * scales where V4's carry 128x128.
+ *  x bf16 [M][K]; w e4m3 [N][K]; w_scale ue8m0 [ceil(N/B)][ceil(K/B)];
+ *  scale_block B = 128 or 32; y fp32 or bf16 [M][N].
+ *  N multiple of 16, K multiple of 128, M >= 1.
  * Errors: QK_ERR_INVALID_ARG, QK_ERR_CUDA; device: QK_ERR_NAN_SCALE.
  * ---------------------------------------------------------------------- */
 qk_status fp8_block_linear(const void* x_bf16, int32_t M, int32_t K, const uint8_t* w,
-                           const uint8_t* w_scale, int32_t N, void* y, int32_t y_is_bf16,
-                           qk_stream_t stream);
+                           const uint8_t* w_scale, int32_t N, int32_t scale_block, void* y,
+                           int32_t y_is_bf16, qk_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * fp8_shared_expert_forward -- the shared expert as a SwiGLU FFN with FP8
- * block-128 weights, ADDED into an fp32 output:
+ * block-scaled weights (B x B tiles, B = scale_block, 128 or 32), ADDED into
+ * an fp32 output:
  *   y[t] += down( silu(gate x[t]) * up x[t] )
  * Shared experts are kept at 8 bits on the pages ([REAP25] MXFP8, [REAP-K180]
  * Q8_0); FP8 E4M3 block-128 is the dense-layer format of [IQ2-FP8].
- *  x bf16 [M][H]; gate/up e4m3 [I][H] + scales [I/128][H/128];
- *  down e4m3 [H][I] + scales [H/128][I/128]; y fp32 [M][H] (read and written).
+ *  x bf16 [M][H]; gate/up e4m3 [I][H] + scales [I/B][H/B];
+ *  down e4m3 [H][I] + scales [H/B][I/B]; y fp32 [M][H] (read and written).
  *  H, I multiples of 128; workspace >= fp8_shared_expert_workspace_size().
  * Errors: as fp8_block_linear, plus QK_ERR_WORKSPACE.
  * ---------------------------------------------------------------------- */
@@ -235,8 +241,9 @@ size_t fp8_shared_expert_workspace_size(int32_t M, int32_t hidden, int32_t inter
 qk_status fp8_shared_expert_forward(const void* x_bf16, int32_t M, int32_t hidden, int32_t inter,
                                     const uint8_t* w_gate, const uint8_t* s_gate,
                                     const uint8_t* w_up, const uint8_t* s_up,
-                                    const uint8_t* w_down, const uint8_t* s_down, float* y,
-                                    void* workspace, size_t workspace_bytes, qk_stream_t stream);
+                                    const uint8_t* w_down, const uint8_t* s_down, int32_t scale_block,
+                                    float* y, void* workspace, size_t workspace_bytes,
+                                    qk_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Status.  qk_last_device_status synchronizes `stream`, returns the first

@@ -130,10 +130,13 @@ def test_forward_argument_errors_are_synchronous():
     assert L.quant_convert_mxfp4_to_nvfp4(p, 2, 4, 48, p, p, p, None) == qk.QK_ERR_INVALID_ARG
     assert L.quant_convert_nvfp4_to_mxfp4(p, p, 2, 4, 48, p, p, None) == qk.QK_ERR_INVALID_ARG
     assert L.quant_convert_nvfp4_to_mxfp4(None, p, 2, 4, 64, p, p, None) == qk.QK_ERR_INVALID_ARG
-    assert L.fp8_block_linear(p, 1, 100, p, p, 16, p, 0, None) == qk.QK_ERR_INVALID_ARG
+    assert L.fp8_block_linear(p, 1, 100, p, p, 16, 128, p, 0, None) == qk.QK_ERR_INVALID_ARG
+    assert L.fp8_block_linear(p, 1, 128, p, p, 16, 64, p, 0, None) == qk.QK_ERR_INVALID_ARG  # tile
     assert L.fp8_shared_expert_workspace_size(8, 4096, 2048) > 0
-    assert L.fp8_shared_expert_forward(p, 8, 4096, 2048, p, p, p, p, p, p, p, p, 0, None) == \
+    assert L.fp8_shared_expert_forward(p, 8, 4096, 2048, p, p, p, p, p, p, 128, p, p, 0, None) == \
         qk.QK_ERR_WORKSPACE
+    assert L.fp8_shared_expert_forward(p, 8, 4096, 2048, p, p, p, p, p, p, 16, p, p, 1 << 30, None) == \
+        qk.QK_ERR_INVALID_ARG
 
 
 def test_noalloc_entry_rejects_before_any_device_work():

@@ -48,3 +48,30 @@ def test_fp8_shared_expert_accumulates(M):
     assert qk.qk_last_device_status() == qk.QK_OK
     so = oracle.fp8_swiglu_ffn(x, *(t.cpu() for t in (sh.wg, sh.sg, sh.wu, sh.su, sh.wd, sh.sd)))
     assert_parity((y.cpu() - y0).numpy(), so, what=f"shared expert M={M}")
+
+
+@pytest.mark.parametrize("M,K,N", [(8, 4096, 2048), (3, 512, 96), (1, 128, 16)])
+def test_fp8_block_linear_32x32_tiles(M, K, N):
+    """32x32 E8M0 tiles (the DeepSeek-V4.1 layout)."""
+    w = synth.fp8_codes(5, M + K, N * K, "cuda").view(N, K)
+    s = synth.scale_codes(5, N + K, ((N + 31) // 32) * (K // 32), 118, 127, "cuda").view((N + 31) // 32, K // 32)
+    x = synth.activations(M + 1, M, K)
+    y = torch.empty((M, N), device="cuda")
+    qk.fp8_block_linear(x.cuda(), w, s, y, scale_block=32)
+    assert qk.qk_last_device_status() == qk.QK_OK
+    yo = oracle.fp8_block_linear(x, w.cpu(), s.cpu(), 32)
+    assert_parity(y.cpu().numpy(), yo, what=f"fp8 linear 32x32 {M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("M", [8, 1])
+def test_fp8_shared_expert_32x32_tiles(M):
+    H, I = 4096, 2048
+    sh = workload.make_fp8_shared(1, 0, H, I, block=32)
+    x = synth.activations(12, M, H)
+    y = torch.zeros((M, H), device="cuda")
+    ws = torch.empty(qk.fp8_shared_expert_workspace_size(M, H, I), dtype=torch.uint8, device="cuda")
+    qk.fp8_shared_expert_forward(x.cuda(), sh.wg, sh.sg, sh.wu, sh.su, sh.wd, sh.sd, y, ws, scale_block=32)
+    assert qk.qk_last_device_status() == qk.QK_OK
+    hs = workload.make_fp8_shared(1, 0, H, I, device="cpu", block=32)
+    so = oracle.fp8_swiglu_ffn(x, hs.wg, hs.sg, hs.wu, hs.su, hs.wd, hs.sd, block=32)
+    assert_parity(y.cpu().numpy(), so, what=f"shared expert 32x32 M={M}")

@@ -192,9 +192,12 @@ def test_route_ties_take_lower_id_and_minus_inf():
 
 # ------------------------------------------------------------------ FP8 --
 
-def test_fp8_block_linear_matches_library_formulation():
+@pytest.mark.parametrize("b", [128, 32])
+def test_fp8_block_linear_matches_library_formulation(b):
+    """128x128 scale tiles (V4) and 32x32 (V4.1: "DeepSeek-V4.1-Flash mixed-Q2
+    GGUF (IQ2_XXS gate/up + Q2_K down)", "Recipe")."""
     rng = np.random.default_rng(11)
-    M, K, N, b = 3, 256, 384, 128
+    M, K, N = 3, 256, 384
     w = synth.fp8_codes(1, 7, N * K).numpy().reshape(N, K)
     s = rng.integers(118, 128, (N // b, K // b), dtype=np.uint8)
     x = synth.activations(4, M, K)
@@ -205,13 +208,14 @@ def test_fp8_block_linear_matches_library_formulation():
     s2 = s.copy()
     s2[1, 0] += 1
     y2 = oracle.fp8_block_linear(x, w, s2, b)
-    assert np.array_equal(y2[:, :128], y[:, :128]) and np.array_equal(y2[:, 256:], y[:, 256:])
-    assert not np.array_equal(y2[:, 128:256], y[:, 128:256])
+    assert np.array_equal(y2[:, :b], y[:, :b]) and np.array_equal(y2[:, 2 * b:], y[:, 2 * b:])
+    assert not np.array_equal(y2[:, b:2 * b], y[:, b:2 * b])
 
 
-def test_fp8_swiglu_ffn_matches_library_formulation():
+@pytest.mark.parametrize("b", [128, 32])
+def test_fp8_swiglu_ffn_matches_library_formulation(b):
     rng = np.random.default_rng(12)
-    M, H, I, b = 2, 256, 128, 128
+    M, H, I = 2, 256, 128
     mats = []
     for t, (rows, cols) in enumerate(((I, H), (I, H), (H, I))):
         mats.append(synth.fp8_codes(2, t, rows * cols).numpy().reshape(rows, cols))
