@@ -57,6 +57,8 @@ def parse():
                     help="profiling only: fewer experts in the prefill layer (0: the workload's 256)")
     ap.add_argument("--prefill-tokens", type=int, default=0,
                     help="profiling only: fewer prefill tokens (0: the workload's 2048)")
+    ap.add_argument("--prefill-act", choices=["none", "e4m3", "mxfp4"], default="none",
+                    help="activation mode of the prefill layer (default: bf16 activations)")
     return ap.parse_args()
 
 
@@ -389,6 +391,7 @@ def run_prefill(args, rank, world, dev):
         import dataclasses
         wl = dataclasses.replace(wl, E=args.prefill_experts or wl.E, T=args.prefill_tokens or wl.T)
     T, k = wl.T, wl.k
+    aq = {"none": qk.QK_ACT_NONE, "e4m3": qk.QK_ACT_E4M3, "mxfp4": qk.QK_ACT_MXFP4}[args.prefill_act]
     layer = workload.make_layer(wl, seed=rank, layer=0)
     lay = layer.c()
     x = synth.activations(rank, T, wl.H).to(dev)
@@ -397,20 +400,20 @@ def run_prefill(args, rank, world, dev):
     w = torch.empty((T, k), dtype=torch.float32, device=dev)
     qk.moe_route_topk(lg, k, ids, w)
     y = torch.empty((T, wl.H), dtype=torch.float32, device=dev)
-    wsp = torch.empty(qk.moe_expert_workspace_size(lay, T, k), dtype=torch.uint8, device=dev)
+    wsp = torch.empty(qk.moe_expert_workspace_size(lay, T, k, aq), dtype=torch.uint8, device=dev)
     touched = int(torch.unique(ids).numel())
     wbytes = touched * layer.expert_bytes()
     flops = 2 * 3 * wl.H * wl.I * T * k
     s = torch.cuda.Stream(device=dev)
     for _ in range(3):
-        qk.moe_expert_forward(lay, x, ids, w, y, wsp)
+        qk.moe_expert_forward(lay, x, ids, w, y, wsp, act_quant=aq)
     torch.cuda.synchronize()
     if qk.qk_last_device_status() != qk.QK_OK:
         raise RuntimeError("device status after prefill warm-up")
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
-            qk.moe_expert_forward(lay, x, ids, w, y, wsp, stream=s)
+            qk.moe_expert_forward(lay, x, ids, w, y, wsp, act_quant=aq, stream=s)
     torch.cuda.synchronize()
     K = args.prefill_steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -441,7 +444,9 @@ def run_prefill(args, rank, world, dev):
     tpeak, tkind = 2 * bf16, f"{src} bf16 x 2 (nominal fp8/bf16 ratio): the MMA kind used, kind::mxf8f6f4"
     return {
         "workload": f"prefill MoE layer: {T} tokens, {wl.E} experts, top-6 Zipf(s=1) routing, hidden 4096, "
-                    "intermediate 2048, MXFP4 gate/up/down, bf16 N(0,1) activations",
+                    "intermediate 2048, MXFP4 gate/up/down, bf16 N(0,1) activations"
+                    + ("" if aq == qk.QK_ACT_NONE else f", quantized in the layer to {args.prefill_act}"
+                       " (one e8m0 scale per 32)"),
         "tokens_per_s": round(T * world / t, 1), "ms_per_layer": round(t * 1e3, 4), "steps": K,
         "experts_touched": touched,
         "hbm": {"bytes_per_layer": wbytes, "achieved_gbs": round(wbytes / t / 1e9, 1), "peak_gbs": peak,
@@ -449,8 +454,11 @@ def run_prefill(args, rank, world, dev):
         "tensor": {"flop_per_layer": flops, "achieved_tflops": round(flops / t / 1e12, 1),
                    "peak_tflops": tpeak, "peak_kind": tkind, "frac": round(flops / t / 1e12 / tpeak, 4),
                    "frac_of_fp4_peak": round(flops / t / 1e12 / (4 * bf16), 4)},
-        "path": "counting sort by expert; x as 2 exact e4m3 terms; block-scaled tcgen05 grouped GEMMs "
-                "(e2m1 weights + e8m0 scales as stored): gate/up, SwiGLU + 3-term h split, down; combine",
+        "path": ("counting sort by expert; x as 2 exact e4m3 terms; block-scaled tcgen05 grouped GEMMs "
+                 "(e2m1 weights + e8m0 scales as stored): gate/up, SwiGLU + 3-term h split, down; combine")
+        if aq == qk.QK_ACT_NONE else
+        (f"counting sort by expert; x and h quantized to {args.prefill_act} (one term, the other term slots "
+         "zero); block-scaled tcgen05 grouped GEMMs; combine"),
     }
 
 
