@@ -155,3 +155,37 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         _lib.load()
+
+
+def test_wrappers_of_the_newer_arguments_marshal_them():
+    """The Python wrappers pass scale_block, act_quant and the reverse
+    conversion's arguments in the header's order: each invalid value comes
+    back as its synchronous error (stream 0: no device is touched)."""
+    import torch
+
+    def code(fn):
+        with pytest.raises(qk.QkError) as ei:
+            fn()
+        return ei.value.code
+
+    e4 = torch.zeros((2, 4, 3), dtype=torch.uint8)             # K = 48: not a multiple of 32
+    assert code(lambda: qk.quant_convert_nvfp4_to_mxfp4(e4, torch.ones(2), torch.zeros((2, 4, 1), dtype=torch.uint8),
+                                                        torch.zeros(1, dtype=torch.int64), stream=0)) == \
+        qk.QK_ERR_INVALID_ARG
+    x = torch.zeros((1, 128), dtype=torch.bfloat16)
+    w = torch.zeros((16, 128), dtype=torch.uint8)
+    s = torch.zeros((1, 4), dtype=torch.uint8)
+    y = torch.zeros((1, 16))
+    assert code(lambda: qk.fp8_block_linear(x, w, s, y, stream=0, scale_block=64)) == qk.QK_ERR_INVALID_ARG
+    wg = torch.zeros((128, 128), dtype=torch.uint8)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8)
+    assert code(lambda: qk.fp8_shared_expert_forward(x, wg, s, wg, s, wg, s, torch.zeros((1, 128)), ws,
+                                                     stream=0, scale_block=16)) == qk.QK_ERR_INVALID_ARG
+    lay = _fake_layer()
+    ids = torch.zeros((1, 6), dtype=torch.int32)
+    wt = torch.zeros((1, 6))
+    yy = torch.zeros((1, 4096))
+    assert code(lambda: qk.moe_expert_forward(lay, torch.zeros((1, 4096), dtype=torch.bfloat16), ids, wt, yy, ws,
+                                              act_quant=7, stream=0)) == qk.QK_ERR_INVALID_ARG
+    assert qk.moe_expert_workspace_size(lay, 1, 6, 7) == 0
+    assert qk.moe_expert_workspace_size(lay, 1, 6, qk.QK_ACT_E4M3) > 0
