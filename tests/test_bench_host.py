@@ -69,3 +69,42 @@ def test_reference_arm_prints_the_contract_line():
 def test_reference_arm_other_ranks_exit_quietly(rank):
     r = _bench({"RANK": rank, "WORLD_SIZE": "2"}, "--impl", "reference", "--steps", "1", "--warmup", "0")
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_kernel_hash_ignores_comments_only():
+    """The recorded decode traffic is used only while the decode kernels'
+    code hashes to the recorded value: comment edits keep the hash, code
+    edits change it, and no string literal in those files holds a comment
+    marker (which would make the comment stripping cut code)."""
+    import re
+    import shutil
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from block_quantized_expert_mxfp4_b200 import build as b
+
+    assert bench._code_only("int a; // note\n/* block\n comment */ int b;\n\n") == "int a;\n int b;"
+    names = ("qk_dmx.cu", "qk_route_table.cuh", "qk_device.cuh", "qk_common.cuh", "qk_group.cuh",
+             "qk_internal.h", "qk_tmap.h")
+    for n in names:
+        for lit in re.findall(r'"(?:[^"\\\n]|\\.)*"', open(os.path.join(b.CSRC, n)).read()):
+            assert "//" not in lit and "/*" not in lit, (n, lit)
+    tmp = os.path.join(ROOT, "tests", "_build", "hash_check")
+    shutil.rmtree(tmp, ignore_errors=True)
+    os.makedirs(tmp)
+    for n in names:
+        shutil.copy(os.path.join(b.CSRC, n), tmp)
+    h0 = bench.kernel_source_hash()
+    orig = b.CSRC
+    try:
+        b.CSRC = tmp
+        assert bench.kernel_source_hash() == h0
+        p = os.path.join(tmp, "qk_dmx.cu")
+        src = open(p).read()
+        open(p, "w").write(src.replace("namespace qk {", "namespace qk {\n// a comment added\n", 1))
+        assert bench.kernel_source_hash() == h0
+        open(p, "w").write(src.replace("namespace qk {", "namespace qk {\nconstexpr int kUnused = 1;\n", 1))
+        assert bench.kernel_source_hash() != h0
+    finally:
+        b.CSRC = orig
+        shutil.rmtree(tmp, ignore_errors=True)
