@@ -3,7 +3,7 @@ block-128) weights: a C-ABI CUDA library (libqk.so, sm_100a) and its thin
 Python binding.  See include/qk.h for the ABI."""
 from ._lib import (  # noqa: F401
     LIB_PATH, QK_ACT_E4M3, QK_ACT_MXFP4, QK_ACT_NONE, QK_ERR_CUDA, QK_ERR_INVALID_ARG,
-    QK_ERR_NAN_SCALE, QK_ERR_TIMEOUT, QK_ERR_UNSUPPORTED, QK_ERR_WORKSPACE, QK_FMT_MXFP4,
+    QK_ERR_NAN_SCALE, QK_ERR_NONFINITE, QK_ERR_TIMEOUT, QK_ERR_UNSUPPORTED, QK_ERR_WORKSPACE, QK_FMT_MXFP4,
     QK_FMT_NVFP4, QK_OK, QkError, fp8_block_linear, fp8_shared_expert_forward,
     fp8_shared_expert_workspace_size, load, make_layer, make_weight, moe_expert_forward,
     moe_expert_forward_noalloc,

@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqk.so")
 
 QK_OK, QK_ERR_INVALID_ARG, QK_ERR_UNSUPPORTED, QK_ERR_WORKSPACE = 0, 1, 2, 3
-QK_ERR_NAN_SCALE, QK_ERR_CUDA, QK_ERR_TIMEOUT = 4, 5, 6
+QK_ERR_NAN_SCALE, QK_ERR_CUDA, QK_ERR_TIMEOUT, QK_ERR_NONFINITE = 4, 5, 6, 7
 QK_FMT_MXFP4, QK_FMT_NVFP4 = 1, 2
 QK_ACT_NONE, QK_ACT_MXFP4, QK_ACT_E4M3 = 0, 1, 2
 

@@ -2,6 +2,8 @@
 // argument validation, workspace carving, dispatch, and the device status word.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "qk_actq.cuh"
 #include "qk_convert_nv.h"
 #include "qk_fp8.h"
@@ -11,6 +13,45 @@
 namespace qk {
 __device__ int g_status = 0;
 __device__ unsigned long long g_wait_limit_ns = 1000000000ull;
+
+namespace {
+struct SmemAttr {
+  const void* fn;
+  int dev;
+  size_t bytes;
+};
+constexpr int kSmemAttrs = 256;
+SmemAttr g_smem_attr[kSmemAttrs];
+int g_smem_attr_n = 0;
+std::mutex g_smem_attr_mu;
+}  // namespace
+
+bool smem_attr(const void* kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return true;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(g_smem_attr_mu);
+  int slot = -1;
+  for (int i = 0; i < g_smem_attr_n; ++i)
+    if (g_smem_attr[i].fn == kernel && g_smem_attr[i].dev == dev) {
+      if (g_smem_attr[i].bytes >= bytes) return true;
+      slot = i;
+      break;
+    }
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+    return false;
+  if (slot < 0 && g_smem_attr_n < kSmemAttrs) slot = g_smem_attr_n++;
+  if (slot >= 0) g_smem_attr[slot] = {kernel, dev, bytes};
+  return true;
+}
+
+void smem_attr_forget(const void* kernel) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  std::lock_guard<std::mutex> lock(g_smem_attr_mu);
+  for (int i = 0; i < g_smem_attr_n; ++i)
+    if (g_smem_attr[i].fn == kernel && g_smem_attr[i].dev == dev) g_smem_attr[i].bytes = 0;
+}
 }  // namespace qk
 
 using namespace qk;
@@ -52,8 +93,8 @@ size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_
     return act_quant_ok(L, act_quant) ? group_workspace_bytes(L, n_tokens, top_k) : 0;
   if (n_tokens > decode_chunk(top_k))
     return group_workspace_bytes(L, n_tokens, top_k);
-  if (dmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter))
-    return dmx_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
+  if (dq_eligible(L->gate, L->up, L->down, L->hidden, L->inter))
+    return dq_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
   return decode_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
 }
 
@@ -92,9 +133,9 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
   if (act_quant != QK_ACT_NONE)
     return group_forward_act(a, act_quant, workspace, reinterpret_cast<cudaStream_t>(stream));
   if (n_tokens > decode_chunk(top_k)) return group_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
-  // All-MXFP4 layers: weights straight to the block-scaled tensor cores.
-  if (dmx_eligible(a.gate, a.up, a.down, a.H, a.I))
-    return dmx_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
+  // All-MXFP4 layers: weights straight to the fp4 block-scaled tensor cores.
+  if (dq_eligible(a.gate, a.up, a.down, a.H, a.I))
+    return dq_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
   decode_carve(a, workspace);
   return decode_forward(a, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -182,6 +223,7 @@ const char* qk_status_string(qk_status s) {
     case QK_ERR_NAN_SCALE: return "NaN scale code";
     case QK_ERR_CUDA: return "CUDA runtime error";
     case QK_ERR_TIMEOUT: return "bounded device wait ran out";
+    case QK_ERR_NONFINITE: return "activation or fp32 intermediate not finite";
     default: return "unknown status";
   }
 }

@@ -56,8 +56,10 @@ __device__ inline void stage_bf16_rows(const uint16_t* __restrict__ x, const int
         const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          v[j] = fmaxf(v[j], fabsf(bf16_bits_to_f32(w[i] & 0xFFFFu)));
-          v[j] = fmaxf(v[j], fabsf(bf16_bits_to_f32(w[i] >> 16)));
+          const float a = bf16_bits_to_f32(w[i] & 0xFFFFu), b = bf16_bits_to_f32(w[i] >> 16);
+          if (!(finite_bits(a) && finite_bits(b))) set_status(QK_ERR_NONFINITE);
+          v[j] = fmaxf(v[j], fabsf(a));
+          v[j] = fmaxf(v[j], fabsf(b));
         }
       }
     }
@@ -140,17 +142,16 @@ inline int device_attr(cudaDeviceAttr attr) {
 inline int num_sms() { return device_attr(cudaDevAttrMultiProcessorCount); }
 inline int max_smem_optin() { return device_attr(cudaDevAttrMaxSharedMemoryPerBlockOptin); }
 
-// Launch `kernel<<<grid, kThreads, smem, st>>>(args)`, optionally as a
-// programmatic dependent launch of the previous kernel on the stream.
-template <typename Kern, typename Args>
-inline qk_status launch_k(Kern kernel, size_t smem, int grid, const Args& args, cudaStream_t st,
-                          bool pdl) {
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return QK_ERR_CUDA;
+// Launch kernel<<<grid, block, smem, st>>>(args...), optionally as a
+// programmatic dependent launch of the previous kernel on the stream, with
+// the shared-memory attribute set once per kernel and device (smem_attr).
+template <typename... KArgs, typename... Args>
+inline qk_status launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                           bool pdl, Args&&... args) {
+  if (!smem_attr(reinterpret_cast<const void*>(kernel), smem)) return QK_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -158,7 +159,21 @@ inline qk_status launch_k(Kern kernel, size_t smem, int grid, const Args& args, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, args) == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess && smem > 48 * 1024) {  // the attribute may have been cleared (device reset)
+    (void)cudaGetLastError();
+    smem_attr_forget(reinterpret_cast<const void*>(kernel));
+    if (!smem_attr(reinterpret_cast<const void*>(kernel), smem)) return QK_ERR_CUDA;
+    e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  }
+  return e == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+}
+
+// Launch `kernel<<<grid, kThreads, smem, st>>>(args)` (see launch_ex).
+template <typename Kern, typename Args>
+inline qk_status launch_k(Kern kernel, size_t smem, int grid, const Args& args, cudaStream_t st,
+                          bool pdl) {
+  return launch_ex(kernel, dim3(grid), dim3(kThreads), smem, st, pdl, args);
 }
 
 }  // namespace qk

@@ -444,7 +444,7 @@ __device__ __forceinline__ void stage_h_raw(const DecodeArgs& a, DHead& S, __hal
 // per-instruction cost of a tensor copy off any single warp's critical path.
 template <int FA, int FB, bool GATEUP>
 __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ DArgs P) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];  // rounded up to 1024 below, at run time
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   DHead& S = *reinterpret_cast<DHead*>(smem);
   const DecodeArgs& a = P.a;
@@ -639,6 +639,7 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
         yv = fmaf(a.w[p], __ldcg(ures + (((size_t)pv * RT + r) * 32 + ln + (j >> 1)) * 4 + el + (j & 1)), yv);
       }
       const size_t o = (size_t)tok * a.H + r * 16 + m;
+      if (!finite_bits(yv)) set_status(QK_ERR_NONFINITE);
       if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(yv);
       else reinterpret_cast<float*>(a.y)[o] = yv;
     }
@@ -686,6 +687,7 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
         hm[jj] = 0.f;
         if (col < n) {
           const float hv = silu_mul(fv[jj], fv[2 + jj]);
+          if (!finite_bits(hv)) set_status(QK_ERR_NONFINITE);
           const int p = S.R.pair_list[S.R.v_p0[v] + col];
           a.h[(size_t)p * a.I + r * 8 + g] = hv;
           hm[jj] = fabsf(hv);
@@ -919,21 +921,7 @@ static bool encode_rows(CUtensorMap* m, const uint8_t* q, int64_t rows, int K, i
 template <int FA, int FB, bool GATEUP>
 static qk_status go(DArgs& P, cudaStream_t st, bool pdl) {
   const int grid = std::max(1, std::min(num_sms(), P.U_max));
-  auto kern = k_decode<FA, FB, GATEUP>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P.G.smem) !=
-      cudaSuccess)
-    return QK_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kDW * 32);
-  cfg.dynamicSmemBytes = P.G.smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, P) == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  return launch_ex(k_decode<FA, FB, GATEUP>, dim3(grid), dim3(kDW * 32), (size_t)P.G.smem, st, pdl, P);
 }
 
 // Geometry of one kernel: tensor-map mode when the maps encode, else rows by cp.async.

@@ -252,6 +252,16 @@ __device__ __forceinline__ int f16_shift_for(float amax) {
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// True when every value is finite (not inf, not NaN).  Non-finite inputs or
+// fp32 intermediates are reported as QK_ERR_NONFINITE.
+__device__ __forceinline__ bool finite_bits(float v) { return (__float_as_uint(v) & 0x7F800000u) != 0x7F800000u; }
+__device__ __forceinline__ bool all_finite32(const float (&v)[32]) {
+  bool ok = true;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) ok &= finite_bits(v[i]);
+  return ok;
+}
+
 }  // namespace qk
 
 // -------------------------------------------------------- tcgen05 / TMEM --

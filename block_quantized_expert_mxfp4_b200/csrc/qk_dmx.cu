@@ -199,7 +199,7 @@ namespace qk {
 template <bool GATEUP>
 __global__ void __launch_bounds__(kDThreads, 2) k_dmx(const __grid_constant__ DmxArgs G) {
   constexpr int NT = GATEUP ? 2 : 3;  // terms per pair
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];  // rounded up to 1024 below, at run time
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   // A blocks first: the MMA reads 128 rows (16 KB) from each 3-KB step block,
   // so the rows past a block's 24 fall on later blocks or the weight ring.
@@ -528,21 +528,8 @@ static bool d_map_weights(CUtensorMap* m, const uint8_t* q, int64_t rows, int K)
 
 template <bool GATEUP>
 static qk_status d_launch(const DmxArgs& A, cudaStream_t st) {
-  auto kern = k_dmx<GATEUP>;
   if (kDSmem > max_smem_optin()) return QK_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDSmem) != cudaSuccess)
-    return QK_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * num_sms());
-  cfg.blockDim = dim3(kDThreads);
-  cfg.dynamicSmemBytes = kDSmem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, A) == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  return launch_ex(k_dmx<GATEUP>, dim3(2 * num_sms()), dim3(kDThreads), (size_t)kDSmem, st, true, A);
 }
 
 qk_status dmx_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {

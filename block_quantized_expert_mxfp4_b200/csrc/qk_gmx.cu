@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
         v[q * 8 + 2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
       }
     }
+    if (!all_finite32(v)) set_status(QK_ERR_NONFINITE);
     uint32_t q0[8], q1[8];
     int c0, c1;
     if (act_quant == QK_ACT_NONE) {
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, in
       v[4 * q + 2] = __fdividef(g.z, 1.0f + __expf(-g.z)) * u.z;
       v[4 * q + 3] = __fdividef(g.w, 1.0f + __expf(-g.w)) * u.w;
     }
+    if (!all_finite32(v)) set_status(QK_ERR_NONFINITE);
     if (act_quant == QK_ACT_NONE) {
 #pragma unroll
       for (int term = 0; term < 3; ++term) {
@@ -255,7 +257,7 @@ __device__ __forceinline__ void gmx_tile(const TileList& L, int MB, int t, int& 
 template <bool GATEUP, int NT>
 __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ GmxArgs G) {
   constexpr int NPQ = NT == 2 ? kXTok1 / 4 : kXTok2 / 4;  // tokens per TMEM lane quadrant
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];  // rounded up to 1024 below, at run time
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sW = base;                                  // kXWS weight stages
   uint8_t* sT = sW + kXWS * kXStageW;                  // kXTS token stages
@@ -548,13 +550,9 @@ static bool x_map_weights(CUtensorMap* m, const uint8_t* q, int64_t rows, int K)
 
 template <bool GATEUP, int NT>
 static qk_status x_launch(const GmxArgs& A, cudaStream_t st) {
-  auto kern = k_gmx<GATEUP, NT>;
   static_assert(sizeof(GmxHead) <= 256, "head");
   if (kXSmem > max_smem_optin()) return QK_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kXSmem) != cudaSuccess)
-    return QK_ERR_CUDA;
-  kern<<<num_sms(), kXThreads, kXSmem, st>>>(A);
-  return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  return launch_ex(k_gmx<GATEUP, NT>, dim3(num_sms()), dim3(kXThreads), (size_t)kXSmem, st, false, A);
 }
 
 qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st) {

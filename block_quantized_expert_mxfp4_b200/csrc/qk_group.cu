@@ -157,13 +157,18 @@ __global__ void __launch_bounds__(kRowThreads) k_grp_scatter(GroupWs W, const ui
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
   const int nv = H / 8;
   float m = 0.f;
+  bool fin = true;
   for (int j = threadIdx.x; j < nv; j += kRowThreads) {
     const uint4 v = __ldg(src + j);
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      m = fmaxf(m, fmaxf(fabsf(bf16_bits_to_f32(wv[q] & 0xFFFFu)), fabsf(bf16_bits_to_f32(wv[q] >> 16))));
+    for (int q = 0; q < 4; ++q) {
+      const float a = bf16_bits_to_f32(wv[q] & 0xFFFFu), b = bf16_bits_to_f32(wv[q] >> 16);
+      fin &= finite_bits(a) && finite_bits(b);
+      m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+    }
   }
+  if (!fin) set_status(QK_ERR_NONFINITE);
   const int shift = block_shift(m, red);
   if (threadIdx.x < k) {
     const int p = t * k + threadIdx.x;
@@ -198,10 +203,13 @@ __global__ void __launch_bounds__(kRowThreads) k_grp_h16(GroupWs W, int E, int I
   const float4* src = reinterpret_cast<const float4*>(W.hperm + (size_t)r * I);
   const int nv = I / 4;
   float m = 0.f;
+  bool fin = true;
   for (int j = threadIdx.x; j < nv; j += kRowThreads) {
     const float4 v = __ldcg(src + j);
+    fin &= finite_bits(v.x) && finite_bits(v.y) && finite_bits(v.z) && finite_bits(v.w);
     m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
   }
+  if (!fin) set_status(QK_ERR_NONFINITE);
   const int shift = block_shift(m, red);
   if (threadIdx.x == 0) W.hshift[r] = shift;
   const float sc = pow2f(-shift);
@@ -232,6 +240,8 @@ __global__ void __launch_bounds__(256) k_grp_combine(GroupWs W, const float* __r
       acc.z = fmaf(ws[s], d.z, acc.z);
       acc.w = fmaf(ws[s], d.w, acc.w);
     }
+    if (!(finite_bits(acc.x) && finite_bits(acc.y) && finite_bits(acc.z) && finite_bits(acc.w)))
+      set_status(QK_ERR_NONFINITE);
     if (y_bf16) {
       __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y) + (size_t)t * H + 4 * j;
       yb[0] = __float2bfloat16_rn(acc.x);
@@ -304,7 +314,7 @@ __device__ __forceinline__ uint32_t f16x2_pow2(int e) {
 
 template <int FA, int FB, bool GATEUP>
 __global__ void __launch_bounds__(kGThreads, 1) k_ggemm(const __grid_constant__ GemmArgs G) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];  // rounded up to 1024 below, at run time
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sA = base;                      // kGAS f16 weight tiles (1024-aligned)
   uint8_t* sB = sA + kGAS * kGStageA;      // kGBS token stages
@@ -754,13 +764,9 @@ static bool g_map_tokens(CUtensorMap (&m)[kGNBox], const __half* x, int64_t P, i
 
 template <int FA, int FB, bool GATEUP>
 static qk_status g_launch(const GemmArgs& A, cudaStream_t st) {
-  auto kern = k_ggemm<FA, FB, GATEUP>;
   const int smem = g_smem_bytes(A.sc_stride);
   if (smem > max_smem_optin()) return QK_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return QK_ERR_CUDA;
-  kern<<<num_sms(), kGThreads, smem, st>>>(A);
-  return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  return launch_ex(k_ggemm<FA, FB, GATEUP>, dim3(num_sms()), dim3(kGThreads), (size_t)smem, st, false, A);
 }
 
 template <bool GATEUP>

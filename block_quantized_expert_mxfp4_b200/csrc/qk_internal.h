@@ -14,6 +14,13 @@ constexpr int kMaxStages = 6;   // deepest bulk-copy ring
 
 inline size_t align256(size_t n) { return (n + 255) / 256 * 256; }
 
+// Dynamic shared memory above the 48 KB default: cudaFuncSetAttribute is
+// called once per (kernel, device, size) and remembered, not on every launch.
+// smem_attr_forget drops the record (a launch that was refused, e.g. after a
+// cudaDeviceReset cleared the attribute, sets it again and retries once).
+bool smem_attr(const void* kernel, size_t bytes);
+void smem_attr_forget(const void* kernel);
+
 // Arguments of the decode kernels (passed by value as a kernel parameter).
 struct DecodeArgs {
   qk_weight gate, up, down;
@@ -38,6 +45,10 @@ qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
 bool dmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
 size_t dmx_workspace_bytes(int T, int k, int H, int I);
 qk_status dmx_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
+// Decode path on the fp4 x fp4 block-scaled tensor cores (kind::mxf4).
+bool dq_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
+size_t dq_workspace_bytes(int T, int k, int H, int I);
+qk_status dq_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
 size_t decode_workspace_bytes(int T, int k, int H, int I);
 void decode_carve(DecodeArgs& a, void* ws);
 

@@ -6,9 +6,11 @@
 // C caller embedded in another runtime that owns every device allocation (and
 // exposes no allocator to plugins), or a host that must not grow its device
 // footprint after start-up.  Such callers cannot size and pass a workspace per
-// call; here the scratch is part of the library image, its address resolved
-// once per device with cudaGetSymbolAddress.  Nothing is allocated: no
-// cudaMalloc/cudaFree, no allocating library.
+// call; here the scratch is part of the library image, its address looked up
+// with cudaGetSymbolAddress on every call (a host-side query: no device work),
+// so it is always the address in the context current at the call, also after
+// a cudaDeviceReset or in a second context on the same device.  Nothing is
+// allocated: no cudaMalloc/cudaFree, no allocating library.
 //
 // The kernels are the decode kernels of moe_expert_forward, unchanged; only
 // the origin of the workspace differs.  Nothing in the scratch has to start at
@@ -16,30 +18,20 @@
 // of every call.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "qk_internal.h"
 
 namespace qk {
 
-constexpr size_t kNoallocScratchBytes = (size_t)4 << 20;  // 4 MiB
-constexpr int kNoallocMaxDevices = 64;
+constexpr size_t kNoallocScratchBytes = (size_t)16 << 20;  // 16 MiB
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 
-static std::mutex g_noalloc_mu;
-static void* g_noalloc_ptr[kNoallocMaxDevices];
-
-// Address of the scratch array on the current device (resolved once per device).
-static void* noalloc_scratch(int dev) {
-  if (dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
-    g_noalloc_ptr[dev] = p;
-  }
-  return g_noalloc_ptr[dev];
+// Device address of the scratch array in the current context.  The host-side
+// name g_noalloc_scratch is only a stand-in; kernels get this address.
+static void* noalloc_scratch() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace qk
@@ -56,9 +48,7 @@ extern "C" qk_status moe_expert_forward_noalloc(const qk_moe_layer* L, const voi
   if (need == 0) return QK_ERR_INVALID_ARG;
   if (n_tokens == 0) return QK_OK;
   if (need > kNoallocScratchBytes) return QK_ERR_WORKSPACE;  // beyond the fixed array
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return QK_ERR_CUDA;
-  void* scratch = noalloc_scratch(dev);
+  void* scratch = noalloc_scratch();
   if (!scratch) return QK_ERR_CUDA;
   return moe_expert_forward(L, x_bf16, n_tokens, topk_ids, topk_w, top_k, y, y_is_bf16,
                             QK_ACT_NONE, scratch, kNoallocScratchBytes, stream);

@@ -10,8 +10,7 @@
 // selected entry is overwritten with NaN (never chosen again).
 #include <math.h>
 
-#include "qk_device.cuh"
-#include "qk_internal.h"
+#include "qk_common.cuh"
 
 namespace qk {
 
@@ -80,12 +79,7 @@ qk_status route_topk_launch(const float* logits, int T, int E, int k, int32_t* i
                             cudaStream_t st) {
   const int grid = (T + kRouteWarps - 1) / kRouteWarps;
   const size_t smem = (size_t)kRouteWarps * E * sizeof(float);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(k_route, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-    return QK_ERR_CUDA;
-  k_route<<<grid, kRouteWarps * 32, smem, st>>>(logits, T, E, k, ids, w);
-  return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+  return launch_ex(k_route, dim3(grid), dim3(kRouteWarps * 32), smem, st, false, logits, T, E, k, ids, w);
 }
 
 }  // namespace qk

@@ -57,7 +57,10 @@ enum {
   QK_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than the query */
   QK_ERR_NAN_SCALE = 4,   /* an e8m0 code 255 or an e4m3 scale code 0x7F/0xFF was read */
   QK_ERR_CUDA = 5,        /* a CUDA runtime call failed (launch, attribute, copy) */
-  QK_ERR_TIMEOUT = 6      /* a bounded device wait ran out; outputs are undefined */
+  QK_ERR_TIMEOUT = 6,     /* a bounded device wait ran out; outputs are undefined */
+  QK_ERR_NONFINITE = 7    /* an activation, or an fp32 intermediate (h = silu(gate) * up, y), is
+                             inf or NaN: an input was not finite or a sum overflowed fp32 (the
+                             kernels accumulate in fp32); the affected outputs are undefined */
 };
 
 enum { QK_FMT_MXFP4 = 1, QK_FMT_NVFP4 = 2 };
@@ -136,20 +139,22 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
 
 /* ------------------------------------------------------------------------
  * moe_expert_forward_noalloc -- moe_expert_forward (act_quant QK_ACT_NONE)
- * with its scratch taken from a fixed 4 MiB device array inside libqk.so
+ * with its scratch taken from a fixed 16 MiB device array inside libqk.so
  * instead of a caller workspace.  The pages have no counterpart: it exists for
  * callers that cannot allocate device memory on the call path (a C caller
  * embedded in a runtime that owns every device allocation).
  *  Arguments as moe_expert_forward.  The call needs
- *  moe_expert_workspace_size(L, n_tokens, top_k, QK_ACT_NONE) <= 4 MiB (hidden 4096,
- *  inter 2048: up to 42 pairs per launch for an all-MXFP4 layer on the
- *  block-scaled decode kernels, 28 for other layers); larger requests return
+ *  moe_expert_workspace_size(L, n_tokens, top_k, QK_ACT_NONE) <= 16 MiB (hidden
+ *  4096, inter 2048: up to 30 pairs per launch at top-6 (34 at top-2) for an
+ *  all-MXFP4 layer on the block-scaled decode kernels, 114 for other layers);
+ *  larger requests return
  *  QK_ERR_WORKSPACE and launch nothing.  Nothing in the array has to start at
  *  zero.  The array is shared by every call on a device: calls that overlap on
  *  the GPU (other streams, other host threads) race on it and must not be
- *  issued.  The first call on each device resolves the array's address
- *  (a host-side runtime query); make that first call before beginning any
- *  stream capture on that device.
+ *  issued.  Every call looks up the array's address in the current context
+ *  (a host-side runtime query, no device work); the first call in a context
+ *  may also load the library's device code, so make it before beginning any
+ *  stream capture in that context.
  * Errors: as moe_expert_forward; QK_ERR_WORKSPACE when the fixed array is too
  * small.
  * ---------------------------------------------------------------------- */

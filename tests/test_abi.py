@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(7):
+    for code in range(8):
         assert qk.status_string(code) not in ("", "unknown status")
     assert qk.status_string(99) == "unknown status"
 
@@ -60,19 +60,22 @@ def test_workspace_query_and_shape_validation():
 
 
 def test_workspace_query_follows_the_path_choice():
-    """All-MXFP4 layers with 32-byte aligned weights take the block-scaled
-    decode and grouped paths (their own workspace layouts); the same layer
-    with misaligned weights, or in NVFP4, takes the f16 paths, whose
-    workspace depends on the shapes only."""
+    """All-MXFP4 layers take the block-scaled decode kernels (16-byte aligned
+    weights suffice: one TMA box per step) and, with 32-byte aligned weights,
+    the block-scaled grouped GEMMs (their own workspace layouts); NVFP4 layers
+    take the f16 paths, whose workspace depends on the shapes only."""
     L = qk.load()
     mx = _fake_layer()
     nv = _fake_layer(fmts=(2, 2, 2))
     mis = _fake_layer()
-    mis.gate.q = mis.gate.q + 16  # 16-byte aligned, not 32: no block-scaled path
-    for T in (1, 16, 100):         # decode (<= 21 tokens at top-6) and grouped
+    mis.gate.q = mis.gate.q + 16  # 16-byte aligned, not 32
+    for T in (1, 16):              # decode (<= 21 tokens at top-6)
         a, b, c = (L.moe_expert_workspace_size(ctypes.byref(x), T, 6, 0) for x in (mx, nv, mis))
         assert a > 0 and b > 0
-        assert c == b and a != b, (T, a, b, c)
+        assert c == a and a != b, (T, a, b, c)
+    a, b, c = (L.moe_expert_workspace_size(ctypes.byref(x), 100, 6, 0) for x in (mx, nv, mis))
+    assert a > 0 and b > 0
+    assert c == b and a != b, (100, a, b, c)  # grouped: no block-scaled GEMMs when misaligned
 
 
 def test_workspace_query_with_activation_modes():
@@ -92,16 +95,18 @@ def test_workspace_query_with_activation_modes():
 
 
 def test_noalloc_limit_in_pairs():
-    """4 MiB of fixed scratch: at hidden 4096, inter 2048 the block-scaled
-    MXFP4 decode needs 96 KiB per pair (42 pairs fit), the f16 decode more
-    (28 pairs)."""
+    """16 MiB of fixed scratch: at hidden 4096, inter 2048 the block-scaled
+    MXFP4 decode needs about 456 KiB per pair (per-step gate/up and down
+    results, h images): 30 pairs fit at top-6, 34 at top-2; the f16 decode
+    for NVFP4 layers needs less (114 / 118 pairs)."""
     L = qk.load()
     mx, nv = _fake_layer(), _fake_layer(fmts=(2, 2, 2))
-    cap = 4 << 20
+    cap = 16 << 20
     q = lambda lay, T, k: L.moe_expert_workspace_size(ctypes.byref(lay), T, k, 0)
-    assert q(mx, 7, 6) <= cap < q(mx, 8, 6)        # 42 pairs fit, 48 do not
-    assert q(mx, 21, 2) <= cap < q(mx, 22, 2)      # 42 / 44
-    assert q(nv, 14, 2) <= cap < q(nv, 15, 2)      # 28 / 30
+    assert q(mx, 5, 6) <= cap < q(mx, 6, 6)        # 30 pairs fit, 36 do not
+    assert q(mx, 17, 2) <= cap < q(mx, 18, 2)      # 34 / 36
+    assert q(nv, 19, 6) <= cap < q(nv, 20, 6)      # 114 / 120
+    assert q(nv, 59, 2) <= cap < q(nv, 60, 2)      # 118 / 120
 
 
 def test_forward_argument_errors_are_synchronous():
@@ -145,7 +150,7 @@ def test_noalloc_entry_rejects_before_any_device_work():
     p = ctypes.c_void_p(1 << 24)
     f = L.moe_expert_forward_noalloc
     assert f(ctypes.byref(lay), p, 0, p, p, 6, p, 0, None) == qk.QK_OK                # T = 0
-    assert f(ctypes.byref(lay), p, 16, p, p, 6, p, 0, None) == qk.QK_ERR_WORKSPACE    # > 4 MiB
+    assert f(ctypes.byref(lay), p, 16, p, p, 6, p, 0, None) == qk.QK_ERR_WORKSPACE    # > 16 MiB
     assert f(ctypes.byref(lay), p, 1, p, p, 9, p, 0, None) == qk.QK_ERR_INVALID_ARG   # top_k > 8
     assert f(None, p, 1, p, p, 6, p, 0, None) == qk.QK_ERR_INVALID_ARG
 

@@ -84,8 +84,7 @@ def test_kernel_hash_ignores_comments_only():
     from block_quantized_expert_mxfp4_b200 import build as b
 
     assert bench._code_only("int a; // note\n/* block\n comment */ int b;\n\n") == "int a;\n int b;"
-    names = ("qk_dmx.cu", "qk_route_table.cuh", "qk_device.cuh", "qk_common.cuh", "qk_group.cuh",
-             "qk_internal.h", "qk_tmap.h")
+    names = bench.DECODE_KERNEL_FILES
     for n in names:
         for lit in re.findall(r'"(?:[^"\\\n]|\\.)*"', open(os.path.join(b.CSRC, n)).read()):
             assert "//" not in lit and "/*" not in lit, (n, lit)
@@ -99,7 +98,7 @@ def test_kernel_hash_ignores_comments_only():
     try:
         b.CSRC = tmp
         assert bench.kernel_source_hash() == h0
-        p = os.path.join(tmp, "qk_dmx.cu")
+        p = os.path.join(tmp, names[0])
         src = open(p).read()
         open(p, "w").write(src.replace("namespace qk {", "namespace qk {\n// a comment added\n", 1))
         assert bench.kernel_source_hash() == h0

@@ -11,6 +11,10 @@ from helpers import assert_parity, oracle_moe
 pytestmark = pytest.mark.gpu
 
 WL = synth.Workload("small", 8, 2, 256, 256, 4, 118, 127)
+# hidden 2048, inter 1024: multiples of 1024, so MXFP4 layers take the
+# block-scaled kernels (decode up to floor(128 / top_k) = 32 tokens, grouped
+# GEMMs above)
+BS = synth.Workload("bs_status", 16, 4, 2048, 1024, 4, 118, 127)
 
 
 def _setup(seed=0):
@@ -74,19 +78,73 @@ def test_out_of_range_id_reported_and_skipped():
     assert_parity(y.cpu().numpy(), yo, what="skipped pairs")
 
 
-def test_timeout_path_reports_and_context_survives():
-    layer, x = _setup(2)
-    ids = torch.tensor([[0, 1]] * 4, dtype=torch.int32, device="cuda")
-    w = torch.full((4, 2), 0.5, device="cuda")
+def _fwd_wl(wl, layer, x, ids, w):
+    lay = layer.c()
+    y = torch.zeros((x.shape[0], wl.H), device="cuda")
+    ws = torch.empty(qk.moe_expert_workspace_size(lay, x.shape[0], ids.shape[1]),
+                     dtype=torch.uint8, device="cuda")
+    qk.moe_expert_forward(lay, x.cuda(), ids, w, y, ws)
+    return y
+
+
+def _timeout_then_parity(wl, layer, seed, x, ids_np, w_np, what):
+    """Three calls with the wait limit at 0 (the first wait not already
+    complete runs out: weight copies take about a microsecond to land, so at
+    least one does), then a call at the default limit checked against the
+    oracle: the kernels stop cleanly and the context stays usable."""
+    ids = torch.from_numpy(ids_np).cuda()
+    w = torch.from_numpy(w_np).float().cuda()
+    seen = []
     try:
         qk.qk_debug_set_wait_limit_ns(0)
         for _ in range(3):
-            _fwd(layer, x, ids, w)
-        st = qk.qk_last_device_status()
+            _fwd_wl(wl, layer, x, ids, w)
+            seen.append(qk.qk_last_device_status())
     finally:
         qk.qk_debug_set_wait_limit_ns(1_000_000_000)
-    assert st in (qk.QK_ERR_TIMEOUT, qk.QK_OK)  # a copy may land before the first poll
-    y = _fwd(layer, x, ids, w)
+    assert qk.QK_ERR_TIMEOUT in seen, seen
+    assert all(s in (qk.QK_ERR_TIMEOUT, qk.QK_OK) for s in seen), seen
+    y = _fwd_wl(wl, layer, x, ids, w)
     assert qk.qk_last_device_status() == qk.QK_OK
-    yo = oracle_moe(WL, 2, 0, x, np.array([[0, 1]] * 4, np.int32), np.full((4, 2), 0.5))
-    assert_parity(y.cpu().numpy(), yo, what="after timeout")
+    yo = oracle_moe(wl, seed, 0, x, ids_np, w_np)
+    assert_parity(y.cpu().numpy(), yo, what=what)
+
+
+def test_timeout_path_reports_and_context_survives():
+    """The f16 decode kernels (hidden 256 is below the block-scaled shapes)."""
+    layer, x = _setup(2)
+    _timeout_then_parity(WL, layer, 2, x, np.array([[0, 1]] * 4, np.int32), np.full((4, 2), 0.5),
+                         "f16 decode after timeout")
+
+
+def _bs_routing(T, seed):
+    """Slot 0 of every token is expert 3; the other slots are distinct random
+    experts."""
+    rng = np.random.default_rng(seed)
+    others = [e for e in range(BS.E) if e != 3]
+    ids = np.array([[3] + list(rng.choice(others, size=BS.k - 1, replace=False)) for _ in range(T)],
+                   dtype=np.int32)
+    w = np.full((T, BS.k), 1.0 / BS.k)
+    return ids, w
+
+
+@pytest.mark.parametrize("T", [2, 40])
+def test_timeout_block_scaled(T):
+    """Block-scaled MXFP4 kernels: T = 2 runs the decode kernels, T = 40 (160
+    pairs) the grouped GEMMs; every wait there is bounded and reports."""
+    layer = workload.make_layer(BS, 6, 0)
+    x = synth.activations(6, T, BS.H)
+    ids, w = _bs_routing(T, 6 + T)
+    _timeout_then_parity(BS, layer, 6, x, ids, w, f"block-scaled T={T} after timeout")
+
+
+@pytest.mark.parametrize("T", [2, 40])
+def test_nan_scale_reported_block_scaled(T):
+    """e8m0 code 255 in expert 3's up projection, block-scaled decode (T = 2)
+    and grouped (T = 40) kernels."""
+    layer = workload.make_layer(BS, 7, 0)
+    layer.up.scales[3, 7, 2] = 255
+    x = synth.activations(7, T, BS.H)
+    ids, w = _bs_routing(T, 7 + T)
+    _fwd_wl(BS, layer, x, torch.from_numpy(ids).cuda(), torch.from_numpy(w).float().cuda())
+    assert qk.qk_last_device_status() == qk.QK_ERR_NAN_SCALE
