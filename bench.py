@@ -145,8 +145,8 @@ def _code_only(text: str) -> str:
 
 
 # The decode kernels' code: the kernel file first, then the headers it includes.
-DECODE_KERNEL_FILES = ("qk_dq.cu", "qk_route_table.cuh", "qk_device.cuh", "qk_common.cuh", "qk_internal.h",
-                       "qk_tmap.h")
+DECODE_KERNEL_FILES = ("qk_dmx.cu", "qk_group.cuh", "qk_route_table.cuh", "qk_device.cuh", "qk_common.cuh",
+                       "qk_internal.h", "qk_tmap.h")
 
 
 def kernel_source_hash() -> str:
@@ -354,15 +354,14 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(elapsed_max / K * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e2m1 x e8m0 weights, activations as 8 e2m1 terms x ue8m0 (kind::mxf4 block-scaled MMA), "
-                 "f32 accumulate",
+        "dtype": "e2m1 x e8m0 weights, activations as e4m3 terms x ue8m0 (block-scaled MMA), f32 accumulate",
         "data": "synthetic (seeded; random-init MXFP4 weights of the DeepSeek-V4-Flash expert shape)",
         "config": {"workload": WORKLOAD_DESC, "layers_resident": L,
                    "resident_weight_GB": round(L * wl.E * expert_bytes / 1e9, 2),
                    "bytes_per_step": bytes_per_step,
                    "l2": "inputs larger than L2: steps rotate over the resident layers",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "moe_expert_forward (k_dq gate/up -> k_dq down, kind::mxf4 tcgen05, PDL-chained)",
+        "roofline": {"kernel": "moe_expert_forward (k_dmx gate/up -> k_dmx down, block-scaled tcgen05, PDL-chained)",
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "ffn_us": round(ffn_s * 1e6, 3), "ffn_calls_timed": len(ffn_ms),

@@ -93,8 +93,8 @@ size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_
     return act_quant_ok(L, act_quant) ? group_workspace_bytes(L, n_tokens, top_k) : 0;
   if (n_tokens > decode_chunk(top_k))
     return group_workspace_bytes(L, n_tokens, top_k);
-  if (dq_eligible(L->gate, L->up, L->down, L->hidden, L->inter))
-    return dq_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
+  if (dmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter))
+    return dmx_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
   return decode_workspace_bytes(n_tokens, top_k, L->hidden, L->inter);
 }
 
@@ -134,8 +134,8 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
     return group_forward_act(a, act_quant, workspace, reinterpret_cast<cudaStream_t>(stream));
   if (n_tokens > decode_chunk(top_k)) return group_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
   // All-MXFP4 layers: weights straight to the fp4 block-scaled tensor cores.
-  if (dq_eligible(a.gate, a.up, a.down, a.H, a.I))
-    return dq_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
+  if (dmx_eligible(a.gate, a.up, a.down, a.H, a.I))
+    return dmx_forward(a, workspace, reinterpret_cast<cudaStream_t>(stream));
   decode_carve(a, workspace);
   return decode_forward(a, reinterpret_cast<cudaStream_t>(stream));
 }

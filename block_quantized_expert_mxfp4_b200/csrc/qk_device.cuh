@@ -18,14 +18,19 @@
 namespace qk {
 
 // ---------------------------------------------------------------- status --
-// First device-side error wins; read and cleared by qk_last_device_status().
+// First device-side error wins (except that any other error replaces
+// QK_ERR_NONFINITE, which is usually its consequence: a NaN scale code makes
+// NaN products); read and cleared by qk_last_device_status().
 extern __device__ int g_status;
 // Limit of every bounded wait, in ns (qk_debug_set_wait_limit_ns).
 extern __device__ unsigned long long g_wait_limit_ns;
 // Limit used when draining copies after a wait ran out (never 0).
 constexpr unsigned long long kDrainLimitNs = 1000000000ull;
 
-__device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
+__device__ __forceinline__ void set_status(int code) {
+  const int old = atomicCAS(&g_status, 0, code);
+  if (old == QK_ERR_NONFINITE && code != QK_ERR_NONFINITE) atomicCAS(&g_status, QK_ERR_NONFINITE, code);
+}
 
 __device__ __forceinline__ unsigned long long globaltimer() {
   unsigned long long t;
@@ -67,13 +72,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Phase `parity` of `bar` complete now (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes or about `ns` nanoseconds have passed.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for phase `parity` of `bar` for at most `limit_ns`; false if it ran out.
+// A limit of 0 takes one non-suspending look.  Otherwise the thread sleeps in
+// hardware between looks (a suspend hint of 1 us, woken by the phase
+// completing) and reads the timer once per look: waiting warps that poll in
+// software take the issue slots and the barrier unit away from the few busy
+// threads (the one issuing copies or tensor-core instructions), which slows
+// those down severalfold.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   unsigned long long limit_ns) {
+  if (limit_ns == 0) return mbar_test_wait(bar, parity);
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
     if (globaltimer() - t0 >= limit_ns) return false;
   }
 }
@@ -146,6 +183,11 @@ __device__ __forceinline__ void tmap_prefetch(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

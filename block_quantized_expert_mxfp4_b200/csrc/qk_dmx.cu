@@ -76,6 +76,7 @@ struct DmxHead {
   alignas(8) uint64_t acc_full[2];   // [0]: the accumulator holds a finished unit
   alignas(8) uint64_t acc_empty[2];  // [0]: the epilogue has read it ([1] unused)
   alignas(8) uint64_t drained;
+  alignas(8) uint64_t epi_done;      // the epilogue warp has left its loop (TMEM reads done)
   uint32_t tmem;
   int abort;
 };
@@ -140,6 +141,10 @@ __device__ __forceinline__ void build_x(const DmxArgs& G, const Route& R, int v,
       v8[2 * i] = bf16_bits_to_f32(wd[i] & 0xFFFFu);
       v8[2 * i + 1] = bf16_bits_to_f32(wd[i] >> 16);
     }
+    bool fin = true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) fin &= finite_bits(v8[i]);
+    if (!fin) set_status(QK_ERR_NONFINITE);  // an inf or NaN in x
     const int s = b >> 2, kb = b & 3;
     uint32_t q[2];
 #pragma unroll
@@ -182,6 +187,10 @@ __device__ __forceinline__ void build_h(const DmxArgs& G, const Route& R, int v,
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) g[i] = __fdividef(g[i], 1.0f + __expf(-g[i])) * u[i];
+    bool fin = true;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) fin &= finite_bits(g[i]);
+    if (!fin) set_status(QK_ERR_NONFINITE);  // h beyond fp32 (or from non-finite inputs)
     const int s = b >> 2, kb = b & 3;
     uint32_t q[2];
 #pragma unroll
@@ -229,6 +238,7 @@ __global__ void __launch_bounds__(kDThreads, 2) k_dmx(const __grid_constant__ Dm
       mbar_init(&S.acc_empty[s], 1);
     }
     mbar_init(&S.drained, 1);
+    mbar_init(&S.epi_done, 1);
     S.abort = 0;
     fence_mbar_init();
   }
@@ -470,6 +480,8 @@ __global__ void __launch_bounds__(kDThreads, 2) k_dmx(const __grid_constant__ Dm
 #pragma unroll
               for (int q = 0; q < 4; ++q) acc[q] = fmaf(wt, d[q], acc[q]);
             }
+            if (!(finite_bits(acc[0]) && finite_bits(acc[1]) && finite_bits(acc[2]) && finite_bits(acc[3])))
+              set_status(QK_ERR_NONFINITE);
             const size_t o = (size_t)t * G.H + nb * kDN + lane * 4;
             if (G.y_bf16) {
               __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(G.y) + o;
@@ -483,8 +495,15 @@ __global__ void __launch_bounds__(kDThreads, 2) k_dmx(const __grid_constant__ Dm
       }
     }
   }
+  if (warp == 4) {  // the epilogue's TMEM reads are done (also on an early exit)
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_one(&S.epi_done);
+  }
   __syncthreads();
   if (warp == 1) {
+    // (a CTA barrier after long single-lane loops is not relied on alone)
+    mbar_wait_bounded(&S.epi_done, 0, kDrainLimitNs);
     tc_fence_after();
     tmem_free(tmem, kDTmemCols);
   }

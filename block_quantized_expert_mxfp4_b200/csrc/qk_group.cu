@@ -296,12 +296,6 @@ __host__ __device__ inline int g_smem_bytes(int sc_stride) {
   return 1024 + kGAS * kGStageA + kGBS * kGStageB + kGRS * kGStageR + kGM * sc_stride + (int)sizeof(GHead);
 }
 
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
 __device__ __forceinline__ int box_index(int n) { return n <= 32 ? 0 : n <= 64 ? 1 : n <= 128 ? 2 : 3; }
 
 // f16x2 broadcast of 2^e (0 below the smallest f16 subnormal).

@@ -45,10 +45,6 @@ qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
 bool dmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
 size_t dmx_workspace_bytes(int T, int k, int H, int I);
 qk_status dmx_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
-// Decode path on the fp4 x fp4 block-scaled tensor cores (kind::mxf4).
-bool dq_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
-size_t dq_workspace_bytes(int T, int k, int H, int I);
-qk_status dq_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
 size_t decode_workspace_bytes(int T, int k, int H, int I);
 void decode_carve(DecodeArgs& a, void* ws);
 

@@ -109,9 +109,14 @@ typedef struct qk_moe_layer {
  *  topk_w    [T][top_k] fp32.         y        [T][hidden] fp32 (y_is_bf16=0) or bf16.
  *  act_quant QK_ACT_* (above).        workspace >= moe_expert_workspace_size(), 256-B aligned.
  * Shapes: hidden and inter multiples of 128; 1 <= top_k <= 8.  Up to
- * floor(128/top_k) tokens run the decode kernels (nibbles and scales decoded
- * in registers, tensor-core m16n8k16 products, fp32 accumulation).  More
- * tokens run the grouped path ([REAP25] "What's actually different": one
+ * floor(128/top_k) tokens run the decode kernels: for all-MXFP4 layers with
+ * hidden and inter multiples of 1024 and 32-byte aligned weights, the
+ * block-scaled tensor cores (tcgen05 kind::mxf8f6f4 block_scale) with the
+ * e2m1 weights and e8m0 scales as stored and the activations as e4m3 terms
+ * with e8m0 scales per 32 (bf16 x as two terms, exact; h as three, relative
+ * error below 2^-12); for other layers nibbles and scales decoded in
+ * registers and tensor-core m16n8k16 f16 products; fp32 accumulation in
+ * both.  More tokens run the grouped path ([REAP25] "What's actually different": one
  * grouped GEMM per projection): the pairs are sorted by expert and each
  * projection is a grouped tcgen05 GEMM -- on the block-scaled tensor cores
  * with the e2m1 weights and e8m0 scales as stored and the activations as
@@ -124,7 +129,10 @@ typedef struct qk_moe_layer {
  * a layer the block-scaled kernels do not take), QK_ERR_CUDA; device:
  * QK_ERR_NAN_SCALE,
  * QK_ERR_INVALID_ARG (id out of range: that pair contributes nothing),
- * QK_ERR_TIMEOUT.
+ * QK_ERR_TIMEOUT, QK_ERR_NONFINITE (an inf or NaN in x, or a gate/up/h/y
+ * value that overflowed fp32: the kernels accumulate in fp32, so products of
+ * scale codes near 254 with ordinary activations exceed its range where the
+ * exact result does not).
  * moe_expert_workspace_size returns the workspace bytes of the path the same
  * (layer, n_tokens, top_k, act_quant) call takes, or 0 for arguments the call
  * would reject (including a quantized act_quant the layer does not take).
@@ -145,8 +153,9 @@ qk_status moe_expert_forward(const qk_moe_layer* L, const void* x_bf16, int32_t 
  * embedded in a runtime that owns every device allocation).
  *  Arguments as moe_expert_forward.  The call needs
  *  moe_expert_workspace_size(L, n_tokens, top_k, QK_ACT_NONE) <= 16 MiB (hidden
- *  4096, inter 2048: up to 30 pairs per launch at top-6 (34 at top-2) for an
- *  all-MXFP4 layer on the block-scaled decode kernels, 114 for other layers);
+ *  4096, inter 2048: every launch of an all-MXFP4 layer on the block-scaled
+ *  decode kernels (up to 128 pairs) fits; other layers up to 114 pairs at
+ *  top-6, 118 at top-2; the grouped kernels above 128 pairs do not fit);
  *  larger requests return
  *  QK_ERR_WORKSPACE and launch nothing.  Nothing in the array has to start at
  *  zero.  The array is shared by every call on a device: calls that overlap on

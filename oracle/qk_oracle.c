@@ -171,10 +171,6 @@ int qko_convert_mx_to_nv(const uint8_t* e8m0, int32_t E, int32_t N, int32_t K,
   return QKO_OK;
 }
 
-/* -------------------------------------------------------------- router --
- * Softmax over the E logits in fp64, the k largest probabilities (equal
- * probabilities: lower expert id first), renormalised to sum to 1, slots in
- * that order.  (The pages name 256 experts and top-6 but not the function.) */
 /* NVFP4 -> MXFP4, scales only (the reverse of the conversion above; the pages
  * define only the forward direction, so the rule is the reading adopted).  A
  * 32-block's two half scales e4m3(s0) * scale_2 and e4m3(s1) * scale_2 (exact
@@ -182,8 +178,10 @@ int qko_convert_mx_to_nv(const uint8_t* e8m0, int32_t E, int32_t N, int32_t K,
  * -127 <= p <= 127: code p + 127.  Any other block is counted once in
  * n_inexact and gets the code whose power of two is nearest in log2 to the
  * larger magnitude of the two (2^p for a mantissa below sqrt 2, else 2^(p+1);
- * clamped to codes 0 .. 254; code 0 for two zero scales).  A NaN code or a
- * non-finite product is QKO_ERR_NAN_SCALE. */
+ * clamped to codes 0 .. 254; code 0 for two zero scales: e8m0 has no zero, so
+ * such a block's nonzero nibbles turn into values of 2^-127 scale and the block
+ * counts as inexact).  A NaN code or a non-finite product is
+ * QKO_ERR_NAN_SCALE. */
 int qko_convert_nv_to_mx(const uint8_t* e4m3, const float* scale_2, int32_t E, int32_t N, int32_t K,
                          uint8_t* e8m0, uint64_t* n_inexact) {
   int64_t e, i, per;
@@ -221,6 +219,10 @@ int qko_convert_nv_to_mx(const uint8_t* e4m3, const float* scale_2, int32_t E, i
   return QKO_OK;
 }
 
+/* -------------------------------------------------------------- router --
+ * Softmax over the E logits in fp64, the k largest probabilities (equal
+ * probabilities: lower expert id first), renormalised to sum to 1, slots in
+ * that order.  (The pages name 256 experts and top-6 but not the function.) */
 int qko_route_topk(const float* logits, int32_t T, int32_t E, int32_t k,
                    int32_t* ids, double* w) {
   int32_t t, i, s;

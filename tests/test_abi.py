@@ -60,22 +60,19 @@ def test_workspace_query_and_shape_validation():
 
 
 def test_workspace_query_follows_the_path_choice():
-    """All-MXFP4 layers take the block-scaled decode kernels (16-byte aligned
-    weights suffice: one TMA box per step) and, with 32-byte aligned weights,
-    the block-scaled grouped GEMMs (their own workspace layouts); NVFP4 layers
-    take the f16 paths, whose workspace depends on the shapes only."""
+    """All-MXFP4 layers with 32-byte aligned weights take the block-scaled
+    decode and grouped paths (their own workspace layouts); the same layer
+    with misaligned weights, or in NVFP4, takes the f16 paths, whose
+    workspace depends on the shapes only."""
     L = qk.load()
     mx = _fake_layer()
     nv = _fake_layer(fmts=(2, 2, 2))
     mis = _fake_layer()
-    mis.gate.q = mis.gate.q + 16  # 16-byte aligned, not 32
-    for T in (1, 16):              # decode (<= 21 tokens at top-6)
+    mis.gate.q = mis.gate.q + 16  # 16-byte aligned, not 32: no block-scaled path
+    for T in (1, 16, 100):         # decode (<= 21 tokens at top-6) and grouped
         a, b, c = (L.moe_expert_workspace_size(ctypes.byref(x), T, 6, 0) for x in (mx, nv, mis))
         assert a > 0 and b > 0
-        assert c == a and a != b, (T, a, b, c)
-    a, b, c = (L.moe_expert_workspace_size(ctypes.byref(x), 100, 6, 0) for x in (mx, nv, mis))
-    assert a > 0 and b > 0
-    assert c == b and a != b, (100, a, b, c)  # grouped: no block-scaled GEMMs when misaligned
+        assert c == b and a != b, (T, a, b, c)
 
 
 def test_workspace_query_with_activation_modes():
@@ -96,15 +93,15 @@ def test_workspace_query_with_activation_modes():
 
 def test_noalloc_limit_in_pairs():
     """16 MiB of fixed scratch: at hidden 4096, inter 2048 the block-scaled
-    MXFP4 decode needs about 456 KiB per pair (per-step gate/up and down
-    results, h images): 30 pairs fit at top-6, 34 at top-2; the f16 decode
-    for NVFP4 layers needs less (114 / 118 pairs)."""
+    MXFP4 decode needs about 96 KiB per pair, so every decode launch (up to
+    128 pairs) fits, while the grouped kernels above 128 pairs do not; the
+    f16 decode for NVFP4 layers fits 114 pairs at top-6 and 118 at top-2."""
     L = qk.load()
     mx, nv = _fake_layer(), _fake_layer(fmts=(2, 2, 2))
     cap = 16 << 20
     q = lambda lay, T, k: L.moe_expert_workspace_size(ctypes.byref(lay), T, k, 0)
-    assert q(mx, 5, 6) <= cap < q(mx, 6, 6)        # 30 pairs fit, 36 do not
-    assert q(mx, 17, 2) <= cap < q(mx, 18, 2)      # 34 / 36
+    assert q(mx, 21, 6) <= cap < q(mx, 22, 6)      # 126 pairs (decode) fit, 132 (grouped) do not
+    assert q(mx, 64, 2) <= cap < q(mx, 65, 2)      # 128 / 130
     assert q(nv, 19, 6) <= cap < q(nv, 20, 6)      # 114 / 120
     assert q(nv, 59, 2) <= cap < q(nv, 60, 2)      # 118 / 120
 
@@ -150,7 +147,7 @@ def test_noalloc_entry_rejects_before_any_device_work():
     p = ctypes.c_void_p(1 << 24)
     f = L.moe_expert_forward_noalloc
     assert f(ctypes.byref(lay), p, 0, p, p, 6, p, 0, None) == qk.QK_OK                # T = 0
-    assert f(ctypes.byref(lay), p, 16, p, p, 6, p, 0, None) == qk.QK_ERR_WORKSPACE    # > 16 MiB
+    assert f(ctypes.byref(lay), p, 22, p, p, 6, p, 0, None) == qk.QK_ERR_WORKSPACE    # > 16 MiB (grouped)
     assert f(ctypes.byref(lay), p, 1, p, p, 9, p, 0, None) == qk.QK_ERR_INVALID_ARG   # top_k > 8
     assert f(None, p, 1, p, p, 6, p, 0, None) == qk.QK_ERR_INVALID_ARG
 

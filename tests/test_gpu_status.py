@@ -87,7 +87,7 @@ def _fwd_wl(wl, layer, x, ids, w):
     return y
 
 
-def _timeout_then_parity(wl, layer, seed, x, ids_np, w_np, what):
+def _timeout_then_parity(wl, layer, seed, x, ids_np, w_np, what, fmts=(1, 1, 1)):
     """Three calls with the wait limit at 0 (the first wait not already
     complete runs out: weight copies take about a microsecond to land, so at
     least one does), then a call at the default limit checked against the
@@ -97,7 +97,9 @@ def _timeout_then_parity(wl, layer, seed, x, ids_np, w_np, what):
     seen = []
     try:
         qk.qk_debug_set_wait_limit_ns(0)
-        for _ in range(3):
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        for i in range(3):
+            flush.fill_(i)  # the weights leave L2: the first copies cannot have landed at the first poll
             _fwd_wl(wl, layer, x, ids, w)
             seen.append(qk.qk_last_device_status())
     finally:
@@ -106,15 +108,20 @@ def _timeout_then_parity(wl, layer, seed, x, ids_np, w_np, what):
     assert all(s in (qk.QK_ERR_TIMEOUT, qk.QK_OK) for s in seen), seen
     y = _fwd_wl(wl, layer, x, ids, w)
     assert qk.qk_last_device_status() == qk.QK_OK
-    yo = oracle_moe(wl, seed, 0, x, ids_np, w_np)
+    yo = oracle_moe(wl, seed, 0, x, ids_np, w_np, fmts)
     assert_parity(y.cpu().numpy(), yo, what=what)
 
 
 def test_timeout_path_reports_and_context_survives():
-    """The f16 decode kernels (hidden 256 is below the block-scaled shapes)."""
-    layer, x = _setup(2)
-    _timeout_then_parity(WL, layer, 2, x, np.array([[0, 1]] * 4, np.int32), np.full((4, 2), 0.5),
-                         "f16 decode after timeout")
+    """The f16 decode kernels: the full-size NVFP4 decode layer (256 experts,
+    hidden 4096, inter 2048; the block-scaled decode takes MXFP4 layers only)
+    at one token, its weights out of L2 before each call."""
+    wl = synth.WORKLOADS["decode_nv"]
+    layer = workload.make_layer(wl, 2, 0, (2, 2, 2))
+    x = synth.activations(2, 1, wl.H)
+    ids = np.array([[3, 17, 40, 99, 150, 201]], np.int32)
+    w = np.full((1, 6), 1.0 / 6)
+    _timeout_then_parity(wl, layer, 2, x, ids, w, "f16 decode after timeout", fmts=(2, 2, 2))
 
 
 def _bs_routing(T, seed):

@@ -39,8 +39,8 @@ def test_noalloc_matches_workspace_entry(name, T):
 
 def test_noalloc_rejects_requests_beyond_the_array():
     wl = synth.WORKLOADS["decode_mx"]
-    layer, x, ids, w = _inputs(wl, 16, 4)  # 96 pairs: ~13 MB of scratch
-    y = torch.empty((16, wl.H), dtype=torch.float32, device="cuda")
+    layer, x, ids, w = _inputs(wl, 22, 4)  # 132 pairs: the grouped kernels, ~200 MB of scratch
+    y = torch.empty((22, wl.H), dtype=torch.float32, device="cuda")
     with pytest.raises(qk.QkError) as e:
         qk.moe_expert_forward_noalloc(layer.c(), x, ids, w, y)
     assert e.value.code == qk.QK_ERR_WORKSPACE
