@@ -59,6 +59,10 @@ def parse():
                     help="profiling only: fewer prefill tokens (0: the workload's 2048)")
     ap.add_argument("--prefill-act", choices=["none", "e4m3", "mxfp4"], default="none",
                     help="activation mode of the prefill layer (default: bf16 activations)")
+    ap.add_argument("--extra", choices=["all", "none"], default="all",
+                    help="the other configurations' objects: NVFP4 decode at 1/4/16 tokens, the 43-layer "
+                         "stack, the 16,384-token prefill layer and the W4A8 prefill layer")
+    ap.add_argument("--stack-steps", type=int, default=5, help="timed passes over the 43-layer stack")
     return ap.parse_args()
 
 
@@ -372,18 +376,164 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 3 * K,
         "clocks": clocks.summary(),
     }
+    del layers, lays
+    torch.cuda.empty_cache()
     if args.prefill_steps > 0:
-        del layers, lays
-        torch.cuda.empty_cache()
         out["prefill"] = run_prefill(args, rank, world, dev)
         # count, two tile-list scans, x split, gate/up GEMM, h split, down GEMM, combine
-        out["gpu_launches"] += 8 * args.prefill_steps
+        out["gpu_launches"] += out["prefill"]["gpu_launches"]
+    if args.extra == "all":
+        # the other configurations, each timed in its own region (not part of `value`)
+        out["decode_nvfp4"] = run_decode_nv(args, rank, world, dev)
+        out["stack43"] = run_stack(args, rank, world, dev)
+        out["prefill_16k"] = run_prefill(args, rank, world, dev, tokens=16384, steps=3)
+        out["prefill_w4a8"] = run_prefill(args, rank, world, dev, act="e4m3", steps=10)
+        for key in ("decode_nvfp4", "stack43", "prefill_16k", "prefill_w4a8"):
+            out["gpu_launches"] += out[key]["gpu_launches"]
     return out
 
 
-def run_prefill(args, rank, world, dev):
+def _graph_time(fn, K, world, dev, reps_warm=3):
+    """Seconds per replay of a CUDA graph of fn() (CUDA events on its stream,
+    after warm-up replays; max over ranks)."""
+    import torch
+    import torch.distributed as dist
+    s = torch.cuda.Stream(device=dev)
+    fn(None)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            fn(s)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        for _ in range(reps_warm):
+            g.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0.record(s)
+        for _ in range(K):
+            g.replay()
+        e1.record(s)
+        torch.cuda.synchronize()
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / K, world, dev)
+    del g
+    return t
+
+
+def run_decode_nv(args, rank, world, dev):
+    """The decode MoE layer in NVFP4 (the MXFP4 layer converted scale-only:
+    e4m3 block scales per 16 and an fp32 scale_2 per expert) at 1, 4 and 16
+    tokens: the FFN call alone, rotating over 4 resident layers."""
+    import torch
+
+    import block_quantized_expert_mxfp4_b200 as qk
+    from block_quantized_expert_mxfp4_b200 import synth, workload
+
+    wl = synth.WORKLOADS["decode_nv"]
+    L = 4
+    layers = [workload.make_layer(wl, seed=rank, layer=l) for l in range(L)]
+    lays = [ly.c() for ly in layers]
+    peak, peak_kind = peaks()
+    res = {"workload": "decode MoE layer in NVFP4 (256 experts, top-6, hidden 4096, intermediate 2048; "
+                       "e2m1 + e4m3 per 16 + fp32 scale_2, from the seeded MXFP4 layer by the scale-only "
+                       "conversion), softmax top-6 router, bf16 N(0,1) activations",
+           "layers_resident": L, "peak_gbs": peak, "peak_kind": peak_kind, "by_tokens": {}}
+    launches = 0
+    for T in (1, 4, 16):
+        xs, ids_, ws_, nbytes = [], [], [], 0
+        for l in range(L):
+            x = synth.activations(rank * 131 + l, T, wl.H).to(dev)
+            lg = synth.router_logits(rank * 131 + l, T, wl.E).to(dev)
+            ids = torch.empty((T, wl.k), dtype=torch.int32, device=dev)
+            w = torch.empty((T, wl.k), dtype=torch.float32, device=dev)
+            qk.moe_route_topk(lg, wl.k, ids, w)
+            xs.append(x), ids_.append(ids), ws_.append(w)
+            nbytes += int(torch.unique(ids).numel()) * layers[l].expert_bytes()
+        y = torch.empty((T, wl.H), dtype=torch.float32, device=dev)
+        wsp = torch.empty(qk.moe_expert_workspace_size(lays[0], T, wl.k), dtype=torch.uint8, device=dev)
+        reps = 10
+
+        def step(st):
+            for _ in range(reps):
+                for l in range(L):
+                    qk.moe_expert_forward(lays[l], xs[l], ids_[l], ws_[l], y, wsp, stream=st)
+        t = _graph_time(step, 20, world, dev) / (reps * L)
+        if qk.qk_last_device_status() != qk.QK_OK:
+            raise RuntimeError("device status after the NVFP4 decode layer")
+        b = nbytes / L
+        res["by_tokens"][str(T)] = {"us_per_call": round(t * 1e6, 3), "bytes_per_call": int(b),
+                                    "achieved_gbs": round(b / t / 1e9, 1), "frac": round(b / t / 1e9 / peak, 4),
+                                    "tokens_per_s": round(T * world / t, 1)}
+        launches += 20 * reps * L * 2  # gate/up and down kernels (f16 decode path) per call
+    res["gpu_launches"] = launches
+    res["path"] = "f16 decode kernels (k_decode: e2m1 and e4m3 scales decoded in registers, m16n8k16 MMA)"
+    del layers, lays
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_stack(args, rank, world, dev):
+    """The pruned 43-layer expert stack at 8 tokens: per layer the router, the
+    routed experts (180 per layer, top-6, each projection's format drawn per
+    layer) and the FP8 block-128 shared expert added into the same output;
+    all 43 layers resident, one step = one pass over the stack."""
+    import torch
+
+    import block_quantized_expert_mxfp4_b200 as qk
+    from block_quantized_expert_mxfp4_b200 import synth, workload
+
+    wl = synth.WORKLOADS["stack43"]
+    fm = synth.format_choice(rank, wl.layers)
+    layers = [workload.make_layer(wl, rank, l, tuple(int(f) for f in fm[l])) for l in range(wl.layers)]
+    lays = [ly.c() for ly in layers]
+    shared = [workload.make_fp8_shared(rank, l, wl.H, wl.I, device=dev) for l in range(wl.layers)]
+    T, k = wl.T, wl.k
+    xs, lgs, ids_, ws_, ys = [], [], [], [], []
+    nbytes = 0
+    for l in range(wl.layers):
+        xs.append(synth.activations(rank, T, wl.H, stream=l).to(dev))
+        lgs.append(synth.router_logits(rank, T, wl.E, stream=l).to(dev))
+        ids_.append(torch.empty((T, k), dtype=torch.int32, device=dev))
+        ws_.append(torch.empty((T, k), dtype=torch.float32, device=dev))
+        ys.append(torch.empty((T, wl.H), dtype=torch.float32, device=dev))
+        qk.moe_route_topk(lgs[l], k, ids_[l], ws_[l])
+        nbytes += int(torch.unique(ids_[l]).numel()) * layers[l].expert_bytes() + shared[l].nbytes()
+    wsp = torch.empty(max(qk.moe_expert_workspace_size(ly, T, k) for ly in lays), dtype=torch.uint8, device=dev)
+    wss = torch.empty(qk.fp8_shared_expert_workspace_size(T, wl.H, wl.I), dtype=torch.uint8, device=dev)
+
+    def step(st):
+        for l in range(wl.layers):
+            qk.moe_route_topk(lgs[l], k, ids_[l], ws_[l], stream=st)
+            qk.moe_expert_forward(lays[l], xs[l], ids_[l], ws_[l], ys[l], wsp, stream=st)
+            sh = shared[l]
+            qk.fp8_shared_expert_forward(xs[l], sh.wg, sh.sg, sh.wu, sh.su, sh.wd, sh.sd, ys[l], wss, stream=st)
+    K = args.stack_steps
+    t = _graph_time(step, K, world, dev)
+    if qk.qk_last_device_status() != qk.QK_OK:
+        raise RuntimeError("device status after the stack")
+    peak, peak_kind = peaks()
+    mixed = [sum(int(f == 1) for f in fm[l]) for l in range(wl.layers)]
+    res = {"workload": f"pruned 43-layer expert stack: 180 experts per layer, top-6, hidden 4096, intermediate "
+                       f"2048, {T} tokens; per layer and projection a seeded MXFP4 or NVFP4 format "
+                       f"({sum(m == 3 for m in mixed)} layers all-MXFP4); FP8 E4M3 block-128 UE8M0 shared "
+                       "expert 4096x2048 SwiGLU per layer",
+           "ms_per_step": round(t * 1e3, 4), "tokens_per_s": round(T * world / t, 1), "steps": K,
+           "bytes_per_step": nbytes, "achieved_gbs": round(nbytes / t / 1e9, 1), "peak_gbs": peak,
+           "peak_kind": peak_kind, "frac": round(nbytes / t / 1e9 / peak, 4),
+           "hbm_floor_ms": round(nbytes / peak / 1e6, 4),
+           "gpu_launches": K * wl.layers * 5}  # router, routed gate/up and down, shared gate/up and down
+    del layers, lays, shared
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0):
     """The 2048-token Zipf prefill layer through moe_expert_forward (grouped
-    path): tokens/s, HBM fraction on the touched experts' bytes, tensor rate."""
+    path): tokens/s, HBM fraction on the touched experts' bytes, tensor rate.
+    `tokens`, `act` and `steps` override the command line's choices."""
     import torch
     import torch.distributed as dist
 
@@ -391,11 +541,12 @@ def run_prefill(args, rank, world, dev):
     from block_quantized_expert_mxfp4_b200 import synth, workload
 
     wl = synth.WORKLOADS["prefill"]
-    if args.prefill_experts or args.prefill_tokens:
+    if args.prefill_experts or args.prefill_tokens or tokens:
         import dataclasses
-        wl = dataclasses.replace(wl, E=args.prefill_experts or wl.E, T=args.prefill_tokens or wl.T)
+        wl = dataclasses.replace(wl, E=args.prefill_experts or wl.E, T=tokens or args.prefill_tokens or wl.T)
     T, k = wl.T, wl.k
-    aq = {"none": qk.QK_ACT_NONE, "e4m3": qk.QK_ACT_E4M3, "mxfp4": qk.QK_ACT_MXFP4}[args.prefill_act]
+    act_name = act or args.prefill_act
+    aq = {"none": qk.QK_ACT_NONE, "e4m3": qk.QK_ACT_E4M3, "mxfp4": qk.QK_ACT_MXFP4}[act_name]
     layer = workload.make_layer(wl, seed=rank, layer=0)
     lay = layer.c()
     x = synth.activations(rank, T, wl.H).to(dev)
@@ -419,7 +570,7 @@ def run_prefill(args, rank, world, dev):
         with torch.cuda.graph(g, stream=s):
             qk.moe_expert_forward(lay, x, ids, w, y, wsp, act_quant=aq, stream=s)
     torch.cuda.synchronize()
-    K = args.prefill_steps
+    K = steps or args.prefill_steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(s):
         for _ in range(3):
@@ -449,7 +600,7 @@ def run_prefill(args, rank, world, dev):
     return {
         "workload": f"prefill MoE layer: {T} tokens, {wl.E} experts, top-6 Zipf(s=1) routing, hidden 4096, "
                     "intermediate 2048, MXFP4 gate/up/down, bf16 N(0,1) activations"
-                    + ("" if aq == qk.QK_ACT_NONE else f", quantized in the layer to {args.prefill_act}"
+                    + ("" if aq == qk.QK_ACT_NONE else f", quantized in the layer to {act_name}"
                        " (one e8m0 scale per 32)"),
         "tokens_per_s": round(T * world / t, 1), "ms_per_layer": round(t * 1e3, 4), "steps": K,
         "experts_touched": touched,
@@ -461,8 +612,9 @@ def run_prefill(args, rank, world, dev):
         "path": ("counting sort by expert; x as 2 exact e4m3 terms; block-scaled tcgen05 grouped GEMMs "
                  "(e2m1 weights + e8m0 scales as stored): gate/up, SwiGLU + 3-term h split, down; combine")
         if aq == qk.QK_ACT_NONE else
-        (f"counting sort by expert; x and h quantized to {args.prefill_act} (one term, the other term slots "
+        (f"counting sort by expert; x and h quantized to {act_name} (one term, the other term slots "
          "zero); block-scaled tcgen05 grouped GEMMs; combine"),
+        "gpu_launches": 8 * K,
     }
 
 
