@@ -85,44 +85,65 @@ def test_stack_sampled_layers_with_shared_expert(layer_id):
     assert_parity(y_total, ro + so, what=what + " routed + shared")
 
 
+def _cover_tokens(oids, max_hot_bounds, seed):
+    """Tokens that reach every expert's first and last token tile: each
+    expert's first and last routed token (its pairs are grouped in token
+    order, so these open and close its tile list), the tile boundaries of the
+    hottest expert's list for both tile heights (40 and 64 tokens; evenly
+    spaced, at most max_hot_bounds of them), and 10 random tokens."""
+    T = oids.shape[0]
+    first, last = {}, {}
+    for t in range(T):
+        for e in oids[t]:
+            first.setdefault(int(e), t)
+            last[int(e)] = t
+    pick = set(first.values()) | set(last.values())
+    counts = np.bincount(oids.reshape(-1))
+    toks = np.nonzero((oids == int(np.argmax(counts))).any(1))[0]
+    bounds = set()
+    for tile in (40, 64):
+        for b in range(0, len(toks), tile):
+            bounds |= {int(toks[b]), int(toks[min(b + tile - 1, len(toks) - 1)])}
+    bounds = sorted(bounds)
+    if len(bounds) > max_hot_bounds:
+        bounds = [bounds[i] for i in np.linspace(0, len(bounds) - 1, max_hot_bounds).round().astype(int)]
+    pick |= set(bounds)
+    pick |= set(int(t) for t in np.random.default_rng(seed).choice(T, 10, replace=False))
+    return sorted(pick), len(first)
+
+
 def test_prefill_zipf_sampled_tokens():
-    """2048 tokens, Zipf-skewed routing over 256 experts; 12 sampled tokens
-    (including ones routed to the most and least loaded experts) against the
-    oracle."""
+    """2048 tokens, Zipf-skewed routing over 256 experts, the bench's layer
+    and routing: the tokens that open and close every expert's token tiles
+    (so every expert group, its first and its last tile, and the tile
+    boundaries of the hottest expert), about 380 of 2048, against the oracle."""
     wl = synth.WORKLOADS["prefill"]
     layer = workload.make_layer(wl, 0, 0)
     x = synth.activations(0, wl.T, wl.H)
     lg = synth.zipf_logits(0, wl.T, wl.E, wl.k)
     oids, ow = oracle.route_topk(lg, wl.k)
     y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
-    counts = np.bincount(oids.reshape(-1), minlength=wl.E)
-    hot, cold = int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
-    pick = {int(np.nonzero((oids == hot).any(1))[0][0]), int(np.nonzero((oids == cold).any(1))[0][0])}
-    rng = np.random.default_rng(7)
-    pick |= set(int(t) for t in rng.choice(wl.T, 10, replace=False))
-    pick = sorted(pick)
+    pick, n_exp = _cover_tokens(oids, 64, 7)
+    assert n_exp == wl.E
     yo = oracle_moe(wl, 0, 0, x[pick], oids[pick], ow[pick].astype(np.float32).astype(np.float64))
-    assert_parity(y.cpu().numpy()[pick], yo, what="prefill sampled tokens")
+    assert_parity(y.cpu().numpy()[pick], yo, what=f"prefill: {len(pick)} tokens covering every expert's tiles")
 
 
 def test_prefill_16k_tokens_sampled():
     """The same prefill layer at 16,384 tokens (Zipf s=1, top-6, 256 experts,
-    MXFP4: 98,304 pairs, past the size where the layer turns tensor-bound);
-    12 sampled tokens, including ones routed to the most and the least loaded
-    experts, against the oracle."""
+    MXFP4: 98,304 pairs, past the size where the layer turns tensor-bound):
+    every expert's first and last token and 32 tile boundaries spread over
+    the hottest expert's ~11,000 pairs, against the oracle."""
     wl = synth.WORKLOADS["prefill"]
     T = 16384
     layer = workload.make_layer(wl, 0, 0)
     x = synth.activations(40, T, wl.H)
     oids, ow = oracle.route_topk(synth.zipf_logits(40, T, wl.E, wl.k), wl.k)
     y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda())
-    counts = np.bincount(oids.reshape(-1), minlength=wl.E)
-    hot, cold = int(np.argmax(counts)), int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
-    pick = {int(np.nonzero((oids == hot).any(1))[0][0]), int(np.nonzero((oids == cold).any(1))[0][0])}
-    pick |= set(int(t) for t in np.random.default_rng(41).choice(T, 10, replace=False))
-    pick = sorted(pick)
+    pick, n_exp = _cover_tokens(oids, 32, 41)
+    assert n_exp == wl.E
     yo = oracle_moe(wl, 0, 0, x[pick], oids[pick], ow[pick].astype(np.float32).astype(np.float64))
-    assert_parity(y.cpu().numpy()[pick], yo, what="prefill 16k sampled tokens")
+    assert_parity(y.cpu().numpy()[pick], yo, what=f"prefill 16k: {len(pick)} tokens covering every expert")
 
 
 @pytest.mark.parametrize("fmts", [(NV, NV, NV), (MX, NV, NV), (NV, MX, MX)])

@@ -34,11 +34,20 @@ def _forward(layer, x, ids, w, aq):
 
 
 def _check(wl, seed, x, oids, ow, y, aq, what):
+    """Parity in the mode, and a bound on the h codes taken from the other
+    side of a decision boundary: an h value lies within the helper's relative
+    window (2^-13) of a midpoint for well under 1 % of the codes (e4m3 steps
+    are 2^-3 relative), so more than 0.5 % would mean a real difference, not
+    rounding."""
     experts = sorted(set(int(e) for e in oids.reshape(-1)))
     remap = {e: i for i, e in enumerate(experts)}
     L = oracle_sublayer(wl, seed, 0, experts)
     sub = np.vectorize(remap.get)(oids).astype(np.int32)
-    return assert_parity_act_quant(y, L, x, sub, ow.astype(np.float32).astype(np.float64), aq, what=what)
+    e, c, used, offered = assert_parity_act_quant(y, L, x, sub, ow.astype(np.float32).astype(np.float64), aq,
+                                                  what=what)
+    n_codes = oids.size * wl.I
+    assert used <= offered and used <= max(8, n_codes // 200), (what, used, offered, n_codes)
+    return e, c, used, offered
 
 
 @pytest.mark.parametrize("aq", MODES)
@@ -66,15 +75,26 @@ def test_grouped_sizes(aq):
 
 
 def test_w4a8_prefill_zipf_sampled_tokens():
-    """The 2048-token Zipf prefill layer in W4A8; 10 sampled tokens."""
+    """The 2048-token Zipf prefill layer in W4A8: the tokens that open and
+    close every expert's token tiles, and 10 random ones."""
     wl = synth.WORKLOADS["prefill"]
     layer = workload.make_layer(wl, 23, 0)
     x = synth.activations(23, wl.T, wl.H)
     oids, ow = oracle.route_topk(synth.zipf_logits(23, wl.T, wl.E, wl.k), wl.k)
     y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda(),
                  qk.QK_ACT_E4M3)
-    pick = sorted(int(t) for t in np.random.default_rng(24).choice(wl.T, 10, replace=False))
-    _check(wl, 23, x[pick], oids[pick], ow[pick], y[pick], qk.QK_ACT_E4M3, "w4a8 prefill sampled tokens")
+    # every expert's first and last token (the first and last tile of each
+    # expert group) and 10 random tokens
+    first, last = {}, {}
+    for t in range(wl.T):
+        for e in oids[t]:
+            first.setdefault(int(e), t)
+            last[int(e)] = t
+    pick = set(first.values()) | set(last.values())
+    pick |= set(int(t) for t in np.random.default_rng(24).choice(wl.T, 10, replace=False))
+    pick = sorted(pick)
+    _check(wl, 23, x[pick], oids[pick], ow[pick], y[pick], qk.QK_ACT_E4M3,
+           f"w4a8 prefill: {len(pick)} tokens covering every expert")
 
 
 @pytest.mark.parametrize("aq", MODES)
