@@ -388,7 +388,8 @@ def run_ours(args, rank, world, local_rank):
         out["stack43"] = run_stack(args, rank, world, dev)
         out["prefill_16k"] = run_prefill(args, rank, world, dev, tokens=16384, steps=3)
         out["prefill_w4a8"] = run_prefill(args, rank, world, dev, act="e4m3", steps=10)
-        for key in ("decode_nvfp4", "stack43", "prefill_16k", "prefill_w4a8"):
+        out["shared_fp8_prefill"] = run_shared_fp8(args, rank, world, dev)
+        for key in ("decode_nvfp4", "stack43", "prefill_16k", "prefill_w4a8", "shared_fp8_prefill"):
             out["gpu_launches"] += out[key]["gpu_launches"]
     return out
 
@@ -421,6 +422,53 @@ def _graph_time(fn, K, world, dev, reps_warm=3):
     t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / K, world, dev)
     del g
     return t
+
+
+def run_shared_fp8(args, rank, world, dev):
+    """The FP8 E4M3 block-128 shared expert (4096 x 2048 SwiGLU) at prefill
+    sizes (2048 and 16,384 rows), added into y: the block-scaled grouped
+    GEMMs; tensor rate on the useful FLOPs and HBM rate on its bytes."""
+    import torch
+
+    import block_quantized_expert_mxfp4_b200 as qk
+    from block_quantized_expert_mxfp4_b200 import synth, workload
+
+    H, I = 4096, 2048
+    sh = workload.make_fp8_shared(rank, 0, H, I, device=dev)
+    peak, peak_kind = peaks()
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16, src = float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        bf16, src = 1590.0, "fallback"
+    res = {"workload": "FP8 E4M3 shared expert, hidden 4096, intermediate 2048, UE8M0 per 128x128 tile, "
+                       "bf16 N(0,1) activations, result added into y",
+           "path": "one group of M tokens on the block-scaled grouped GEMMs: x as 2 exact e4m3 terms, "
+                   "e4m3 weights as stored (kind::mxf8f6f4), SwiGLU + 3-term h split, add into y",
+           "tensor_peak_tflops": 2 * bf16,
+           "tensor_peak_kind": f"{src} bf16 x 2 (nominal fp8/bf16 ratio): kind::mxf8f6f4",
+           "by_rows": {}}
+    launches = 0
+    for M in (2048, 16384):
+        x = synth.activations(rank + 7, M, H).to(dev)
+        y = torch.zeros((M, H), dtype=torch.float32, device=dev)
+        ws = torch.empty(qk.fp8_shared_expert_workspace_size(M, H, I), dtype=torch.uint8, device=dev)
+
+        def step(st):
+            qk.fp8_shared_expert_forward(x, sh.wg, sh.sg, sh.wu, sh.su, sh.wd, sh.sd, y, ws, stream=st)
+        K = 10
+        t = _graph_time(step, K, world, dev)
+        if qk.qk_last_device_status() != qk.QK_OK:
+            raise RuntimeError("device status after the shared expert")
+        flops = 2 * 3 * H * I * M
+        res["by_rows"][str(M)] = {"ms": round(t * 1e3, 4), "rows_per_s": round(M * world / t, 1),
+                                  "achieved_tflops": round(flops / t / 1e12, 1),
+                                  "tensor_frac": round(flops / t / 1e12 / (2 * bf16), 4),
+                                  "weight_bytes": sh.nbytes(), "hbm_frac": round(sh.nbytes() / t / 1e9 / peak, 4)}
+        launches += K * 9  # route fill, count, two scans, x split, gate/up, h split, down, combine
+        del x, y, ws
+    res["gpu_launches"] = launches
+    return res
 
 
 def run_decode_nv(args, rank, world, dev):

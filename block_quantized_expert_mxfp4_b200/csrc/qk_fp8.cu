@@ -281,8 +281,22 @@ qk_status fp8_linear_launch_blk(const void* x, int M, int K, const uint8_t* w, c
   return fp8_go<kLinear>(a, N / 16, 200 * 1024, st, false);
 }
 
+// From this many rows the shared expert runs on the block-scaled grouped
+// GEMMs (tcgen05, e4m3 weights as stored): there the weights are read once
+// per 64 (gate/up) or 40 (down) rows of tokens, while this file's kernel is
+// shaped for a handful of rows.
+constexpr int kFp8BigM = 128;
+
+static bool fp8_big_shape(int M, int H, int I) { return M >= kFp8BigM && H % 512 == 0 && I % 512 == 0; }
+
+static bool fp8_big_eligible(int M, int H, int I, const uint8_t* sg, const uint8_t* su, const uint8_t* sd) {
+  auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  return fp8_big_shape(M, H, I) && al(sg) && al(su) && al(sd);
+}
+
 size_t fp8_ffn_workspace_bytes(int M, int H, int I) {
-  return align256((size_t)M * I * 4) + align256((size_t)M * (I / 8) * 4);
+  const size_t small = align256((size_t)M * I * 4) + align256((size_t)M * (I / 8) * 4);
+  return fp8_big_shape(M, H, I) ? std::max(small, fp8_group_workspace_bytes(M, H, I)) : small;
 }
 
 qk_status fp8_ffn_launch(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
@@ -294,6 +308,8 @@ qk_status fp8_ffn_launch(const void* x, int M, int H, int I, const uint8_t* wg, 
 qk_status fp8_ffn_launch_blk(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
                              const uint8_t* wu, const uint8_t* su, const uint8_t* wd, const uint8_t* sd,
                              float* y, void* ws, int blk, cudaStream_t st) {
+  if (fp8_big_eligible(M, H, I, sg, su, sd))
+    return fp8_group_forward(x, M, H, I, wg, sg, wu, su, wd, sd, blk, y, ws, st);
   float* h = static_cast<float*>(ws);
   float* hmax = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256((size_t)M * I * 4));
   Fp8Args a = {};

@@ -220,7 +220,9 @@ struct GmxArgs {
   const uint8_t* sf_b;   // e8m0 scales of the up rows (gate/up phase)
   float* out;            // gate/up: gu [P][2 I]; down: dperm [P][H]
   int K, rows_per_e, MB, MBA, out_ld;  // MBA: weight blocks taken from ta / sf_a (the rest: tb / sf_b)
-  alignas(64) CUtensorMap ta, tb;  // packed weights, 16 x 4-bit -> 16-byte slots, box {128, 256}, 128B swizzle
+  int wfp8;              // 0: MXFP4 weights (e2m1, e8m0 per 32 in [rows][K / 32]); 1: FP8 E4M3 weights with
+  int sblk;              //    UE8M0 tile scales, one per sblk x sblk tile (128 or 32) in [rows / sblk][K / sblk]
+  alignas(64) CUtensorMap ta, tb;  // MXFP4: 16 x 4-bit -> 16-byte slots; FP8: bytes; box {128, 256}, 128B swizzle
 };
 
 struct GmxHead {
@@ -336,7 +338,8 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
           else if (has_next && pk - KS < KS) tma_prefetch_2d(nmap, (pk - KS) * kXK, nrow);
           const int s = n % kXWS;
           if (n >= kXWS && !wait(&S.wempty[s], (uint32_t)((n / kXWS - 1) & 1))) break;
-          mbar_arrive_expect_tx(&S.wfull[s], (uint32_t)kXStageW / 2);  // counted in packed (4-bit) bytes
+          // counted in global bytes: packed (4-bit) codes, or one byte per FP8 code
+          mbar_arrive_expect_tx(&S.wfull[s], (uint32_t)(G.wfp8 ? kXStageW : kXStageW / 2));
           tma_load_2d(sW + s * kXStageW, map, ks * kXK, wrow, &S.wfull[s], pw);
         }
         map = nmap;
@@ -350,21 +353,38 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
     // ----------------------------------------------------- weight scales --
     // Four reduction steps at a time: every lane loads 16 bytes (4 steps x 4
     // blocks) of eight of the tile's 256 rows, one chunk ahead, and writes
-    // the four steps' two atoms each; one proxy fence and one arrival.
-    const int srow = G.K / 32;  // scale bytes per weight row
-    auto rows_of = [&](int t, const uint8_t*& p) {
+    // the four steps' two atoms each; one proxy fence and one arrival.  FP8
+    // tile scales are expanded to the same per-32 bytes: a 128 x 128 tile's
+    // code serves its rows' four blocks of each step, a 32 x 32 tile's code
+    // one block of 32 rows.
+    const int srow = G.K / 32;  // MXFP4 scale bytes per weight row
+    // the 16 bytes of chunk `chunk` (4 steps) of rows lane + 32 j of tile t
+    auto fetch = [&](int t, int chunk, uint4 (&r)[8]) {
       int f, mb;
       gmx_tile(L, MB, t, f, mb);
       const bool b = mb >= G.MBA;
-      p = (b ? G.sf_b : G.sf_a) + ((size_t)L.tile_e[f] * G.rows_per_e + (b ? mb - G.MBA : mb) * kWN + lane) * srow;
+      const uint8_t* sf = b ? G.sf_b : G.sf_a;
+      const int base = L.tile_e[f] * G.rows_per_e + (b ? mb - G.MBA : mb) * kWN;
+      if (!G.wfp8) {
+        const uint8_t* rp = sf + (size_t)(base + lane) * srow + chunk * 16;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[j] = __ldg(reinterpret_cast<const uint4*>(rp + (size_t)32 * j * srow));
+      } else if (G.sblk == 128) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t c4 = __ldg(reinterpret_cast<const uint32_t*>(
+              sf + (size_t)((base + 32 * j) / 128) * (G.K / 128) + 4 * chunk));
+          r[j] = make_uint4((c4 & 0xFFu) * 0x01010101u, ((c4 >> 8) & 0xFFu) * 0x01010101u,
+                            ((c4 >> 16) & 0xFFu) * 0x01010101u, (c4 >> 24) * 0x01010101u);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          r[j] = __ldg(reinterpret_cast<const uint4*>(sf + (size_t)((base + 32 * j) / 32) * (G.K / 32) + 16 * chunk));
+      }
     };
     uint4 cur[8], nxt[8];
-    const uint8_t* rp = nullptr;
-    if ((int)blockIdx.x < n_tiles) {
-      rows_of(blockIdx.x, rp);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) nxt[j] = __ldg(reinterpret_cast<const uint4*>(rp + (size_t)32 * j * srow));
-    }
+    if ((int)blockIdx.x < n_tiles) fetch(blockIdx.x, 0, nxt);
     int n = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
@@ -372,13 +392,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
 #pragma unroll
         for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
         const int tn = c + 1 < KS / 4 ? t : t + (int)gridDim.x;
-        if (tn < n_tiles) {
-          if (tn != t) rows_of(tn, rp);
-          const int chunk = tn == t ? c + 1 : 0;
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            nxt[j] = __ldg(reinterpret_cast<const uint4*>(rp + (size_t)32 * j * srow + chunk * 16));
-        }
+        if (tn < n_tiles) fetch(tn, tn == t ? c + 1 : 0, nxt);
         uint32_t ff = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -433,7 +447,8 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
     // --------------------------------------------------------------- MMA --
     if (lane == 0) {
       const uint32_t t_sfa = tmem + kXSfaCol, t_sfb = t_sfa + 4;
-      const uint32_t idesc = umma_idesc_mx(128, kWN, 0, 5);  // A e4m3 (token terms), B e2m1 (weights)
+      // A e4m3 (token terms); B e2m1 (MXFP4 weights) or e4m3 (FP8 weights)
+      const uint32_t idesc = umma_idesc_mx(128, kWN, 0, G.wfp8 ? 0 : 5);
       int nw = 0, nt = 0, nc = 0, i = 0;
       for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x, ++i) {
         if (i >= 1 && !wait(&S.acc_empty, (uint32_t)((i - 1) & 1))) break;
@@ -548,6 +563,16 @@ static bool x_map_weights(CUtensorMap* m, const uint8_t* q, int64_t rows, int K)
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
+// FP8 E4M3 rows [rows][K] bytes, boxes {128, 256}, 128-byte swizzle: the same
+// shared-memory layout as the expanded e2m1 slots (one code per byte).
+static bool x_map_fp8(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
+  const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)K};
+  const uint32_t box[2] = {(uint32_t)kXK, (uint32_t)kWN};
+  return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+}
+
 template <bool GATEUP, int NT>
 static qk_status x_launch(const GmxArgs& A, cudaStream_t st) {
   static_assert(sizeof(GmxHead) <= 256, "head");
@@ -597,6 +622,54 @@ qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, 
   g2.MBA = H / kWN;
   g2.out_ld = H;
   if (!x_map_weights(&g2.ta, a.down.q, (int64_t)E * H, I)) return QK_ERR_CUDA;
+  g2.tb = g2.ta;
+  return x_launch<false, 3>(g2, st);
+}
+
+// The FP8 SwiGLU FFN of a shared expert at large M on the same kernels: the M
+// tokens form one group (one expert), x splits into 2 e4m3 terms, gate/up and
+// down run as block-scaled GEMMs with e4m3 weights, and h splits into 3 terms
+// between them.  The caller has counted and tiled the group (W) and adds
+// W.dperm into y.
+qk_status gmx_fp8_ffn(const GroupWs& W, const uint16_t* x, const int32_t* ids, int M, int H, int I,
+                      const uint8_t* wg, const uint8_t* sg, const uint8_t* wu, const uint8_t* su,
+                      const uint8_t* wd, const uint8_t* sd, int blk, cudaStream_t st) {
+  k_gmx_xsplit<<<M, kRowThreads, 0, st>>>(W, x, ids, 1, 1, H, QK_ACT_NONE);
+  if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
+  GmxArgs g1 = {};
+  g1.L = W.L1;
+  g1.blocks = W.xt;
+  g1.atoms = W.sfx;
+  g1.sf_a = sg;
+  g1.sf_b = su;
+  g1.out = W.gu;
+  g1.K = H;
+  g1.rows_per_e = I;
+  g1.MB = 2 * I / kWN;
+  g1.MBA = I / kWN;
+  g1.out_ld = 2 * I;
+  g1.wfp8 = 1;
+  g1.sblk = blk;
+  if (!x_map_fp8(&g1.ta, wg, I, H) || !x_map_fp8(&g1.tb, wu, I, H)) return QK_ERR_CUDA;
+  qk_status rc = x_launch<true, 2>(g1, st);
+  if (rc != QK_OK) return rc;
+  k_gmx_hsplit<<<M, kRowThreads, 0, st>>>(W, 1, I, QK_ACT_NONE);
+  if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
+  GmxArgs g2 = {};
+  g2.L = W.L2;
+  g2.blocks = W.ht;
+  g2.atoms = W.sfh;
+  g2.sf_a = sd;
+  g2.sf_b = sd;
+  g2.out = W.dperm;
+  g2.K = I;
+  g2.rows_per_e = H;
+  g2.MB = H / kWN;
+  g2.MBA = H / kWN;
+  g2.out_ld = H;
+  g2.wfp8 = 1;
+  g2.sblk = blk;
+  if (!x_map_fp8(&g2.ta, wd, H, I)) return QK_ERR_CUDA;
   g2.tb = g2.ta;
   return x_launch<false, 3>(g2, st);
 }

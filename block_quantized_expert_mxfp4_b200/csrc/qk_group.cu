@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kRowThreads) k_grp_h16(GroupWs W, int E, int I
 
 // One block per token: y[t] = sum_s w[t][s] d[pair (t, s)], slots in order.
 __global__ void __launch_bounds__(256) k_grp_combine(GroupWs W, const float* __restrict__ w, int k, int H,
-                                                     void* y, int y_bf16) {
+                                                     void* y, int y_bf16, int accumulate) {
   const int t = blockIdx.x;
   int pos[8];
   float ws[8];
@@ -231,7 +231,9 @@ __global__ void __launch_bounds__(256) k_grp_combine(GroupWs W, const float* __r
     ws[s] = w[t * k + s];
   }
   for (int j = threadIdx.x; j < H / 4; j += blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // y added to (accumulate: the shared expert's output joins the routed one)
+    float4 acc = accumulate ? reinterpret_cast<const float4*>(reinterpret_cast<const float*>(y) + (size_t)t * H)[j]
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s = 0; s < k; ++s) {
       if (pos[s] < 0) continue;
       const float4 d = __ldcg(reinterpret_cast<const float4*>(W.dperm + (size_t)pos[s] * H) + j);
@@ -792,7 +794,7 @@ qk_status group_forward_act(const DecodeArgs& a, int act_quant, void* workspace,
   if (mx) {
     const qk_status rc = gmx_forward_act(a, W, act_quant, st);
     if (rc != QK_OK) return rc;
-    k_grp_combine<<<T, 256, 0, st>>>(W, a.w, k, H, a.y, a.y_bf16);
+    k_grp_combine<<<T, 256, 0, st>>>(W, a.w, k, H, a.y, a.y_bf16, 0);
     return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
   }
   k_grp_scatter<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H);
@@ -829,7 +831,39 @@ qk_status group_forward_act(const DecodeArgs& a, int act_quant, void* workspace,
   g2.tqb = g2.tqa;
   rc = g_dispatch<false>(g2, st);
   if (rc != QK_OK) return rc;
-  k_grp_combine<<<T, 256, 0, st>>>(W, a.w, k, H, a.y, a.y_bf16);
+  k_grp_combine<<<T, 256, 0, st>>>(W, a.w, k, H, a.y, a.y_bf16, 0);
+  return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
+}
+
+// ------------------------------------------------ FP8 shared expert, large M --
+// Every token routed to the one (shared) expert with weight 1.
+__global__ void k_fp8_route_all(int32_t* ids, float* w, int M) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < M; i += gridDim.x * blockDim.x) {
+    ids[i] = 0;
+    w[i] = 1.0f;
+  }
+}
+
+size_t fp8_group_workspace_bytes(int M, int H, int I) {
+  return g_layout(M, 1, 1, H, I, true).total + 2 * align256((size_t)M * 4);
+}
+
+qk_status fp8_group_forward(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
+                            const uint8_t* wu, const uint8_t* su, const uint8_t* wd, const uint8_t* sd, int blk,
+                            float* y, void* workspace, cudaStream_t st) {
+  const size_t base = g_layout(M, 1, 1, H, I, true).total;
+  int32_t* ids = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + base);
+  float* w = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + base + align256((size_t)M * 4));
+  GroupWs W = g_carve(workspace, M, 1, 1, H, I, true);
+  if (cudaMemsetAsync(W.counts, 0, W.zero_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
+  k_fp8_route_all<<<(M + 255) / 256, 256, 0, st>>>(ids, w, M);
+  k_grp_count<<<(M + 255) / 256, 256, 0, st>>>(ids, M, 1, W.counts);
+  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L1, 1, kXTok1, 1, 1);
+  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L2, 1, kXTok2, 1, 0);
+  if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
+  const qk_status rc = gmx_fp8_ffn(W, static_cast<const uint16_t*>(x), ids, M, H, I, wg, sg, wu, su, wd, sd, blk, st);
+  if (rc != QK_OK) return rc;
+  k_grp_combine<<<M, 256, 0, st>>>(W, w, 1, H, y, 0, 1);
   return cudaGetLastError() == cudaSuccess ? QK_OK : QK_ERR_CUDA;
 }
 

@@ -60,6 +60,10 @@ struct GroupWs {
 // MXFP4, hidden and inter are multiples of 512 and the packed weights (32 B)
 // and scales (16 B) are aligned for its copies.
 bool gmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
+// The FP8 shared expert's two GEMMs on the block-scaled grouped kernels.
+qk_status gmx_fp8_ffn(const GroupWs& W, const uint16_t* x, const int32_t* ids, int M, int H, int I,
+                      const uint8_t* wg, const uint8_t* sg, const uint8_t* wu, const uint8_t* su,
+                      const uint8_t* wd, const uint8_t* sd, int blk, cudaStream_t st);
 
 // x split, gate/up GEMM, h split, down GEMM of the MXFP4 path (the counting
 // sort and both tile lists are done; the combine follows).

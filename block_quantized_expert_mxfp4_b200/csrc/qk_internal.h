@@ -55,6 +55,12 @@ qk_status convert_launch(const uint8_t* e8m0, int E, int N, int K, uint8_t* e4m3
 qk_status fp8_linear_launch(const void* x, int M, int K, const uint8_t* w, const uint8_t* ws, int N,
                             void* y, int y_bf16, cudaStream_t st);
 size_t fp8_ffn_workspace_bytes(int M, int H, int I);
+// The FP8 shared expert at large M on the block-scaled grouped kernels (one
+// group of M tokens); fp8_ffn_launch_blk takes it where fp8_big_eligible.
+size_t fp8_group_workspace_bytes(int M, int H, int I);
+qk_status fp8_group_forward(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
+                            const uint8_t* wu, const uint8_t* su, const uint8_t* wd, const uint8_t* sd, int blk,
+                            float* y, void* workspace, cudaStream_t st);
 qk_status fp8_ffn_launch(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
                          const uint8_t* wu, const uint8_t* su, const uint8_t* wd, const uint8_t* sd,
                          float* y, void* ws, cudaStream_t st);

@@ -75,3 +75,25 @@ def test_fp8_shared_expert_32x32_tiles(M):
     hs = workload.make_fp8_shared(1, 0, H, I, device="cpu", block=32)
     so = oracle.fp8_swiglu_ffn(x, hs.wg, hs.sg, hs.wu, hs.su, hs.wd, hs.sd, block=32)
     assert_parity(y.cpu().numpy(), so, what=f"shared expert 32x32 M={M}")
+
+
+@pytest.mark.parametrize("M,block", [(200, 128), (200, 32), (2048, 128)])
+def test_fp8_shared_expert_large_m_block_scaled(M, block):
+    """From 128 rows the shared expert runs on the block-scaled grouped GEMMs
+    (e4m3 weights as stored, tile scales expanded to per-32 codes): 200 rows
+    (ragged token tiles: 3 x 64 + 8 for gate/up, 5 x 40 for down) checked
+    whole, 2048 rows (the prefill size) on 64 rows spread over every tile;
+    the result is added into y."""
+    H, I = 4096, 2048
+    sh = workload.make_fp8_shared(2, 0, H, I, block=block)
+    x = synth.activations(13, M, H)
+    y0 = torch.from_numpy(np.random.default_rng(M + block).standard_normal((M, H)).astype(np.float32))
+    y = y0.cuda().clone()
+    ws = torch.empty(qk.fp8_shared_expert_workspace_size(M, H, I), dtype=torch.uint8, device="cuda")
+    qk.fp8_shared_expert_forward(x.cuda(), sh.wg, sh.sg, sh.wu, sh.su, sh.wd, sh.sd, y, ws, scale_block=block)
+    assert qk.qk_last_device_status() == qk.QK_OK
+    rows = np.arange(M) if M <= 256 else np.unique(np.r_[np.linspace(0, M - 1, 62).round().astype(int), 63, 64])
+    hs = workload.make_fp8_shared(2, 0, H, I, device="cpu", block=block)
+    so = oracle.fp8_swiglu_ffn(x[rows], hs.wg, hs.sg, hs.wu, hs.su, hs.wd, hs.sd, block=block)
+    got = (y.cpu() - y0).numpy()[rows]
+    assert_parity(got, so, what=f"shared expert block-scaled M={M} block={block} ({len(rows)} rows)")
