@@ -388,8 +388,11 @@ def run_ours(args, rank, world, local_rank):
         out["stack43"] = run_stack(args, rank, world, dev)
         out["prefill_16k"] = run_prefill(args, rank, world, dev, tokens=16384, steps=3)
         out["prefill_w4a8"] = run_prefill(args, rank, world, dev, act="e4m3", steps=10)
+        out["prefill_w4a4"] = run_prefill(args, rank, world, dev, act="mxfp4", steps=10)
+        out["prefill_w4a4_16k"] = run_prefill(args, rank, world, dev, tokens=16384, act="mxfp4", steps=3)
         out["shared_fp8_prefill"] = run_shared_fp8(args, rank, world, dev)
-        for key in ("decode_nvfp4", "stack43", "prefill_16k", "prefill_w4a8", "shared_fp8_prefill"):
+        for key in ("decode_nvfp4", "stack43", "prefill_16k", "prefill_w4a8", "prefill_w4a4", "prefill_w4a4_16k",
+                    "shared_fp8_prefill"):
             out["gpu_launches"] += out[key]["gpu_launches"]
     return out
 
@@ -644,7 +647,10 @@ def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0):
     # FP4 (kind::mxf4, four times) is the format's own ceiling.  `flops` is the
     # layer's useful work; the activation terms multiply the MMAs issued (2 for
     # gate/up, 3 for down) but not the work.
-    tpeak, tkind = 2 * bf16, f"{src} bf16 x 2 (nominal fp8/bf16 ratio): the MMA kind used, kind::mxf8f6f4"
+    if aq == qk.QK_ACT_MXFP4:  # both operands e2m1: kind::mxf4, four times the bf16 rate
+        tpeak, tkind = 4 * bf16, f"{src} bf16 x 4 (nominal fp4/bf16 ratio): the MMA kind used, kind::mxf4"
+    else:
+        tpeak, tkind = 2 * bf16, f"{src} bf16 x 2 (nominal fp8/bf16 ratio): the MMA kind used, kind::mxf8f6f4"
     return {
         "workload": f"prefill MoE layer: {T} tokens, {wl.E} experts, top-6 Zipf(s=1) routing, hidden 4096, "
                     "intermediate 2048, MXFP4 gate/up/down, bf16 N(0,1) activations"
@@ -660,8 +666,10 @@ def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0):
         "path": ("counting sort by expert; x as 2 exact e4m3 terms; block-scaled tcgen05 grouped GEMMs "
                  "(e2m1 weights + e8m0 scales as stored): gate/up, SwiGLU + 3-term h split, down; combine")
         if aq == qk.QK_ACT_NONE else
-        (f"counting sort by expert; x and h quantized to {act_name} (one term, the other term slots "
-         "zero); block-scaled tcgen05 grouped GEMMs; combine"),
+        (f"counting sort by expert; x and h quantized to {act_name} (one term per token, 128-token tiles); "
+         + ("both operands packed e2m1, block-scaled tcgen05 kind::mxf4 grouped GEMMs (weights as stored)"
+            if aq == qk.QK_ACT_MXFP4 else "block-scaled tcgen05 kind::mxf8f6f4 grouped GEMMs")
+         + "; combine"),
         "gpu_launches": 8 * K,
     }
 

@@ -8,12 +8,13 @@
 // emax = 8 (e4m3) or 2 (e2m1), scale code X + 127 clamped to [0, 254] (0 for
 // an all-zero block), elements rounded to nearest even and saturated.
 //
-// Each activation is then ONE term in the block-scaled paths' token tiles,
-// instead of the two or three exact e4m3 terms of QK_ACT_NONE; the other
-// term slots are written as zeros (code 0, scale 2^-127), so the tiles, the
-// MMAs and their indexing are exactly those of the exact path.  An e2m1 value
-// is exact in e4m3, so QK_ACT_MXFP4 feeds the same kind::mxf8f6f4 MMA e4m3
-// codes of e2m1 values with the same scale.
+// Each activation is then ONE term in the grouped path's token tiles,
+// instead of the two or three exact e4m3 terms of QK_ACT_NONE, so a tile
+// holds 128 tokens (gmx_tok1/gmx_tok2 give the tile heights per mode).
+// QK_ACT_E4M3 feeds e4m3 codes (one byte each) to kind::mxf8f6f4 against the
+// e2m1 weights; QK_ACT_MXFP4 packs two e2m1 codes per byte (element 2 i in
+// the low nibble of byte i, the weights' own packing) and runs kind::mxf4
+// with both operands as stored, 64 elements of K per instruction.
 //
 // The arithmetic below is host and device code: a CPU test compiles it for
 // the host (QK_ACTQ_ARITHMETIC_ONLY: without the path declarations at the end)
@@ -106,6 +107,32 @@ QK_HD int actq_block(const float (&v)[32], uint32_t (&q)[8], int fp4) {
   return c;
 }
 
+// e2m1 code (bit 3: sign) of a value already on the e2m1 grid.
+QK_HD uint32_t actq_e2m1_code(float r) {
+  const float m = fabsf(r);
+  const uint32_t c = m < 2.f ? (uint32_t)(m * 2.f) : m < 4.f ? (uint32_t)m + 2u : m < 6.f ? 6u : 7u;
+  return c | (signbit(r) ? 8u : 0u);
+}
+
+// One e2m1 term of 32 values as packed codes for the fp4 x fp4 tensor core
+// (element 2 i in the low nibble of byte i, 16 bytes in q): the same values
+// and e8m0 code as actq_block with fp4 set.
+QK_HD int actq_block_fp4(const float (&v)[32], uint32_t (&q)[4]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+  const int c = actq_scale_code(m, actq_emax(1));
+  const float up = actq_up(c);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) word |= actq_e2m1_code(actq_e2m1_rn(v[8 * w + i] * up)) << (4 * i);
+    q[w] = word;
+  }
+  return c;
+}
+
 }  // namespace qk
 
 #if defined(__CUDACC__) && !defined(QK_ACTQ_ARITHMETIC_ONLY)
@@ -117,5 +144,10 @@ namespace qk {
 // group_forward_act(a, QK_ACT_NONE, ...), gmx_forward likewise.
 qk_status group_forward_act(const DecodeArgs& a, int act_quant, void* workspace, cudaStream_t st);
 qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, cudaStream_t st);
+// Token tile heights of the grouped block-scaled path: 64 (gate/up, x as 2
+// terms) and 40 (down, h as 3) with exact activations; 128 for both in the
+// activation-quantized modes (one term per token, every TMEM lane a token).
+__host__ __device__ inline int gmx_tok1(int act_quant) { return act_quant == QK_ACT_NONE ? kXTok1 : 128; }
+__host__ __device__ inline int gmx_tok2(int act_quant) { return act_quant == QK_ACT_NONE ? kXTok2 : 128; }
 }  // namespace qk
 #endif

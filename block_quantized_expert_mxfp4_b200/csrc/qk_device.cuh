@@ -363,6 +363,18 @@ __device__ __forceinline__ void umma_mx(uint32_t tmem_d, uint64_t desc_a, uint64
       "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb));
 }
 
+// The same with both operands packed e2m1 (kind::mxf4, K = 64 per
+// instruction, one ue8m0 scale per 32: the scale column's byte pair from the
+// index in bits 30-31).
+__device__ __forceinline__ void umma_mxf4(uint32_t tmem_d, uint64_t desc_a, uint64_t desc_b, uint32_t idesc,
+                                          uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(
+          tmem_d),
+      "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb));
+}
+
 // Shared-memory descriptor of a scale-factor atom for tcgen05.cp: 32 rows of
 // 16 bytes, contiguous (no swizzle; 8-row groups 128 bytes apart).
 __device__ __forceinline__ uint64_t umma_desc_sf(const void* smem_atom) {

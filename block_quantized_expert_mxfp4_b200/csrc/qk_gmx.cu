@@ -26,12 +26,25 @@
 // the epilogue sums a token's terms with shuffles inside one warp.  Each MMA
 // instruction covers 256 weight rows x 32 elements of K.
 //
-//   k_gmx_xsplit  per token: x -> 2 e4m3 terms, written into the tile blocks
-//                 of each of its pairs (gate/up tiles of 64 tokens).
+// Activation-quantized modes (QK_ACT_E4M3, QK_ACT_MXFP4: one quantized term
+// per token, qk_actq.cuh) use the one-term geometry: lane m of A is token m,
+// 128 tokens per tile, no shuffles in the epilogue.  In QK_ACT_MXFP4 the token
+// blocks hold packed e2m1 (256 elements of K per 128-byte row, a plain byte
+// tensor map for the weights too) and each instruction is kind::mxf4
+// .block_scale.block32 over 64 elements of K, both operands fp4 as stored.
+// The pages' own W8A8/W4A8 kernels keep the activations in 8 bits; fp4 x fp4
+// at 4 x the bf16 rate is what sm_100a adds.  A third mode keeps the weights
+// in e4m3 (kind::mxf8f6f4 with e4m3 on both sides, 128-block scales expanded
+// to per-32 codes): the FP8 shared expert at large M.
+//
+//   k_gmx_xsplit  per token: x -> 2 e4m3 terms (1 term, or packed e2m1, in
+//                 the quantized modes), written into the tile blocks of each
+//                 of its pairs (gate/up tiles of 64 tokens, 128 quantized).
 //   k_gmx<gate/up>  per (expert, 256 gate or up rows, token tile): gate and up
 //                 outputs (fp32) to gu.
 //   k_gmx_hsplit  per sorted row: h = silu(gate) * up -> 3 e4m3 terms in the
-//                 down tile blocks (40 tokens per tile).
+//                 down tile blocks (40 tokens per tile; 1 term or packed
+//                 e2m1 and 128 tokens in the quantized modes).
 //   k_gmx<down>   per (expert, 256 down rows, token tile): d (fp32).
 //
 // Token block (one reduction step of a tile, the MMA's A operand as it sits
@@ -93,13 +106,27 @@ __device__ __forceinline__ void put_term(uint8_t* blocks, uint8_t* atoms, int f,
   atoms[((size_t)f * ns + step) * kSfAtom + (m & 31) * 16 + (m >> 5) * 4 + kb] = (uint8_t)c;
 }
 
+// Packed e2m1 (the fp4 x fp4 tiles of QK_ACT_MXFP4): one reduction step is
+// 256 elements, a 128-byte row of eight 16-byte chunks, one per 32-block
+// (chunk b % 8 of row j, swizzled), and two scale atoms (blocks 0-3 and 4-7
+// of the step).  Row j = token j of the 128-token tile.
+__device__ __forceinline__ void put_fp4(uint8_t* blocks, uint8_t* atoms, int f, int ns4, int j, int b,
+                                        const uint32_t (&q)[4], int c) {
+  const int step = b >> 3, c8 = b & 7;
+  uint8_t* row = blocks + ((size_t)f * ns4 + step) * kXBlock + j * kXK;
+  *reinterpret_cast<uint4*>(row + ((c8 ^ (j & 7)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+  atoms[(((size_t)f * ns4 + step) * 2 + (c8 >> 2)) * kSfAtom + (j & 31) * 16 + (j >> 5) * 4 + (c8 & 3)] = (uint8_t)c;
+}
+
 // One block per token: its pairs' sorted rows (counting-sort scatter) and
-// tile positions, then x split into two e4m3 terms per 32-block (QK_ACT_NONE)
-// or quantized to one term (the activation-quantized modes; second term
-// zero), written into the gate/up tile of each pair.
+// tile positions, then x split into two e4m3 terms per 32-block (QK_ACT_NONE,
+// 64-token tiles) or quantized to one term (the activation-quantized modes,
+// 128-token tiles: e4m3 codes, or packed e2m1 for QK_ACT_MXFP4), written into
+// the gate/up tile of each pair.
 __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uint16_t* __restrict__ x,
                                                             const int32_t* __restrict__ ids, int k, int E, int H,
                                                             int act_quant) {
+  const int tok1 = gmx_tok1(act_quant), tok2 = gmx_tok2(act_quant);
   __shared__ int fj[8];
   const int t = blockIdx.x;
   if (threadIdx.x < k) {
@@ -110,8 +137,8 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
       const int o = W.offsets[e];
       r = o + atomicAdd(&W.fill[e], 1);
       const int rel = r - o;
-      tj = ((W.L1.exp_tile0[e] + rel / kXTok1) << 8) | (rel % kXTok1);
-      W.rtile2[r] = ((W.L2.exp_tile0[e] + rel / kXTok2) << 8) | (rel % kXTok2);
+      tj = ((W.L1.exp_tile0[e] + rel / tok1) << 8) | (rel % tok1);
+      W.rtile2[r] = ((W.L2.exp_tile0[e] + rel / tok2) << 8) | (rel % tok2);
     } else {
       set_status(QK_ERR_INVALID_ARG);
     }
@@ -134,17 +161,21 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
       }
     }
     if (!all_finite32(v)) set_status(QK_ERR_NONFINITE);
-    uint32_t q0[8], q1[8];
-    int c0, c1;
-    if (act_quant == QK_ACT_NONE) {
-      c0 = split_term(v, q0);
-      c1 = split_term(v, q1);
-    } else {
-      c0 = actq_block(v, q0, act_quant == QK_ACT_MXFP4);
-      c1 = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) q1[i] = 0u;
+    if (act_quant == QK_ACT_MXFP4) {
+      uint32_t q4[4];
+      const int c = actq_block_fp4(v, q4);
+      for (int s = 0; s < k; ++s)
+        if (fj[s] >= 0) put_fp4(W.xt, W.sfx, fj[s] >> 8, H / 256, fj[s] & 255, b, q4, c);
+      continue;
     }
+    uint32_t q0[8], q1[8];
+    if (act_quant == QK_ACT_E4M3) {
+      const int c = actq_block(v, q0, 0);
+      for (int s = 0; s < k; ++s)
+        if (fj[s] >= 0) put_term(W.xt, W.sfx, fj[s] >> 8, ns, 32, fj[s] & 255, 0, b, q0, c);
+      continue;
+    }
+    const int c0 = split_term(v, q0), c1 = split_term(v, q1);
     for (int s = 0; s < k; ++s) {
       const int tj = fj[s];
       if (tj < 0) continue;
@@ -155,9 +186,9 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
 }
 
 // One block per sorted row: h = silu(gate) * up in fp32, split into three
-// e4m3 terms per 32-block (QK_ACT_NONE) or quantized to one term (the
-// activation-quantized modes; the other two zero), written into the row's
-// down tile.
+// e4m3 terms per 32-block (QK_ACT_NONE, 40-token tiles) or quantized to one
+// term (the activation-quantized modes, 128-token tiles: e4m3 codes, or
+// packed e2m1 for QK_ACT_MXFP4), written into the row's down tile.
 __global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, int I, int act_quant) {
   const int r = blockIdx.x;
   if (r >= W.offsets[E]) return;  // block-uniform
@@ -183,14 +214,14 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, in
         const int c = split_term(v, q);
         put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, term, b, q, c);
       }
-    } else {
+    } else if (act_quant == QK_ACT_MXFP4) {  // one packed e2m1 term, 128-token tiles
+      uint32_t q4[4];
+      const int c = actq_block_fp4(v, q4);
+      put_fp4(W.ht, W.sfh, f, I / 256, j, b, q4, c);
+    } else {  // one e4m3 term, 128-token tiles
       uint32_t q[8];
-      const int c = actq_block(v, q, act_quant == QK_ACT_MXFP4);
-      put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, 0, b, q, c);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) q[i] = 0u;
-      put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, 1, b, q, 0);
-      put_term(W.ht, W.sfh, f, ns, kXTok2 / 4, j, 2, b, q, 0);
+      const int c = actq_block(v, q, 0);
+      put_term(W.ht, W.sfh, f, ns, 32, j, 0, b, q, c);
     }
   }
 }
@@ -210,7 +241,7 @@ constexpr int kXSS = 2;                // weight-scale chunk slots (4 steps x 2 
 constexpr int kXSfaCol = 256;          // token scales: 4 columns; weight scales: 8 columns after them
 constexpr int kXPrefetch = 8;          // weight steps prefetched into L2 ahead of the TMA ring
 constexpr int kXTmemCols = 512;
-constexpr int kXSmem = 1024 + kXWS * kXStageW + kXTS * (kXStageT + 2 * kSfAtom) + kXSS * 8 * kSfAtom + 256;
+constexpr int kXSmem = 1024 + kXWS * kXStageW + kXTS * (kXStageT + 4 * kSfAtom) + kXSS * 8 * kSfAtom + 256;
 
 struct GmxArgs {
   TileList L;            // token tiles of this phase
@@ -256,19 +287,27 @@ __device__ __forceinline__ void gmx_tile(const TileList& L, int MB, int t, int& 
   f = first + (u - mb * cnt);
 }
 
-template <bool GATEUP, int NT>
+// NT: terms per token (2 for x, 3 for h, 1 in the activation-quantized
+// modes).  FP4: both operands packed e2m1 (QK_ACT_MXFP4), kind::mxf4 with a
+// reduction step of 256 elements (the weights copied as stored, 32 KB per
+// stage), two token scale atoms per step and two steps per weight-scale
+// chunk; otherwise kind::mxf8f6f4 with steps of 128.
+template <bool GATEUP, int NT, bool FP4>
 __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ GmxArgs G) {
-  constexpr int NPQ = NT == 2 ? kXTok1 / 4 : kXTok2 / 4;  // tokens per TMEM lane quadrant
+  static_assert(!FP4 || NT == 1, "the fp4 x fp4 tiles hold one term");
+  constexpr int NPQ = NT == 1 ? 32 : NT == 2 ? kXTok1 / 4 : kXTok2 / 4;  // tokens per TMEM lane quadrant
+  constexpr int AT = FP4 ? 2 : 1;    // token scale atoms per step
+  constexpr int SPC = FP4 ? 2 : 4;   // steps per weight-scale chunk (16 bytes of each row: 512 elements)
   extern __shared__ __align__(16) uint8_t smem_raw[];  // rounded up to 1024 below, at run time
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sW = base;                                  // kXWS weight stages
   uint8_t* sT = sW + kXWS * kXStageW;                  // kXTS token stages
-  uint8_t* sTa = sT + kXTS * kXStageT;                 // kXTS x 2 token scale atoms
-  uint8_t* sSa = sTa + kXTS * 2 * kSfAtom;             // kXSS x 8 weight scale atoms
+  uint8_t* sTa = sT + kXTS * kXStageT;                 // kXTS x 4 token scale atoms (2 steps x AT)
+  uint8_t* sSa = sTa + kXTS * 4 * kSfAtom;             // kXSS x 8 weight scale atoms
   GmxHead& S = *reinterpret_cast<GmxHead*>(sSa + kXSS * 8 * kSfAtom);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const TileList& L = G.L;
-  const int MB = G.MB, KS = G.K / kXK;
+  const int MB = G.MB, KS = G.K / (FP4 ? 2 * kXK : kXK);
   const unsigned long long limit = g_wait_limit_ns;
 
   if (threadIdx.x == 0) {
@@ -339,7 +378,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
           const int s = n % kXWS;
           if (n >= kXWS && !wait(&S.wempty[s], (uint32_t)((n / kXWS - 1) & 1))) break;
           // counted in global bytes: packed (4-bit) codes, or one byte per FP8 code
-          mbar_arrive_expect_tx(&S.wfull[s], (uint32_t)(G.wfp8 ? kXStageW : kXStageW / 2));
+          mbar_arrive_expect_tx(&S.wfull[s], (uint32_t)(G.wfp8 || FP4 ? kXStageW : kXStageW / 2));
           tma_load_2d(sW + s * kXStageW, map, ks * kXK, wrow, &S.wfull[s], pw);
         }
         map = nmap;
@@ -388,10 +427,10 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
     int n = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-      for (int c = 0; c < KS / 4; ++c, ++n) {
+      for (int c = 0; c < KS / SPC; ++c, ++n) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
-        const int tn = c + 1 < KS / 4 ? t : t + (int)gridDim.x;
+        const int tn = c + 1 < KS / SPC ? t : t + (int)gridDim.x;
         if (tn < n_tiles) fetch(tn, tn == t ? c + 1 : 0, nxt);
         uint32_t ff = 0;
 #pragma unroll
@@ -433,10 +472,10 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
           if (k0 + 2 * kXTS < KS)  // the stage after the ring into L2
             bulk_prefetch_l2(G.blocks + ((size_t)f * KS + k0 + 2 * kXTS) * kXBlock, (uint32_t)kXStageT);
           if (n >= kXTS && !wait(&S.tempty[s], (uint32_t)((n / kXTS - 1) & 1))) break;
-          mbar_arrive_expect_tx(&S.tfull[s], (uint32_t)(kXStageT + 2 * kSfAtom));
+          mbar_arrive_expect_tx(&S.tfull[s], (uint32_t)(kXStageT + 2 * AT * kSfAtom));
           const size_t blk = (size_t)f * KS + k0;
           bulk_g2s(sT + s * kXStageT, G.blocks + blk * kXBlock, (uint32_t)kXStageT, &S.tfull[s]);
-          bulk_g2s(sTa + s * 2 * kSfAtom, G.atoms + blk * kSfAtom, (uint32_t)(2 * kSfAtom), &S.tfull[s]);
+          bulk_g2s(sTa + s * 4 * kSfAtom, G.atoms + blk * AT * kSfAtom, (uint32_t)(2 * AT * kSfAtom), &S.tfull[s]);
         }
       }
       for (int q = n > kXTS ? n - kXTS : 0; q < n; ++q)
@@ -446,16 +485,17 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
   } else if (warp == 1) {
     // --------------------------------------------------------------- MMA --
     if (lane == 0) {
-      const uint32_t t_sfa = tmem + kXSfaCol, t_sfb = t_sfa + 4;
-      // A e4m3 (token terms); B e2m1 (MXFP4 weights) or e4m3 (FP8 weights)
-      const uint32_t idesc = umma_idesc_mx(128, kWN, 0, G.wfp8 ? 0 : 5);
+      const uint32_t t_sfa = tmem + kXSfaCol, t_sfb = t_sfa + 4 * AT;
+      // A e4m3 (token terms); B e2m1 (MXFP4 weights) or e4m3 (FP8 weights);
+      // FP4: both e2m1 (format 1 of kind::mxf4)
+      const uint32_t idesc = FP4 ? umma_idesc_mx(128, kWN, 1, 1) : umma_idesc_mx(128, kWN, 0, G.wfp8 ? 0 : 5);
       int nw = 0, nt = 0, nc = 0, i = 0;
       for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x, ++i) {
         if (i >= 1 && !wait(&S.acc_empty, (uint32_t)((i - 1) & 1))) break;
         tc_fence_after();
         bool ok = true;
         for (int ks = 0; ks < KS; ++ks, ++nw) {
-          const int sw = nw % kXWS, st = nt % kXTS, sc = nc % kXSS, j = ks & 1, q = ks & 3;
+          const int sw = nw % kXWS, st = nt % kXTS, sc = nc % kXSS, j = ks & 1, q = ks % SPC;
           if (!wait(&S.wfull[sw], (uint32_t)((nw / kXWS) & 1)) ||
               (j == 0 && !wait(&S.tfull[st], (uint32_t)((nt / kXTS) & 1))) ||
               (q == 0 && !wait(&S.sfull[sc], (uint32_t)((nc / kXSS) & 1)))) {
@@ -463,21 +503,41 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
             break;
           }
           tc_fence_after();
-          utccp_32x128b_x4(t_sfa, umma_desc_sf(sTa + (st * 2 + j) * kSfAtom));
-          utccp_32x128b_x4(t_sfb, umma_desc_sf(sSa + (sc * 8 + q * 2) * kSfAtom));
-          utccp_32x128b_x4(t_sfb + 4, umma_desc_sf(sSa + (sc * 8 + q * 2 + 1) * kSfAtom));
           const uint64_t da = umma_desc_k_sw128(sT + st * kXStageT + j * kXBlock);
           const uint64_t db = umma_desc_k_sw128(sW + sw * kXStageW);
+          if (!FP4) {
+            utccp_32x128b_x4(t_sfa, umma_desc_sf(sTa + (st * 4 + j) * kSfAtom));
+            utccp_32x128b_x4(t_sfb, umma_desc_sf(sSa + (sc * 8 + q * 2) * kSfAtom));
+            utccp_32x128b_x4(t_sfb + 4, umma_desc_sf(sSa + (sc * 8 + q * 2 + 1) * kSfAtom));
 #pragma unroll
-          for (int kb = 0; kb < kXK / 32; ++kb)
-            umma_mx(tmem, da + 2 * kb, db + 2 * kb, umma_idesc_sf_ids(idesc, kb, kb), t_sfa | ((uint32_t)kb << 30),
-                    t_sfb | ((uint32_t)kb << 30), (ks | kb) != 0 ? 1u : 0u);
+            for (int kb = 0; kb < kXK / 32; ++kb)
+              umma_mx(tmem, da + 2 * kb, db + 2 * kb, umma_idesc_sf_ids(idesc, kb, kb), t_sfa | ((uint32_t)kb << 30),
+                      t_sfb | ((uint32_t)kb << 30), (ks | kb) != 0 ? 1u : 0u);
+          } else {
+            // blocks 0-3 and 4-7 of the step: token atoms in columns t_sfa and
+            // t_sfa + 4, weight atoms (rows 0-127, 128-255) at t_sfb + 8 g and
+            // + 4; MMA k (K = 64) takes blocks 2 k, 2 k + 1: group k / 2, byte
+            // pair 2 (k % 2)
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              utccp_32x128b_x4(t_sfa + 4 * g, umma_desc_sf(sTa + (st * 4 + j * 2 + g) * kSfAtom));
+              utccp_32x128b_x4(t_sfb + 8 * g, umma_desc_sf(sSa + (sc * 8 + (2 * q + g) * 2) * kSfAtom));
+              utccp_32x128b_x4(t_sfb + 8 * g + 4, umma_desc_sf(sSa + (sc * 8 + (2 * q + g) * 2 + 1) * kSfAtom));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t sid = (uint32_t)(kk & 1) * 2;
+              umma_mxf4(tmem, da + 2 * kk, db + 2 * kk, umma_idesc_sf_ids(idesc, (int)sid, (int)sid),
+                        (t_sfa + 4 * (kk >> 1)) | (sid << 30), (t_sfb + 8 * (kk >> 1)) | (sid << 30),
+                        (ks | kk) != 0 ? 1u : 0u);
+            }
+          }
           umma_commit(&S.wempty[sw]);
           if (j == 1) {
             umma_commit(&S.tempty[st]);
             ++nt;
           }
-          if (q == 3) {
+          if (q == SPC - 1) {
             umma_commit(&S.sempty[sc]);
             ++nc;
           }
@@ -514,12 +574,14 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
           __syncwarp();
           if (lane == 0) mbar_arrive_one(&S.acc_empty);
         }
+        if (NT > 1) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          float a = __uint_as_float(v[jj]);
-          a += __shfl_down_sync(0xffffffffu, a, NPQ);
-          if (NT == 3) a += __shfl_down_sync(0xffffffffu, __uint_as_float(v[jj]), 2 * NPQ);
-          v[jj] = __float_as_uint(a);
+          for (int jj = 0; jj < 32; ++jj) {
+            float a = __uint_as_float(v[jj]);
+            a += __shfl_down_sync(0xffffffffu, a, NPQ);
+            if (NT == 3) a += __shfl_down_sync(0xffffffffu, __uint_as_float(v[jj]), 2 * NPQ);
+            v[jj] = __float_as_uint(a);
+          }
         }
         if (st) {
           float4* o4 = reinterpret_cast<float4*>(out + c * 32);
@@ -573,11 +635,21 @@ static bool x_map_fp8(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
-template <bool GATEUP, int NT>
+template <bool GATEUP, int NT, bool FP4 = false>
 static qk_status x_launch(const GmxArgs& A, cudaStream_t st) {
   static_assert(sizeof(GmxHead) <= 256, "head");
   if (kXSmem > max_smem_optin()) return QK_ERR_UNSUPPORTED;
-  return launch_ex(k_gmx<GATEUP, NT>, dim3(num_sms()), dim3(kXThreads), (size_t)kXSmem, st, false, A);
+  return launch_ex(k_gmx<GATEUP, NT, FP4>, dim3(num_sms()), dim3(kXThreads), (size_t)kXSmem, st, false, A);
+}
+
+// Packed e2m1 rows [rows][K / 2] as bytes, boxes {128 bytes (256 codes), 256
+// rows}, 128-byte swizzle: the fp4 x fp4 path reads the weights as stored.
+static bool x_map_packed(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
+  const uint64_t dims[2] = {(uint64_t)K / 2, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)K / 2};
+  const uint32_t box[2] = {(uint32_t)kXK, (uint32_t)kWN};
+  return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st) {
@@ -586,8 +658,12 @@ qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st) {
 
 qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, cudaStream_t st) {
   const int T = a.T, k = a.k, E = a.E, H = a.H, I = a.I;
+  const bool fp4 = act_quant == QK_ACT_MXFP4, one = act_quant != QK_ACT_NONE;
   k_gmx_xsplit<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H, act_quant);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
+  auto wmap = [&](CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
+    return fp4 ? x_map_packed(m, q, rows, K) : x_map_weights(m, q, rows, K);
+  };
 
   GmxArgs g1 = {};
   g1.L = W.L1;
@@ -601,9 +677,8 @@ qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, 
   g1.MB = 2 * I / kWN;  // gate blocks, then up blocks
   g1.MBA = I / kWN;
   g1.out_ld = 2 * I;
-  if (!x_map_weights(&g1.ta, a.gate.q, (int64_t)E * I, H) || !x_map_weights(&g1.tb, a.up.q, (int64_t)E * I, H))
-    return QK_ERR_CUDA;
-  qk_status rc = x_launch<true, 2>(g1, st);
+  if (!wmap(&g1.ta, a.gate.q, (int64_t)E * I, H) || !wmap(&g1.tb, a.up.q, (int64_t)E * I, H)) return QK_ERR_CUDA;
+  qk_status rc = fp4 ? x_launch<true, 1, true>(g1, st) : one ? x_launch<true, 1>(g1, st) : x_launch<true, 2>(g1, st);
   if (rc != QK_OK) return rc;
 
   k_gmx_hsplit<<<a.P, kRowThreads, 0, st>>>(W, E, I, act_quant);
@@ -621,9 +696,9 @@ qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, 
   g2.MB = H / kWN;
   g2.MBA = H / kWN;
   g2.out_ld = H;
-  if (!x_map_weights(&g2.ta, a.down.q, (int64_t)E * H, I)) return QK_ERR_CUDA;
+  if (!wmap(&g2.ta, a.down.q, (int64_t)E * H, I)) return QK_ERR_CUDA;
   g2.tb = g2.ta;
-  return x_launch<false, 3>(g2, st);
+  return fp4 ? x_launch<false, 1, true>(g2, st) : one ? x_launch<false, 1>(g2, st) : x_launch<false, 3>(g2, st);
 }
 
 // The FP8 SwiGLU FFN of a shared expert at large M on the same kernels: the M

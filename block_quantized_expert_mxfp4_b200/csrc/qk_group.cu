@@ -788,8 +788,8 @@ qk_status group_forward_act(const DecodeArgs& a, int act_quant, void* workspace,
   GroupWs W = g_carve(workspace, T, k, E, H, I, mx);
   if (cudaMemsetAsync(W.counts, 0, W.zero_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
   k_grp_count<<<(P + 255) / 256, 256, 0, st>>>(a.ids, P, E, W.counts);
-  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L1, E, mx ? kXTok1 : kGN, mx ? 1 : 0, 1);
-  if (mx) k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L2, E, kXTok2, 1, 0);
+  k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L1, E, mx ? gmx_tok1(act_quant) : kGN, mx ? 1 : 0, 1);
+  if (mx) k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L2, E, gmx_tok2(act_quant), 1, 0);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
   if (mx) {
     const qk_status rc = gmx_forward_act(a, W, act_quant, st);

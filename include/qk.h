@@ -72,7 +72,9 @@ enum { QK_FMT_MXFP4 = 1, QK_FMT_NVFP4 = 2 };
  *                32 ([REAP25] v0.2.3 update: fp4 weights x dynamic E4M3
  *                activations on block-scaled f8f6f4 tensor cores, the model's
  *                own expert numerics), x before gate/up and h before down.
- *  QK_ACT_MXFP4  the same with e2m1 activations (fp4 x fp4).
+ *  QK_ACT_MXFP4  the same with e2m1 activations (fp4 x fp4, run on the
+ *                kind::mxf4 block-scaled tensor cores with both operands
+ *                packed e2m1).
  * Scale rule for both (the pages give none; OCP Microscaling v1.0): X =
  * floor(log2 max|v|) - 8 (e4m3) or - 2 (e2m1) per 32 values, clamped to the
  * e8m0 range; elements rounded to nearest even, saturating (E4M3 to 448,

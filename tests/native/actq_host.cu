@@ -15,3 +15,15 @@ extern "C" void actq_host(const float* v, int n, int fp4, uint8_t* codes, uint8_
     memcpy(codes + b * 32, q, 32);
   }
 }
+
+// The packed e2m1 form of the fp4 x fp4 tiles: 16 bytes per 32 values
+// (element 2 i in the low nibble of byte i) and one e8m0 code per 32.
+extern "C" void actq_host_fp4packed(const float* v, int n, uint8_t* packed, uint8_t* scales) {
+  for (int b = 0; b < n / 32; ++b) {
+    float blk[32];
+    uint32_t q[4];
+    for (int i = 0; i < 32; ++i) blk[i] = v[b * 32 + i];
+    scales[b] = (uint8_t)qk::actq_block_fp4(blk, q);
+    memcpy(packed + b * 16, q, 16);
+  }
+}

@@ -30,6 +30,7 @@ def host():
                                "-I", os.path.join(ROOT, "include"), SRC, "-o", OUT])
     L = ctypes.CDLL(OUT)
     L.actq_host.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    L.actq_host_fp4packed.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
 
     def run(v, fp4):
         v = np.ascontiguousarray(v, np.float32)
@@ -37,6 +38,14 @@ def host():
         scales = np.empty(v.size // 32, np.uint8)
         L.actq_host(v.ctypes.data, v.size, int(fp4), codes.ctypes.data, scales.ctypes.data)
         return codes, scales
+
+    def packed(v):
+        v = np.ascontiguousarray(v, np.float32)
+        p = np.empty(v.size // 2, np.uint8)
+        scales = np.empty(v.size // 32, np.uint8)
+        L.actq_host_fp4packed(v.ctypes.data, v.size, p.ctypes.data, scales.ctypes.data)
+        return p, scales
+    run.packed = packed
     return run
 
 
@@ -93,3 +102,21 @@ def test_matches_oracle_bit_for_bit(host, fp4, kind):
         assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want))
     else:
         assert np.array_equal(codes, oc)
+
+
+@pytest.mark.parametrize("kind", ["fp32", "bf16"])
+def test_packed_e2m1_matches_oracle_codes(host, kind):
+    """The packed form the fp4 x fp4 tensor core reads (QK_ACT_MXFP4 tiles):
+    every nibble is the oracle's e2m1 code (sign included) and every scale its
+    e8m0 code; element 2 i sits in the low nibble of byte i, as in the packed
+    weights."""
+    v = _blocks()
+    if kind == "bf16":
+        v = _bf16(v)
+    p, scales = host.packed(v)
+    oc, os_, _ = oracle.act_quant(v.astype(np.float64), oracle.ACT_MXFP4)
+    nib = np.empty(v.size, np.uint8)
+    nib[0::2], nib[1::2] = p & 0xF, p >> 4
+    assert np.array_equal(scales, os_)
+    assert np.array_equal(nib, oc)
+

@@ -97,6 +97,31 @@ def test_w4a8_prefill_zipf_sampled_tokens():
            f"w4a8 prefill: {len(pick)} tokens covering every expert")
 
 
+def test_w4a4_prefill_zipf_sampled_tokens():
+    """The 2048-token Zipf prefill layer with QK_ACT_MXFP4 (fp4 x fp4:
+    kind::mxf4 on 128-token tiles, the hottest expert's group spanning about
+    eleven of them): the tokens that open and close every expert's token
+    tiles, and 10 random ones."""
+    wl = synth.WORKLOADS["prefill"]
+    layer = workload.make_layer(wl, 26, 0)
+    x = synth.activations(26, wl.T, wl.H)
+    oids, ow = oracle.route_topk(synth.zipf_logits(26, wl.T, wl.E, wl.k), wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda(),
+                 qk.QK_ACT_MXFP4)
+    first, last = {}, {}
+    for t in range(wl.T):
+        for e in oids[t]:
+            first.setdefault(int(e), t)
+            last[int(e)] = t
+    counts = np.bincount(oids.reshape(-1))
+    hot = np.nonzero((oids == int(np.argmax(counts))).any(1))[0]
+    pick = set(first.values()) | set(last.values()) | set(int(t) for t in hot[127::128]) | set(int(t) for t in hot[128::128])
+    pick |= set(int(t) for t in np.random.default_rng(27).choice(wl.T, 10, replace=False))
+    pick = sorted(pick)
+    _check(wl, 26, x[pick], oids[pick], ow[pick], y[pick], qk.QK_ACT_MXFP4,
+           f"w4a4 prefill: {len(pick)} tokens covering every expert")
+
+
 @pytest.mark.parametrize("aq", MODES)
 def test_modes_are_deterministic_and_differ_from_bf16(aq):
     wl = synth.Workload("mid", 16, 4, 1024, 512, 24, 118, 127)
