@@ -81,16 +81,16 @@ extern "C" {
 static int decode_chunk(int top_k) { return kMaxPairs / top_k; }
 
 // The activation-quantized modes run on the grouped block-scaled kernels at
-// every token count (all-MXFP4 layers that qualify for them).
+// every token count: all-MXFP4 layers that qualify for them, and all-NVFP4
+// layers in QK_ACT_MXFP4 (kind::mxf4nvf4).
 static bool act_quant_ok(const qk_moe_layer* L, int32_t act_quant) {
-  return (act_quant == QK_ACT_MXFP4 || act_quant == QK_ACT_E4M3) &&
-         gmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter);
+  return group_workspace_bytes_act(L, 1, 1, act_quant) > 0;
 }
 
 size_t moe_expert_workspace_size(const qk_moe_layer* L, int32_t n_tokens, int32_t top_k, int32_t act_quant) {
   if (layer_ok(L) != QK_OK || n_tokens < 0 || top_k < 1 || top_k > 8) return 0;
   if (act_quant != QK_ACT_NONE)
-    return act_quant_ok(L, act_quant) ? group_workspace_bytes(L, n_tokens, top_k) : 0;
+    return group_workspace_bytes_act(L, n_tokens, top_k, act_quant);
   if (n_tokens > decode_chunk(top_k))
     return group_workspace_bytes(L, n_tokens, top_k);
   if (dmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter))

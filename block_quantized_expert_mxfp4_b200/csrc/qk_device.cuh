@@ -375,6 +375,24 @@ __device__ __forceinline__ void umma_mxf4(uint32_t tmem_d, uint64_t desc_a, uint
       "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb));
 }
 
+// Instruction descriptor of kind::mxf4nvf4 with both operands e2m1 and ue4m3
+// scales (bit 23 clear): the NVFP4 block-16 form.
+__host__ __device__ constexpr uint32_t umma_idesc_nv(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Both operands packed e2m1 with one ue4m3 scale per 16 elements
+// (kind::mxf4nvf4, block16: K = 64 per instruction, the scale column's four
+// bytes are the instruction's four blocks).
+__device__ __forceinline__ void umma_nvf4(uint32_t tmem_d, uint64_t desc_a, uint64_t desc_b, uint32_t idesc,
+                                          uint32_t tsfa, uint32_t tsfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(
+          tmem_d),
+      "l"(desc_a), "l"(desc_b), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb));
+}
+
 // Shared-memory descriptor of a scale-factor atom for tcgen05.cp: 32 rows of
 // 16 bytes, contiguous (no swizzle; 8-row groups 128 bytes apart).
 __device__ __forceinline__ uint64_t umma_desc_sf(const void* smem_atom) {

@@ -118,6 +118,45 @@ __device__ __forceinline__ void put_fp4(uint8_t* blocks, uint8_t* atoms, int f, 
   atoms[(((size_t)f * ns4 + step) * 2 + (c8 >> 2)) * kSfAtom + (j & 31) * 16 + (j >> 5) * 4 + (c8 & 3)] = (uint8_t)c;
 }
 
+// The same tiles with ue4m3 scales per 16 (NVFP4 layers, kind::mxf4nvf4):
+// four atoms per step, atom a holding blocks 4 a .. 4 a + 3 of 16; the
+// 32-block's two halves take the same code.
+__device__ __forceinline__ void put_nv(uint8_t* blocks, uint8_t* atoms, int f, int ns4, int j, int b,
+                                       const uint32_t (&q)[4], uint32_t code) {
+  const int step = b >> 3, c8 = b & 7;
+  uint8_t* row = blocks + ((size_t)f * ns4 + step) * kXBlock + j * kXK;
+  *reinterpret_cast<uint4*>(row + ((c8 ^ (j & 7)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+  *reinterpret_cast<uint16_t*>(atoms + (((size_t)f * ns4 + step) * 4 + (c8 >> 1)) * kSfAtom + (j & 31) * 16 +
+                               (j >> 5) * 4 + 2 * (c8 & 1)) = (uint16_t)(code * 0x0101u);
+}
+
+// ue4m3 code of 2^d (d <= 8); 0 below 2^-9, the smallest subnormal.
+__device__ __forceinline__ uint32_t nv_pow2_code(int d) {
+  if (d >= -6) return (uint32_t)(d + 7) << 3;
+  return d >= -9 ? 1u << (d + 9) : 0u;
+}
+
+// 2^e as fp32 for -149 <= e <= 127 (subnormal below -126).
+__device__ __forceinline__ float pow2f_sub(int e) {
+  return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
+}
+
+// NVFP4 layers in QK_ACT_MXFP4: the row's 32-block scale codes c (the OCP
+// rule, as for MXFP4 layers) become ue4m3 codes of 2^(c - cmax + 8), cmax the
+// row's largest, and the row's factor 2^(cmax - 135) goes to the epilogue:
+// the product is exact while c >= cmax - 17; a block further below its row's
+// largest (values under 2^-17 of them) is flushed to zero.
+__device__ __forceinline__ int row_max_code(int c) {
+  __shared__ int cm;
+  if (threadIdx.x == 0) cm = 0;
+  __syncthreads();
+  atomicMax(&cm, c);
+  __syncthreads();
+  const int r = cm;
+  __syncthreads();
+  return r;
+}
+
 // One block per token: its pairs' sorted rows (counting-sort scatter) and
 // tile positions, then x split into two e4m3 terms per 32-block (QK_ACT_NONE,
 // 64-token tiles) or quantized to one term (the activation-quantized modes,
@@ -125,7 +164,7 @@ __device__ __forceinline__ void put_fp4(uint8_t* blocks, uint8_t* atoms, int f, 
 // the gate/up tile of each pair.
 __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uint16_t* __restrict__ x,
                                                             const int32_t* __restrict__ ids, int k, int E, int H,
-                                                            int act_quant) {
+                                                            int act_quant, int nv) {
   const int tok1 = gmx_tok1(act_quant), tok2 = gmx_tok2(act_quant);
   __shared__ int fj[8];
   const int t = blockIdx.x;
@@ -148,8 +187,7 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
   __syncthreads();
   const int nb = H / 32, ns = H / kXK;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-  for (int b = threadIdx.x; b < nb; b += kRowThreads) {
-    float v[32];
+  auto load = [&](int b, float (&v)[32]) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint4 u = __ldg(src + b * 4 + q);
@@ -160,6 +198,31 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
         v[q * 8 + 2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
       }
     }
+  };
+  if (nv) {  // QK_ACT_MXFP4 on an NVFP4 layer: the codes twice, the row's largest scale between
+    int cm = 0;
+    for (int b = threadIdx.x; b < nb; b += kRowThreads) {
+      float v[32];
+      uint32_t q4[4];
+      load(b, v);
+      if (!all_finite32(v)) set_status(QK_ERR_NONFINITE);
+      cm = max(cm, actq_block_fp4(v, q4));
+    }
+    cm = row_max_code(cm);
+    for (int b = threadIdx.x; b < nb; b += kRowThreads) {
+      float v[32];
+      uint32_t q4[4];
+      load(b, v);
+      const uint32_t code = nv_pow2_code(actq_block_fp4(v, q4) - cm + 8);
+      for (int s = 0; s < k; ++s)
+        if (fj[s] >= 0) put_nv(W.xt, W.sfx, fj[s] >> 8, H / 256, fj[s] & 255, b, q4, code);
+    }
+    if (threadIdx.x < k && fj[threadIdx.x] >= 0) W.fac1[W.inv[t * k + threadIdx.x]] = pow2f_sub(cm - 135);
+    return;
+  }
+  for (int b = threadIdx.x; b < nb; b += kRowThreads) {
+    float v[32];
+    load(b, v);
     if (!all_finite32(v)) set_status(QK_ERR_NONFINITE);
     if (act_quant == QK_ACT_MXFP4) {
       uint32_t q4[4];
@@ -189,15 +252,14 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
 // e4m3 terms per 32-block (QK_ACT_NONE, 40-token tiles) or quantized to one
 // term (the activation-quantized modes, 128-token tiles: e4m3 codes, or
 // packed e2m1 for QK_ACT_MXFP4), written into the row's down tile.
-__global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, int I, int act_quant) {
+__global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, int I, int act_quant, int nv) {
   const int r = blockIdx.x;
   if (r >= W.offsets[E]) return;  // block-uniform
   const int tj = W.rtile2[r], f = tj >> 8, j = tj & 255;
   const float4* g4 = reinterpret_cast<const float4*>(W.gu + (size_t)r * 2 * I);
   const float4* u4 = g4 + I / 4;
   const int nb = I / 32, ns = I / kXK;
-  for (int b = threadIdx.x; b < nb; b += kRowThreads) {
-    float v[32];
+  auto swiglu = [&](int b, float (&v)[32]) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const float4 g = __ldcg(g4 + b * 8 + q), u = __ldcg(u4 + b * 8 + q);
@@ -206,6 +268,30 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, in
       v[4 * q + 2] = __fdividef(g.z, 1.0f + __expf(-g.z)) * u.z;
       v[4 * q + 3] = __fdividef(g.w, 1.0f + __expf(-g.w)) * u.w;
     }
+  };
+  if (nv) {  // QK_ACT_MXFP4 on an NVFP4 layer (see k_gmx_xsplit)
+    int cm = 0;
+    for (int b = threadIdx.x; b < nb; b += kRowThreads) {
+      float v[32];
+      uint32_t q4[4];
+      swiglu(b, v);
+      if (!all_finite32(v)) set_status(QK_ERR_NONFINITE);
+      cm = max(cm, actq_block_fp4(v, q4));
+    }
+    cm = row_max_code(cm);
+    for (int b = threadIdx.x; b < nb; b += kRowThreads) {
+      float v[32];
+      uint32_t q4[4];
+      swiglu(b, v);
+      const uint32_t code = nv_pow2_code(actq_block_fp4(v, q4) - cm + 8);
+      put_nv(W.ht, W.sfh, f, I / 256, j, b, q4, code);
+    }
+    if (threadIdx.x == 0) W.fac2[r] = pow2f_sub(cm - 135);
+    return;
+  }
+  for (int b = threadIdx.x; b < nb; b += kRowThreads) {
+    float v[32];
+    swiglu(b, v);
     if (!all_finite32(v)) set_status(QK_ERR_NONFINITE);
     if (act_quant == QK_ACT_NONE) {
 #pragma unroll
@@ -241,7 +327,8 @@ constexpr int kXSS = 2;                // weight-scale chunk slots (4 steps x 2 
 constexpr int kXSfaCol = 256;          // token scales: 4 columns; weight scales: 8 columns after them
 constexpr int kXPrefetch = 8;          // weight steps prefetched into L2 ahead of the TMA ring
 constexpr int kXTmemCols = 512;
-constexpr int kXSmem = 1024 + kXWS * kXStageW + kXTS * (kXStageT + 4 * kSfAtom) + kXSS * 8 * kSfAtom + 256;
+constexpr int kXTSa = 8;               // token scale atoms per token stage (2 steps x up to 4)
+constexpr int kXSmem = 1024 + kXWS * kXStageW + kXTS * (kXStageT + kXTSa * kSfAtom) + kXSS * 8 * kSfAtom + 256;
 
 struct GmxArgs {
   TileList L;            // token tiles of this phase
@@ -253,6 +340,9 @@ struct GmxArgs {
   int K, rows_per_e, MB, MBA, out_ld;  // MBA: weight blocks taken from ta / sf_a (the rest: tb / sf_b)
   int wfp8;              // 0: MXFP4 weights (e2m1, e8m0 per 32 in [rows][K / 32]); 1: FP8 E4M3 weights with
   int sblk;              //    UE8M0 tile scales, one per sblk x sblk tile (128 or 32) in [rows / sblk][K / sblk]
+  const float* s2a;      // NVFP4 weights: scale_2 [E] of the gate (or down) projection
+  const float* s2b;      //    and of the up projection
+  const float* fac;      // NVFP4 weights: per sorted row, the factor of its token scales
   alignas(64) CUtensorMap ta, tb;  // MXFP4: 16 x 4-bit -> 16-byte slots; FP8: bytes; box {128, 256}, 128B swizzle
 };
 
@@ -291,19 +381,23 @@ __device__ __forceinline__ void gmx_tile(const TileList& L, int MB, int t, int& 
 // modes).  FP4: both operands packed e2m1 (QK_ACT_MXFP4), kind::mxf4 with a
 // reduction step of 256 elements (the weights copied as stored, 32 KB per
 // stage), two token scale atoms per step and two steps per weight-scale
-// chunk; otherwise kind::mxf8f6f4 with steps of 128.
-template <bool GATEUP, int NT, bool FP4>
+// chunk; otherwise kind::mxf8f6f4 with steps of 128.  NV (with FP4): NVFP4
+// weights, kind::mxf4nvf4 with ue4m3 scales per 16: four token and eight
+// weight scale atoms per step (one per instruction and 128 rows), one step
+// per weight-scale chunk, and the epilogue applies scale_2 and the row factor.
+template <bool GATEUP, int NT, bool FP4, bool NV = false>
 __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ GmxArgs G) {
   static_assert(!FP4 || NT == 1, "the fp4 x fp4 tiles hold one term");
+  static_assert(!NV || FP4, "NVFP4 weights run fp4 x fp4 only");
   constexpr int NPQ = NT == 1 ? 32 : NT == 2 ? kXTok1 / 4 : kXTok2 / 4;  // tokens per TMEM lane quadrant
-  constexpr int AT = FP4 ? 2 : 1;    // token scale atoms per step
-  constexpr int SPC = FP4 ? 2 : 4;   // steps per weight-scale chunk (16 bytes of each row: 512 elements)
+  constexpr int AT = NV ? 4 : FP4 ? 2 : 1;   // token scale atoms per step
+  constexpr int SPC = NV ? 1 : FP4 ? 2 : 4;  // steps per weight-scale chunk (16 bytes of each row)
   extern __shared__ __align__(16) uint8_t smem_raw[];  // rounded up to 1024 below, at run time
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sW = base;                                  // kXWS weight stages
   uint8_t* sT = sW + kXWS * kXStageW;                  // kXTS token stages
-  uint8_t* sTa = sT + kXTS * kXStageT;                 // kXTS x 4 token scale atoms (2 steps x AT)
-  uint8_t* sSa = sTa + kXTS * 4 * kSfAtom;             // kXSS x 8 weight scale atoms
+  uint8_t* sTa = sT + kXTS * kXStageT;                 // kXTS x kXTSa token scale atoms (2 steps x AT)
+  uint8_t* sSa = sTa + kXTS * kXTSa * kSfAtom;         // kXSS x 8 weight scale atoms
   GmxHead& S = *reinterpret_cast<GmxHead*>(sSa + kXSS * 8 * kSfAtom);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const TileList& L = G.L;
@@ -396,7 +490,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
     // tile scales are expanded to the same per-32 bytes: a 128 x 128 tile's
     // code serves its rows' four blocks of each step, a 32 x 32 tile's code
     // one block of 32 rows.
-    const int srow = G.K / 32;  // MXFP4 scale bytes per weight row
+    const int srow = G.K / (NV ? 16 : 32);  // MXFP4 (NVFP4) scale bytes per weight row
     // the 16 bytes of chunk `chunk` (4 steps) of rows lane + 32 j of tile t
     auto fetch = [&](int t, int chunk, uint4 (&r)[8]) {
       int f, mb;
@@ -433,10 +527,11 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
         const int tn = c + 1 < KS / SPC ? t : t + (int)gridDim.x;
         if (tn < n_tiles) fetch(tn, tn == t ? c + 1 : 0, nxt);
         uint32_t ff = 0;
+        const uint32_t nm = NV ? 0x80808080u : 0u;  // e4m3 NaN: 0x7F and 0xFF; e8m0 NaN: 0xFF
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          ff |= __vcmpeq4(cur[j].x, 0xFFFFFFFFu) | __vcmpeq4(cur[j].y, 0xFFFFFFFFu) |
-                __vcmpeq4(cur[j].z, 0xFFFFFFFFu) | __vcmpeq4(cur[j].w, 0xFFFFFFFFu);
+          ff |= __vcmpeq4(cur[j].x | nm, 0xFFFFFFFFu) | __vcmpeq4(cur[j].y | nm, 0xFFFFFFFFu) |
+                __vcmpeq4(cur[j].z | nm, 0xFFFFFFFFu) | __vcmpeq4(cur[j].w | nm, 0xFFFFFFFFu);
         if (ff) set_status(QK_ERR_NAN_SCALE);
         const int s = n % kXSS;
         if (n >= kXSS && !__all_sync(0xffffffffu, wait(&S.sempty[s], (uint32_t)((n / kXSS - 1) & 1)))) {
@@ -475,7 +570,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
           mbar_arrive_expect_tx(&S.tfull[s], (uint32_t)(kXStageT + 2 * AT * kSfAtom));
           const size_t blk = (size_t)f * KS + k0;
           bulk_g2s(sT + s * kXStageT, G.blocks + blk * kXBlock, (uint32_t)kXStageT, &S.tfull[s]);
-          bulk_g2s(sTa + s * 4 * kSfAtom, G.atoms + blk * AT * kSfAtom, (uint32_t)(2 * AT * kSfAtom), &S.tfull[s]);
+          bulk_g2s(sTa + s * kXTSa * kSfAtom, G.atoms + blk * AT * kSfAtom, (uint32_t)(2 * AT * kSfAtom), &S.tfull[s]);
         }
       }
       for (int q = n > kXTS ? n - kXTS : 0; q < n; ++q)
@@ -488,7 +583,8 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
       const uint32_t t_sfa = tmem + kXSfaCol, t_sfb = t_sfa + 4 * AT;
       // A e4m3 (token terms); B e2m1 (MXFP4 weights) or e4m3 (FP8 weights);
       // FP4: both e2m1 (format 1 of kind::mxf4)
-      const uint32_t idesc = FP4 ? umma_idesc_mx(128, kWN, 1, 1) : umma_idesc_mx(128, kWN, 0, G.wfp8 ? 0 : 5);
+      const uint32_t idesc = NV ? umma_idesc_nv(128, kWN)
+                             : FP4 ? umma_idesc_mx(128, kWN, 1, 1) : umma_idesc_mx(128, kWN, 0, G.wfp8 ? 0 : 5);
       int nw = 0, nt = 0, nc = 0, i = 0;
       for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x, ++i) {
         if (i >= 1 && !wait(&S.acc_empty, (uint32_t)((i - 1) & 1))) break;
@@ -506,13 +602,26 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
           const uint64_t da = umma_desc_k_sw128(sT + st * kXStageT + j * kXBlock);
           const uint64_t db = umma_desc_k_sw128(sW + sw * kXStageW);
           if (!FP4) {
-            utccp_32x128b_x4(t_sfa, umma_desc_sf(sTa + (st * 4 + j) * kSfAtom));
+            utccp_32x128b_x4(t_sfa, umma_desc_sf(sTa + (st * kXTSa + j) * kSfAtom));
             utccp_32x128b_x4(t_sfb, umma_desc_sf(sSa + (sc * 8 + q * 2) * kSfAtom));
             utccp_32x128b_x4(t_sfb + 4, umma_desc_sf(sSa + (sc * 8 + q * 2 + 1) * kSfAtom));
 #pragma unroll
             for (int kb = 0; kb < kXK / 32; ++kb)
               umma_mx(tmem, da + 2 * kb, db + 2 * kb, umma_idesc_sf_ids(idesc, kb, kb), t_sfa | ((uint32_t)kb << 30),
                       t_sfb | ((uint32_t)kb << 30), (ks | kb) != 0 ? 1u : 0u);
+          } else if (NV) {
+            // instruction kk (K = 64: blocks 4 kk .. 4 kk + 3 of 16): token atom
+            // kk of the step at t_sfa + 4 kk, weight atoms (rows 0-127,
+            // 128-255) at t_sfb + 8 kk and + 4; all four bytes of the column
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              utccp_32x128b_x4(t_sfa + 4 * kk, umma_desc_sf(sTa + (st * kXTSa + j * 4 + kk) * kSfAtom));
+              utccp_32x128b_x4(t_sfb + 8 * kk, umma_desc_sf(sSa + (sc * 8 + kk * 2) * kSfAtom));
+              utccp_32x128b_x4(t_sfb + 8 * kk + 4, umma_desc_sf(sSa + (sc * 8 + kk * 2 + 1) * kSfAtom));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_nvf4(tmem, da + 2 * kk, db + 2 * kk, idesc, t_sfa + 4 * kk, t_sfb + 8 * kk, (ks | kk) != 0 ? 1u : 0u);
           } else {
             // blocks 0-3 and 4-7 of the step: token atoms in columns t_sfa and
             // t_sfa + 4, weight atoms (rows 0-127, 128-255) at t_sfb + 8 g and
@@ -520,7 +629,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
             // pair 2 (k % 2)
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
-              utccp_32x128b_x4(t_sfa + 4 * g, umma_desc_sf(sTa + (st * 4 + j * 2 + g) * kSfAtom));
+              utccp_32x128b_x4(t_sfa + 4 * g, umma_desc_sf(sTa + (st * kXTSa + j * 2 + g) * kSfAtom));
               utccp_32x128b_x4(t_sfb + 8 * g, umma_desc_sf(sSa + (sc * 8 + (2 * q + g) * 2) * kSfAtom));
               utccp_32x128b_x4(t_sfb + 8 * g + 4, umma_desc_sf(sSa + (sc * 8 + (2 * q + g) * 2 + 1) * kSfAtom));
             }
@@ -564,6 +673,8 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
       const int tok = NPQ * quad + lane;
       const bool st = lane < NPQ && tok < nrow;
       float* out = G.out + (size_t)(row0 + (st ? tok : 0)) * G.out_ld + mb * kWN + half * 128;
+      float mul = 1.f;  // NVFP4: scale_2 of the tile's expert and projection, times the row's factor
+      if (NV && st) mul = __ldg((mb >= G.MBA ? G.s2b : G.s2a) + L.tile_e[f]) * __ldg(G.fac + row0 + tok);
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * 128);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -582,6 +693,10 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
             if (NT == 3) a += __shfl_down_sync(0xffffffffu, __uint_as_float(v[jj]), 2 * NPQ);
             v[jj] = __float_as_uint(a);
           }
+        }
+        if (NV) {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * mul);
         }
         if (st) {
           float4* o4 = reinterpret_cast<float4*>(out + c * 32);
@@ -613,6 +728,15 @@ bool gmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& d
          al(down.scales, 16);
 }
 
+bool gmx_nv_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I) {
+  auto al = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
+  if (gate.fmt != QK_FMT_NVFP4 || up.fmt != QK_FMT_NVFP4 || down.fmt != QK_FMT_NVFP4) return false;
+  if (!gate.scale_2 || !up.scale_2 || !down.scale_2) return false;
+  if (H % 512 != 0 || I % 512 != 0) return false;  // 16-byte scale chunks per row (one step of 256), 256-row blocks
+  return al(gate.q, 32) && al(up.q, 32) && al(down.q, 32) && al(gate.scales, 16) && al(up.scales, 16) &&
+         al(down.scales, 16);
+}
+
 // Packed e2m1 rows [rows][K / 2]: 16 codes (8 bytes) per 16-byte slot in
 // shared memory, boxes {128 codes, 256 rows}, 128-byte swizzle.  A box reads
 // 64 bytes of each row; 256-byte L2 promotion brings the row's next three
@@ -635,11 +759,11 @@ static bool x_map_fp8(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
-template <bool GATEUP, int NT, bool FP4 = false>
+template <bool GATEUP, int NT, bool FP4 = false, bool NV = false>
 static qk_status x_launch(const GmxArgs& A, cudaStream_t st) {
   static_assert(sizeof(GmxHead) <= 256, "head");
   if (kXSmem > max_smem_optin()) return QK_ERR_UNSUPPORTED;
-  return launch_ex(k_gmx<GATEUP, NT, FP4>, dim3(num_sms()), dim3(kXThreads), (size_t)kXSmem, st, false, A);
+  return launch_ex(k_gmx<GATEUP, NT, FP4, NV>, dim3(num_sms()), dim3(kXThreads), (size_t)kXSmem, st, false, A);
 }
 
 // Packed e2m1 rows [rows][K / 2] as bytes, boxes {128 bytes (256 codes), 256
@@ -659,7 +783,8 @@ qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st) {
 qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, cudaStream_t st) {
   const int T = a.T, k = a.k, E = a.E, H = a.H, I = a.I;
   const bool fp4 = act_quant == QK_ACT_MXFP4, one = act_quant != QK_ACT_NONE;
-  k_gmx_xsplit<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H, act_quant);
+  const bool nv = fp4 && a.gate.fmt == QK_FMT_NVFP4;  // an all-NVFP4 layer (gmx_nv_eligible): kind::mxf4nvf4
+  k_gmx_xsplit<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H, act_quant, nv ? 1 : 0);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
   auto wmap = [&](CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
     return fp4 ? x_map_packed(m, q, rows, K) : x_map_weights(m, q, rows, K);
@@ -677,11 +802,17 @@ qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, 
   g1.MB = 2 * I / kWN;  // gate blocks, then up blocks
   g1.MBA = I / kWN;
   g1.out_ld = 2 * I;
+  g1.s2a = a.gate.scale_2;
+  g1.s2b = a.up.scale_2;
+  g1.fac = W.fac1;
   if (!wmap(&g1.ta, a.gate.q, (int64_t)E * I, H) || !wmap(&g1.tb, a.up.q, (int64_t)E * I, H)) return QK_ERR_CUDA;
-  qk_status rc = fp4 ? x_launch<true, 1, true>(g1, st) : one ? x_launch<true, 1>(g1, st) : x_launch<true, 2>(g1, st);
+  qk_status rc = nv    ? x_launch<true, 1, true, true>(g1, st)
+                 : fp4 ? x_launch<true, 1, true>(g1, st)
+                 : one ? x_launch<true, 1>(g1, st)
+                       : x_launch<true, 2>(g1, st);
   if (rc != QK_OK) return rc;
 
-  k_gmx_hsplit<<<a.P, kRowThreads, 0, st>>>(W, E, I, act_quant);
+  k_gmx_hsplit<<<a.P, kRowThreads, 0, st>>>(W, E, I, act_quant, nv ? 1 : 0);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
 
   GmxArgs g2 = {};
@@ -696,9 +827,15 @@ qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, 
   g2.MB = H / kWN;
   g2.MBA = H / kWN;
   g2.out_ld = H;
+  g2.s2a = a.down.scale_2;
+  g2.s2b = a.down.scale_2;
+  g2.fac = W.fac2;
   if (!wmap(&g2.ta, a.down.q, (int64_t)E * H, I)) return QK_ERR_CUDA;
   g2.tb = g2.ta;
-  return fp4 ? x_launch<false, 1, true>(g2, st) : one ? x_launch<false, 1>(g2, st) : x_launch<false, 3>(g2, st);
+  return nv    ? x_launch<false, 1, true, true>(g2, st)
+         : fp4 ? x_launch<false, 1, true>(g2, st)
+         : one ? x_launch<false, 1>(g2, st)
+               : x_launch<false, 3>(g2, st);
 }
 
 // The FP8 SwiGLU FFN of a shared expert at large M on the same kernels: the M
@@ -709,7 +846,7 @@ qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, 
 qk_status gmx_fp8_ffn(const GroupWs& W, const uint16_t* x, const int32_t* ids, int M, int H, int I,
                       const uint8_t* wg, const uint8_t* sg, const uint8_t* wu, const uint8_t* su,
                       const uint8_t* wd, const uint8_t* sd, int blk, cudaStream_t st) {
-  k_gmx_xsplit<<<M, kRowThreads, 0, st>>>(W, x, ids, 1, 1, H, QK_ACT_NONE);
+  k_gmx_xsplit<<<M, kRowThreads, 0, st>>>(W, x, ids, 1, 1, H, QK_ACT_NONE, 0);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
   GmxArgs g1 = {};
   g1.L = W.L1;
@@ -728,7 +865,7 @@ qk_status gmx_fp8_ffn(const GroupWs& W, const uint16_t* x, const int32_t* ids, i
   if (!x_map_fp8(&g1.ta, wg, I, H) || !x_map_fp8(&g1.tb, wu, I, H)) return QK_ERR_CUDA;
   qk_status rc = x_launch<true, 2>(g1, st);
   if (rc != QK_OK) return rc;
-  k_gmx_hsplit<<<M, kRowThreads, 0, st>>>(W, 1, I, QK_ACT_NONE);
+  k_gmx_hsplit<<<M, kRowThreads, 0, st>>>(W, 1, I, QK_ACT_NONE, 0);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
   GmxArgs g2 = {};
   g2.L = W.L2;

@@ -646,12 +646,17 @@ struct GWsLayout {
   size_t counts, n_tiles1, n_tiles2, n_flush, zero_end, offsets, fill, inv, dperm;
   size_t t1[5], t2[5], exp1, exp2;  // tile_e, tile_row0, tile_n, tile_first, tile_cnt
   size_t xshift, hshift, xperm, hperm, h16;
-  size_t rtile2, xt, sfx, gu, ht, sfh, total;
+  size_t rtile2, xt, sfx, gu, ht, sfh, fac1, fac2, total;
 };
 
-// Workspace of the grouped path; `mx` selects the MXFP4 block-scaled buffers
-// instead of the f16 ones.
-static GWsLayout g_layout(int T, int k, int E, int H, int I, bool mx) {
+enum { kWsF16 = 0, kWsMx = 1, kWsNv = 2 };
+
+// Workspace of the grouped path: the f16 buffers, the MXFP4 block-scaled
+// ones, or (NVFP4 layers in QK_ACT_MXFP4) those with twice the token scale
+// atoms and the per-row factors.
+static GWsLayout g_layout(int T, int k, int E, int H, int I, int kind) {
+  const bool mx = kind != kWsF16;
+  const size_t sf_mul = kind == kWsNv ? 2 : 1;
   const size_t P = (size_t)T * k;
   const size_t F1 = (size_t)g_max_tiles((int)P, E, mx ? kXTok1 : kGN), F2 = (size_t)g_max_tiles((int)P, E, kXTok2);
   GWsLayout L = {};
@@ -673,10 +678,14 @@ static GWsLayout g_layout(int T, int k, int E, int H, int I, bool mx) {
     L.exp2 = o; o += align256((size_t)E * 4);
     L.rtile2 = o; o += align256(P * 4);
     L.xt = o; o += align256(F1 * (H / kXK) * kXBlock);
-    L.sfx = o; o += align256(F1 * (H / kXK) * kSfAtom);
+    L.sfx = o; o += align256(F1 * (H / kXK) * kSfAtom * sf_mul);
     L.gu = o; o += align256(P * 2 * I * 4);
     L.ht = o; o += align256(F2 * (I / kXK) * kXBlock);
-    L.sfh = o; o += align256(F2 * (I / kXK) * kSfAtom);
+    L.sfh = o; o += align256(F2 * (I / kXK) * kSfAtom * sf_mul);
+    if (kind == kWsNv) {
+      L.fac1 = o; o += align256(P * 4);
+      L.fac2 = o; o += align256(P * 4);
+    }
   } else {
     L.xshift = o; o += align256(P * 4);
     L.hshift = o; o += align256(P * 4);
@@ -691,7 +700,15 @@ static GWsLayout g_layout(int T, int k, int E, int H, int I, bool mx) {
 static bool g_mx(const qk_moe_layer* L) { return gmx_eligible(L->gate, L->up, L->down, L->hidden, L->inter); }
 
 size_t group_workspace_bytes(const qk_moe_layer* L, int T, int k) {
-  return g_layout(T, k, L->gate.n_experts, L->hidden, L->inter, g_mx(L)).total;
+  return g_layout(T, k, L->gate.n_experts, L->hidden, L->inter, g_mx(L) ? kWsMx : kWsF16).total;
+}
+
+size_t group_workspace_bytes_act(const qk_moe_layer* L, int T, int k, int act_quant) {
+  if (act_quant != QK_ACT_MXFP4 && act_quant != QK_ACT_E4M3) return 0;
+  if (g_mx(L)) return g_layout(T, k, L->gate.n_experts, L->hidden, L->inter, kWsMx).total;
+  if (act_quant == QK_ACT_MXFP4 && gmx_nv_eligible(L->gate, L->up, L->down, L->hidden, L->inter))
+    return g_layout(T, k, L->gate.n_experts, L->hidden, L->inter, kWsNv).total;
+  return 0;
 }
 
 static TileList g_list(uint8_t* p, const size_t (&t)[5], size_t exp, size_t n_tiles, bool mx) {
@@ -708,8 +725,9 @@ static TileList g_list(uint8_t* p, const size_t (&t)[5], size_t exp, size_t n_ti
   return L;
 }
 
-static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I, bool mx) {
-  const GWsLayout L = g_layout(T, k, E, H, I, mx);
+static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I, int kind) {
+  const bool mx = kind != kWsF16;
+  const GWsLayout L = g_layout(T, k, E, H, I, kind);
   uint8_t* p = static_cast<uint8_t*>(ws);
   GroupWs W = {};
   W.counts = reinterpret_cast<int*>(p + L.counts);
@@ -728,6 +746,10 @@ static GroupWs g_carve(void* ws, int T, int k, int E, int H, int I, bool mx) {
     W.gu = reinterpret_cast<float*>(p + L.gu);
     W.ht = p + L.ht;
     W.sfh = p + L.sfh;
+    if (kind == kWsNv) {
+      W.fac1 = reinterpret_cast<float*>(p + L.fac1);
+      W.fac2 = reinterpret_cast<float*>(p + L.fac2);
+    }
   } else {
     W.xshift = reinterpret_cast<int*>(p + L.xshift);
     W.hshift = reinterpret_cast<int*>(p + L.hshift);
@@ -783,9 +805,10 @@ qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
 // caller checks eligibility).
 qk_status group_forward_act(const DecodeArgs& a, int act_quant, void* workspace, cudaStream_t st) {
   const int T = a.T, k = a.k, E = a.E, H = a.H, I = a.I, P = a.P;
-  const bool mx = gmx_eligible(a.gate, a.up, a.down, H, I);
+  const bool nv = act_quant == QK_ACT_MXFP4 && gmx_nv_eligible(a.gate, a.up, a.down, H, I);
+  const bool mx = gmx_eligible(a.gate, a.up, a.down, H, I) || nv;  // the block-scaled grouped kernels
   if (act_quant != QK_ACT_NONE && !mx) return QK_ERR_UNSUPPORTED;
-  GroupWs W = g_carve(workspace, T, k, E, H, I, mx);
+  GroupWs W = g_carve(workspace, T, k, E, H, I, nv ? kWsNv : mx ? kWsMx : kWsF16);
   if (cudaMemsetAsync(W.counts, 0, W.zero_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
   k_grp_count<<<(P + 255) / 256, 256, 0, st>>>(a.ids, P, E, W.counts);
   k_grp_scan<<<1, kScanThreads, 0, st>>>(W, W.L1, E, mx ? gmx_tok1(act_quant) : kGN, mx ? 1 : 0, 1);
@@ -845,16 +868,16 @@ __global__ void k_fp8_route_all(int32_t* ids, float* w, int M) {
 }
 
 size_t fp8_group_workspace_bytes(int M, int H, int I) {
-  return g_layout(M, 1, 1, H, I, true).total + 2 * align256((size_t)M * 4);
+  return g_layout(M, 1, 1, H, I, kWsMx).total + 2 * align256((size_t)M * 4);
 }
 
 qk_status fp8_group_forward(const void* x, int M, int H, int I, const uint8_t* wg, const uint8_t* sg,
                             const uint8_t* wu, const uint8_t* su, const uint8_t* wd, const uint8_t* sd, int blk,
                             float* y, void* workspace, cudaStream_t st) {
-  const size_t base = g_layout(M, 1, 1, H, I, true).total;
+  const size_t base = g_layout(M, 1, 1, H, I, kWsMx).total;
   int32_t* ids = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + base);
   float* w = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + base + align256((size_t)M * 4));
-  GroupWs W = g_carve(workspace, M, 1, 1, H, I, true);
+  GroupWs W = g_carve(workspace, M, 1, 1, H, I, kWsMx);
   if (cudaMemsetAsync(W.counts, 0, W.zero_bytes, st) != cudaSuccess) return QK_ERR_CUDA;
   k_fp8_route_all<<<(M + 255) / 256, 256, 0, st>>>(ids, w, M);
   k_grp_count<<<(M + 255) / 256, 256, 0, st>>>(ids, M, 1, W.counts);

@@ -54,12 +54,20 @@ struct GroupWs {
   float* gu;        // [P][2 I] fp32 gate (first I) and up (last I) projections
   uint8_t* ht;      // [F2][I / 128] blocks of the 3 e4m3 terms of h = silu(gate) * up
   uint8_t* sfh;     // [F2][I / 128][512] ue8m0 scales of the h terms, atom layout
+  // NVFP4 layers in QK_ACT_MXFP4 (kind::mxf4nvf4): the token scales are ue4m3
+  // per 16 (twice the atoms of the MXFP4 tiles), re-anchored per row; the row's
+  // factor 2^(cmax - 135) restores them in the epilogue.
+  float* fac1;      // [P] per sorted row: x scale factor
+  float* fac2;      // [P] per sorted row: h scale factor
 };
 
 // The MXFP4 block-scaled path takes a layer when all three projections are
 // MXFP4, hidden and inter are multiples of 512 and the packed weights (32 B)
 // and scales (16 B) are aligned for its copies.
 bool gmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
+// The same kernels take an all-NVFP4 layer in QK_ACT_MXFP4 (fp4 x fp4 on
+// kind::mxf4nvf4, ue4m3 block scales per 16): same shape and alignment rules.
+bool gmx_nv_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);
 // The FP8 shared expert's two GEMMs on the block-scaled grouped kernels.
 qk_status gmx_fp8_ffn(const GroupWs& W, const uint16_t* x, const int32_t* ids, int M, int H, int I,
                       const uint8_t* wg, const uint8_t* sg, const uint8_t* wu, const uint8_t* su,

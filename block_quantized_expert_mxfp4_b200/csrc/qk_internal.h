@@ -40,6 +40,8 @@ struct DecodeArgs {
 qk_status decode_forward(DecodeArgs args, cudaStream_t st);
 // Grouped (prefill) path: pairs grouped by expert, tcgen05 grouped GEMMs.
 size_t group_workspace_bytes(const qk_moe_layer* L, int T, int k);
+// The same with an activation mode (QK_ACT_E4M3 / QK_ACT_MXFP4): 0 if refused.
+size_t group_workspace_bytes_act(const qk_moe_layer* L, int T, int k, int act_quant);
 qk_status group_forward(const DecodeArgs& a, void* workspace, cudaStream_t st);
 // Decode path for all-MXFP4 layers on the block-scaled tensor cores.
 bool dmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& down, int H, int I);

@@ -131,13 +131,16 @@ def act_quant_alternatives(h32, hq, aq, eps):
 
 
 def _down_columns(layer, e, idx):
-    """Columns idx of expert e's dequantized down matrix (MXFP4), decoded
-    with the library tables of ml_dtypes: [hidden][len(idx)]."""
-    from ref_decode import E2M1, E8M0
+    """Columns idx of expert e's dequantized down matrix (MXFP4, or NVFP4
+    with its scale_2), decoded with the library tables of ml_dtypes:
+    [hidden][len(idx)]."""
+    from ref_decode import E2M1, E4M3, E8M0
     d = layer.down
-    assert d.fmt == MX
     byte = d.q[e][:, idx // 2]
     code = np.where(idx % 2 == 1, byte >> 4, byte & 0x0F)
+    if d.fmt == NV:
+        return E2M1[code] * E4M3[d.scales[e][:, idx // 16]] * float(d.scale_2[e])
+    assert d.fmt == MX
     return E2M1[code] * E8M0[d.scales[e][:, idx // 32]]
 
 

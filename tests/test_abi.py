@@ -78,16 +78,25 @@ def test_workspace_query_follows_the_path_choice():
 def test_workspace_query_with_activation_modes():
     """The quantized modes run the grouped block-scaled kernels at every token
     count: their workspace is the grouped one (the bf16 query's size above one
-    decode launch), and 0 where the mode is refused."""
+    decode launch), and 0 where the mode is refused.  An all-NVFP4 layer runs
+    QK_ACT_MXFP4 on kind::mxf4nvf4 (twice the token scale atoms and two
+    per-row factor arrays beyond the MXFP4 layout); W4A8 has no NVFP4 form."""
     L = qk.load()
     q = lambda lay, T, aq: L.moe_expert_workspace_size(ctypes.byref(lay), T, 6, aq)
     mx, nv, mis = _fake_layer(), _fake_layer(fmts=(2, 2, 2)), _fake_layer()
     mis.gate.q = mis.gate.q + 16
+    mixed = _fake_layer(fmts=(1, 2, 1))
     for aq in (qk.QK_ACT_MXFP4, qk.QK_ACT_E4M3):
         assert q(mx, 100, aq) == q(mx, 100, qk.QK_ACT_NONE) > 0
         assert q(mx, 1, aq) > 0 and q(mx, 1, aq) != q(mx, 1, qk.QK_ACT_NONE)
         assert q(mx, 1, aq) < q(mx, 16, aq) < q(mx, 100, aq)
-        assert q(nv, 1, aq) == 0 and q(mis, 1, aq) == 0
+        assert q(mis, 1, aq) == 0 and q(mixed, 1, aq) == 0
+    assert q(nv, 1, qk.QK_ACT_E4M3) == 0
+    for T in (1, 16, 100):
+        assert q(nv, T, qk.QK_ACT_MXFP4) > q(mx, T, qk.QK_ACT_MXFP4)
+    nvmis = _fake_layer(fmts=(2, 2, 2))
+    nvmis.down.scales = nvmis.down.scales + 8
+    assert q(nvmis, 1, qk.QK_ACT_MXFP4) == 0
     assert q(mx, 1, 7) == 0
 
 
@@ -117,10 +126,12 @@ def test_forward_argument_errors_are_synchronous():
     assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 7, p, ws, None) == qk.QK_ERR_INVALID_ARG  # mode
     nv = _fake_layer(fmts=(2, 2, 2))
     for aq in (qk.QK_ACT_MXFP4, qk.QK_ACT_E4M3):
-        # a quantized mode: NVFP4 layers are refused; an all-MXFP4 layer runs
-        # the grouped kernels, whose workspace the bf16-path size does not cover
-        assert f(ctypes.byref(nv), p, 1, p, p, 6, p, 0, aq, p, 1 << 30, None) == qk.QK_ERR_UNSUPPORTED
+        # a quantized mode: an all-MXFP4 layer runs the grouped kernels, whose
+        # workspace the bf16-path size does not cover; NVFP4 layers likewise in
+        # QK_ACT_MXFP4, and are refused in QK_ACT_E4M3
         assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, aq, p, ws, None) == qk.QK_ERR_WORKSPACE
+        want = qk.QK_ERR_WORKSPACE if aq == qk.QK_ACT_MXFP4 else qk.QK_ERR_UNSUPPORTED
+        assert f(ctypes.byref(nv), p, 1, p, p, 6, p, 0, aq, p, 1024, None) == want
     assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 0, p, ws - 1, None) == qk.QK_ERR_WORKSPACE
     assert f(ctypes.byref(lay), p, 1, p, p, 6, p, 0, 0, None, ws, None) == qk.QK_ERR_WORKSPACE
     assert f(ctypes.byref(lay), None, 1, p, p, 6, p, 0, 0, p, ws, None) == qk.QK_ERR_INVALID_ARG

@@ -14,7 +14,7 @@ import torch
 import block_quantized_expert_mxfp4_b200 as qk
 import oracle
 from block_quantized_expert_mxfp4_b200 import synth, workload
-from helpers import assert_parity_act_quant, oracle_sublayer
+from helpers import MX, NV, assert_parity_act_quant, oracle_sublayer
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +33,7 @@ def _forward(layer, x, ids, w, aq):
     return y.cpu().numpy()
 
 
-def _check(wl, seed, x, oids, ow, y, aq, what):
+def _check(wl, seed, x, oids, ow, y, aq, what, fmts=(MX, MX, MX), nv_codes=None):
     """Parity in the mode, and a bound on the h codes taken from the other
     side of a decision boundary: an h value lies within the helper's relative
     window (2^-13) of a midpoint for well under 1 % of the codes (e4m3 steps
@@ -41,7 +41,7 @@ def _check(wl, seed, x, oids, ow, y, aq, what):
     rounding."""
     experts = sorted(set(int(e) for e in oids.reshape(-1)))
     remap = {e: i for i, e in enumerate(experts)}
-    L = oracle_sublayer(wl, seed, 0, experts)
+    L = oracle_sublayer(wl, seed, 0, experts, fmts, nv_codes)
     sub = np.vectorize(remap.get)(oids).astype(np.int32)
     e, c, used, offered = assert_parity_act_quant(y, L, x, sub, ow.astype(np.float32).astype(np.float64), aq,
                                                   what=what)
@@ -120,6 +120,48 @@ def test_w4a4_prefill_zipf_sampled_tokens():
     pick = sorted(pick)
     _check(wl, 26, x[pick], oids[pick], ow[pick], y[pick], qk.QK_ACT_MXFP4,
            f"w4a4 prefill: {len(pick)} tokens covering every expert")
+
+
+# NVFP4 layers in QK_ACT_MXFP4 run fp4 x fp4 on kind::mxf4nvf4: converted
+# from MXFP4 (power-of-two block scales and scale_2), and general (any e4m3
+# block scale, scale_2 not a power of two).
+NV_SOURCES = [None, (synth.NV_CODE_LO, synth.NV_CODE_HI)]
+
+
+@pytest.mark.parametrize("codes", NV_SOURCES, ids=["converted", "general"])
+@pytest.mark.parametrize("T", [1, 48])
+def test_nvfp4_w4a4_mxf4nvf4(codes, T):
+    """48 tokens (or 1) x top-4 over 16 experts, hidden 1024, intermediate 512,
+    all three projections NVFP4."""
+    wl = synth.Workload("mid", 16, 4, 1024, 512, T, 118, 127)
+    layer = workload.make_layer(wl, 31, 0, (NV, NV, NV), nv_codes=codes)
+    x = synth.activations(31, T, wl.H)
+    oids, ow = oracle.route_topk(synth.router_logits(31, T, wl.E), wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda(),
+                 qk.QK_ACT_MXFP4)
+    _check(wl, 31, x, oids, ow, y, qk.QK_ACT_MXFP4, f"nvfp4 w4a4 T={T} {'general' if codes else 'converted'}",
+           (NV, NV, NV), codes)
+
+
+def test_nvfp4_w4a4_decode_layer():
+    """The decode MoE layer in NVFP4 (256 experts, top-6, hidden 4096,
+    intermediate 2048, converted from the seeded MXFP4 layer) at 4 tokens."""
+    wl = synth.WORKLOADS["decode_mx"]
+    layer = workload.make_layer(wl, 32, 0, (NV, NV, NV))
+    x = synth.activations(32, 4, wl.H)
+    oids, ow = oracle.route_topk(synth.router_logits(32, 4, wl.E), wl.k)
+    y = _forward(layer, x.cuda(), torch.from_numpy(oids).cuda(), torch.from_numpy(ow).float().cuda(),
+                 qk.QK_ACT_MXFP4)
+    _check(wl, 32, x, oids, ow, y, qk.QK_ACT_MXFP4, "nvfp4 w4a4 decode layer T=4", (NV, NV, NV))
+
+
+def test_nvfp4_w4a8_refused():
+    """W4A8 has no NVFP4 form on sm_100a: kind::mxf8f6f4 takes ue8m0 scales
+    only, so an NVFP4 layer in QK_ACT_E4M3 is refused (workspace 0)."""
+    wl = synth.Workload("mid", 16, 4, 1024, 512, 4, 118, 127)
+    lay = workload.make_layer(wl, 33, 0, (NV, NV, NV)).c()
+    assert qk.moe_expert_workspace_size(lay, 4, 4, qk.QK_ACT_E4M3) == 0
+    assert qk.moe_expert_workspace_size(lay, 4, 4, qk.QK_ACT_MXFP4) > 0
 
 
 @pytest.mark.parametrize("aq", MODES)
