@@ -390,9 +390,12 @@ def run_ours(args, rank, world, local_rank):
         out["prefill_w4a8"] = run_prefill(args, rank, world, dev, act="e4m3", steps=10)
         out["prefill_w4a4"] = run_prefill(args, rank, world, dev, act="mxfp4", steps=10)
         out["prefill_w4a4_16k"] = run_prefill(args, rank, world, dev, tokens=16384, act="mxfp4", steps=3)
+        out["prefill_w4a4_nvfp4"] = run_prefill(args, rank, world, dev, act="mxfp4", steps=10, nv=True)
+        out["prefill_w4a4_nvfp4_16k"] = run_prefill(args, rank, world, dev, tokens=16384, act="mxfp4", steps=3,
+                                                    nv=True)
         out["shared_fp8_prefill"] = run_shared_fp8(args, rank, world, dev)
         for key in ("decode_nvfp4", "stack43", "prefill_16k", "prefill_w4a8", "prefill_w4a4", "prefill_w4a4_16k",
-                    "shared_fp8_prefill"):
+                    "prefill_w4a4_nvfp4", "prefill_w4a4_nvfp4_16k", "shared_fp8_prefill"):
             out["gpu_launches"] += out[key]["gpu_launches"]
     return out
 
@@ -581,10 +584,12 @@ def run_stack(args, rank, world, dev):
     return res
 
 
-def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0):
+def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0, nv=False):
     """The 2048-token Zipf prefill layer through moe_expert_forward (grouped
     path): tokens/s, HBM fraction on the touched experts' bytes, tensor rate.
-    `tokens`, `act` and `steps` override the command line's choices."""
+    `tokens`, `act` and `steps` override the command line's choices; `nv`
+    converts the layer to NVFP4 (scale-only conversion of the seeded MXFP4
+    layer)."""
     import torch
     import torch.distributed as dist
 
@@ -598,7 +603,8 @@ def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0):
     T, k = wl.T, wl.k
     act_name = act or args.prefill_act
     aq = {"none": qk.QK_ACT_NONE, "e4m3": qk.QK_ACT_E4M3, "mxfp4": qk.QK_ACT_MXFP4}[act_name]
-    layer = workload.make_layer(wl, seed=rank, layer=0)
+    fmts = (qk.QK_FMT_NVFP4,) * 3 if nv else None
+    layer = workload.make_layer(wl, seed=rank, layer=0, fmts=fmts)
     lay = layer.c()
     x = synth.activations(rank, T, wl.H).to(dev)
     lg = synth.zipf_logits(rank, T, wl.E, k).to(dev)
@@ -647,13 +653,16 @@ def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0):
     # FP4 (kind::mxf4, four times) is the format's own ceiling.  `flops` is the
     # layer's useful work; the activation terms multiply the MMAs issued (2 for
     # gate/up, 3 for down) but not the work.
-    if aq == qk.QK_ACT_MXFP4:  # both operands e2m1: kind::mxf4, four times the bf16 rate
-        tpeak, tkind = 4 * bf16, f"{src} bf16 x 4 (nominal fp4/bf16 ratio): the MMA kind used, kind::mxf4"
+    if aq == qk.QK_ACT_MXFP4:  # both operands e2m1: kind::mxf4 (mxf4nvf4), four times the bf16 rate
+        kind = "kind::mxf4nvf4" if nv else "kind::mxf4"
+        tpeak, tkind = 4 * bf16, f"{src} bf16 x 4 (nominal fp4/bf16 ratio): the MMA kind used, {kind}"
     else:
         tpeak, tkind = 2 * bf16, f"{src} bf16 x 2 (nominal fp8/bf16 ratio): the MMA kind used, kind::mxf8f6f4"
     return {
         "workload": f"prefill MoE layer: {T} tokens, {wl.E} experts, top-6 Zipf(s=1) routing, hidden 4096, "
-                    "intermediate 2048, MXFP4 gate/up/down, bf16 N(0,1) activations"
+                    + ("intermediate 2048, NVFP4 gate/up/down (scale-only conversion of the seeded MXFP4 layer), "
+                       if nv else "intermediate 2048, MXFP4 gate/up/down, ")
+                    + "bf16 N(0,1) activations"
                     + ("" if aq == qk.QK_ACT_NONE else f", quantized in the layer to {act_name}"
                        " (one e8m0 scale per 32)"),
         "tokens_per_s": round(T * world / t, 1), "ms_per_layer": round(t * 1e3, 4), "steps": K,
@@ -667,7 +676,9 @@ def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0):
                  "(e2m1 weights + e8m0 scales as stored): gate/up, SwiGLU + 3-term h split, down; combine")
         if aq == qk.QK_ACT_NONE else
         (f"counting sort by expert; x and h quantized to {act_name} (one term per token, 128-token tiles); "
-         + ("both operands packed e2m1, block-scaled tcgen05 kind::mxf4 grouped GEMMs (weights as stored)"
+         + ("both operands packed e2m1, block-scaled tcgen05 kind::mxf4nvf4 grouped GEMMs (e2m1 + e4m3 per 16 "
+            "as stored; activation scales as ue4m3 re-anchored per row; scale_2 in the epilogue)" if nv else
+            "both operands packed e2m1, block-scaled tcgen05 kind::mxf4 grouped GEMMs (weights as stored)"
             if aq == qk.QK_ACT_MXFP4 else "block-scaled tcgen05 kind::mxf8f6f4 grouped GEMMs")
          + "; combine"),
         "gpu_launches": 8 * K,

@@ -74,13 +74,22 @@ enum { QK_FMT_MXFP4 = 1, QK_FMT_NVFP4 = 2 };
  *                own expert numerics), x before gate/up and h before down.
  *  QK_ACT_MXFP4  the same with e2m1 activations (fp4 x fp4, run on the
  *                kind::mxf4 block-scaled tensor cores with both operands
- *                packed e2m1).
+ *                packed e2m1; NVFP4 layers on kind::mxf4nvf4, whose scales
+ *                are ue4m3 per 16: each row's e8m0 activation scales are
+ *                re-anchored as ue4m3 2^(c - cmax + 8), cmax the row's
+ *                largest, and 2^(cmax - 135) times scale_2 multiplies the
+ *                result; exact while a block's code is within 17 of cmax, a
+ *                block further below, under 2^-17 of the row's largest
+ *                values, is dropped).
  * Scale rule for both (the pages give none; OCP Microscaling v1.0): X =
  * floor(log2 max|v|) - 8 (e4m3) or - 2 (e2m1) per 32 values, clamped to the
  * e8m0 range; elements rounded to nearest even, saturating (E4M3 to 448,
  * e2m1 to 6).  The quantized modes need an all-MXFP4 layer that qualifies for
- * the block-scaled grouped kernels (see moe_expert_forward) and run on them
- * at every token count; other layers return QK_ERR_UNSUPPORTED. */
+ * the block-scaled grouped kernels (see moe_expert_forward), or for
+ * QK_ACT_MXFP4 an all-NVFP4 one with the same shape and alignment, and run
+ * on them at every token count; other layers (mixed formats, and NVFP4 in
+ * QK_ACT_E4M3: the f8f6f4 kind takes ue8m0 scales only) return
+ * QK_ERR_UNSUPPORTED. */
 enum { QK_ACT_NONE = 0, QK_ACT_MXFP4 = 1, QK_ACT_E4M3 = 2 };
 
 /* One projection of one layer, all experts.  Device pointers. */
