@@ -325,7 +325,6 @@ constexpr int kXTS = 2;                // token stages (two steps each)
 constexpr int kXStageT = 2 * kXBlock;  // 32 KB
 constexpr int kXSS = 2;                // weight-scale chunk slots (4 steps x 2 atoms each)
 constexpr int kXSfaCol = 256;          // token scales: 4 columns; weight scales: 8 columns after them
-constexpr int kXPrefetch = 8;          // weight steps prefetched into L2 ahead of the TMA ring
 constexpr int kXTmemCols = 512;
 constexpr int kXTSa = 8;               // token scale atoms per token stage (2 steps x up to 4)
 constexpr int kXSmem = 1024 + kXWS * kXStageW + kXTS * (kXStageT + kXTSa * kSfAtom) + kXSS * 8 * kSfAtom + 256;
@@ -441,9 +440,9 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
 
   if (warp == 0) {
     // ----------------------------------------------------- weight tiles --
-    // Every step also prefetches the step kXPrefetch ahead (this tile's or
-    // the next one's) into L2, so more DRAM requests are in flight than the
-    // ring's shared memory holds.
+    // Loads only: an L2 prefetch of later steps costs the SM's TMA unit as
+    // much as a load, and measured slower (the 2048-token fp4 x fp4 layer
+    // 1.13 -> 0.97 ms without it).
     if (lane == 0) {
       const uint64_t pw = policy_evict_normal();
       auto coords = [&](int t, const void*& map, int& wrow) {
@@ -454,29 +453,17 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
         wrow = L.tile_e[f] * G.rows_per_e + (b ? mb - G.MBA : mb) * kWN;
       };
       int n = 0;
-      const void* map = nullptr;
-      int wrow = 0;
-      if ((int)blockIdx.x < n_tiles) {
-        coords(blockIdx.x, map, wrow);
-        for (int ks = 0; ks < kXPrefetch && ks < KS; ++ks) tma_prefetch_2d(map, ks * kXK, wrow);
-      }
       for (int t = blockIdx.x; t < n_tiles && !aborted(); t += gridDim.x) {
-        const void* nmap = nullptr;
-        int nrow = 0;
-        const bool has_next = t + (int)gridDim.x < n_tiles;
-        if (has_next) coords(t + gridDim.x, nmap, nrow);
+        const void* map = nullptr;
+        int wrow = 0;
+        coords(t, map, wrow);
         for (int ks = 0; ks < KS; ++ks, ++n) {
-          const int pk = ks + kXPrefetch;
-          if (pk < KS) tma_prefetch_2d(map, pk * kXK, wrow);
-          else if (has_next && pk - KS < KS) tma_prefetch_2d(nmap, (pk - KS) * kXK, nrow);
           const int s = n % kXWS;
           if (n >= kXWS && !wait(&S.wempty[s], (uint32_t)((n / kXWS - 1) & 1))) break;
           // counted in global bytes: packed (4-bit) codes, or one byte per FP8 code
           mbar_arrive_expect_tx(&S.wfull[s], (uint32_t)(G.wfp8 || FP4 ? kXStageW : kXStageW / 2));
           tma_load_2d(sW + s * kXStageW, map, ks * kXK, wrow, &S.wfull[s], pw);
         }
-        map = nmap;
-        wrow = nrow;
       }
       for (int q = n > kXWS ? n - kXWS : 0; q < n; ++q)  // nothing may still be landing at exit
         if (!mbar_wait_bounded(&S.wfull[q % kXWS], (uint32_t)((q / kXWS) & 1), kDrainLimitNs)) break;
