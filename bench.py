@@ -373,7 +373,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": T * wl.H * 2 + T * wl.E * 4,
                 "d2h_bytes_per_step": T * wl.H * 4, "steps": E2},
-        "gpu_launches": 3 * K,
+        "gpu_launches": 4 * K,  # route, gate/up, down, y
         "clocks": clocks.summary(),
     }
     del layers, lays
@@ -521,7 +521,7 @@ def run_decode_nv(args, rank, world, dev):
         res["by_tokens"][str(T)] = {"us_per_call": round(t * 1e6, 3), "bytes_per_call": int(b),
                                     "achieved_gbs": round(b / t / 1e9, 1), "frac": round(b / t / 1e9 / peak, 4),
                                     "tokens_per_s": round(T * world / t, 1)}
-        launches += 20 * reps * L * 2  # gate/up and down kernels (f16 decode path) per call
+        launches += 20 * reps * L * 3  # gate/up, down and y kernels (f16 decode path) per call
     res["gpu_launches"] = launches
     res["path"] = "f16 decode kernels (k_decode: e2m1 and e4m3 scales decoded in registers, m16n8k16 MMA)"
     del layers, lays
@@ -578,7 +578,7 @@ def run_stack(args, rank, world, dev):
            "bytes_per_step": nbytes, "achieved_gbs": round(nbytes / t / 1e9, 1), "peak_gbs": peak,
            "peak_kind": peak_kind, "frac": round(nbytes / t / 1e9 / peak, 4),
            "hbm_floor_ms": round(nbytes / peak / 1e6, 4),
-           "gpu_launches": K * wl.layers * 5}  # router, routed gate/up and down, shared gate/up and down
+           "gpu_launches": K * wl.layers * 6}  # router, routed gate/up, down and y, shared gate/up and down
     del layers, lays, shared
     torch.cuda.empty_cache()
     return res

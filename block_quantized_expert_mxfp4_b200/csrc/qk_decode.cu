@@ -19,9 +19,8 @@
 // contiguously over its warps, so every warp streams about the same number of
 // bytes.  A unit cut by a warp boundary is summed in shared memory by the warp
 // holding its first chunk, adding the pieces in chunk order (deterministic for
-// a given grid).  k_down writes each unit's 16 x 8 result; the last unit of a
-// row tile to finish (a per-row-tile counter) forms y for those 16 rows in
-// fixed slot order.
+// a given grid).  k_down writes each unit's 16 x 8 result; k_decode_y, the
+// next launch, forms y in fixed slot order.
 //
 // Data path.  Each warp streams its chunks through its own ring of shared-
 // memory stages.  Packed rows arrive by tensor-map TMA as 3-D boxes of 8 or 16
@@ -461,13 +460,7 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
   const int rows_per_e = GATEUP ? a.I : a.H;  // weight rows of one expert
   const bool fast = G.fast != 0;
 
-  if (GATEUP) {
-    pdl_launch_dependents();
-    // k_down's row-tile counters start at zero; k_down touches them only after
-    // this grid has completed
-    if (blockIdx.x == 0)
-      for (int i = threadIdx.x; i < a.H / 16; i += blockDim.x) a.cnt[i] = 0u;
-  }
+  pdl_launch_dependents();  // the next kernel (k_down, then k_decode_y) may start its prologue
   if (lane == 0) {
     for (int i = 0; i < G.D; ++i) mbar_init(&full[i], 33);
     fence_mbar_init();
@@ -520,20 +513,10 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
       pc_dst[npc] = (isb ? 8 * G.sca + row * G.scb : row * G.sca) + pc * G.sc_vec;
     }
   }
-  // Unit order.  Expert-major (u = v * RT + r) in general.  k_down with every
-  // pair row staged orders its units row-tile-major (u = r * n_v + v): a
-  // block then holds every expert's unit of most of its row tiles, so the
-  // row-tile combines are spread over the blocks instead of all falling to
-  // the blocks that hold the last expert.
-  const bool rmajor = !GATEUP && fast;
+  // Unit order: expert-major (u = v * RT + r).
   auto unit_vr = [&](int u, int& v, int& r) {
-    if (rmajor) {
-      r = u / n_v;
-      v = u - r * n_v;
-    } else {
-      v = u / RT;
-      r = u - v * RT;
-    }
+    v = u / RT;
+    r = u - v * RT;
   };
   // Position of a chunk: unit u (expert slot v, row tile r), chunk kc of the unit.
   struct Cur {
@@ -550,12 +533,7 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     if (++q.kc == nk) {
       q.kc = 0;
       ++q.u;
-      if (rmajor) {
-        if (++q.v == n_v) {
-          q.v = 0;
-          ++q.r;
-        }
-      } else if (++q.r == RT) {
+      if (++q.r == RT) {
         q.r = 0;
         ++q.v;
       }
@@ -606,64 +584,6 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     }
   };
 
-  // k_down: units this warp finished whose row-tile counters are not yet bumped
-  // (lane i holds the i-th); bumped in batches so the round trips overlap.
-  int pend = -1, npend = 0;
-  auto combine = [&](int r) {  // y rows r*16 .. r*16+15 of every token
-    const float* ures = a.ures;
-    for (int idx = lane; idx < a.T * 16; idx += 32) {
-      const int tok = idx >> 4, m = idx & 15;
-      const int ln = (m & 7) * 4, el = (m >= 8) ? 2 : 0;
-      float d[8];
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {  // issue the loads of up to 8 slots together
-        d[s] = 0.f;
-        if (s < a.k) {
-          const int p = tok * a.k + s;
-          const int pv = S.R.pair_v[p];
-          if (pv >= 0) {
-            const int j = S.R.pair_j[p];
-            d[s] = __ldcg(ures + (((size_t)pv * RT + r) * 32 + ln + (j >> 1)) * 4 + el + (j & 1));
-          }
-        }
-      }
-      float yv = 0.f;
-#pragma unroll
-      for (int s = 0; s < 8; ++s)
-        if (s < a.k) yv = fmaf(a.w[tok * a.k + s], d[s], yv);
-      for (int s = 8; s < a.k; ++s) {
-        const int p = tok * a.k + s;
-        const int pv = S.R.pair_v[p];
-        if (pv < 0) continue;
-        const int j = S.R.pair_j[p];
-        yv = fmaf(a.w[p], __ldcg(ures + (((size_t)pv * RT + r) * 32 + ln + (j >> 1)) * 4 + el + (j & 1)), yv);
-      }
-      const size_t o = (size_t)tok * a.H + r * 16 + m;
-      if (!finite_bits(yv)) set_status(QK_ERR_NONFINITE);
-      if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.y)[o] = __float2bfloat16_rn(yv);
-      else reinterpret_cast<float*>(a.y)[o] = yv;
-    }
-  };
-  auto flush = [&]() {
-    __threadfence();  // this warp's unit results, before the counters
-    __syncwarp();
-    bool last = false;
-    int r = 0;
-    if (lane < npend) {
-      int v_unused;
-      unit_vr(pend, v_unused, r);
-      last = atom_add_acq_rel(a.cnt + r, 1u) + 1u == (uint32_t)n_v;
-    }
-    unsigned m = __ballot_sync(0xffffffffu, last);
-    if (m) __threadfence();
-    while (m) {
-      const int i = __ffs(m) - 1;
-      m &= m - 1;
-      combine(__shfl_sync(0xffffffffu, r, i));
-    }
-    npend = 0;
-  };
-
   // A finished unit: scale, then SwiGLU into h (k_gateup) or the unit result (k_down).
   auto finalize = [&](int u, float4 f, int seg_v0) {
     int v, r;
@@ -707,8 +627,6 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     } else {
       // stored expert-major whatever the processing order (the combine reads v * RT + r)
       reinterpret_cast<float4*>(a.ures)[((size_t)v * RT + r) * 32 + lane] = make_float4(fv[0], fv[1], fv[2], fv[3]);
-      if (lane == npend) pend = u;
-      if (++npend == 32) flush();
     }
   };
 
@@ -883,8 +801,44 @@ __global__ void __launch_bounds__(kDW * 32, 1) k_decode(const __grid_constant__ 
     __syncthreads();  // the next segment reuses the staged rows and the pieces
     u_seg = seg_u1;
   }
-  if (!GATEUP && npend > 0 && !dead) flush();
   if (bad) set_status(QK_ERR_NAN_SCALE);
+}
+
+// y[t][m] = sum over slots s in order of w[t][s] * (the k_down unit result of
+// pair (t, s) for row m): one thread per output, the loads of up to 8 slots in
+// flight together.  Launched after k_down (programmatic dependent launch): the
+// routing table is built while k_down runs; griddepcontrol.wait returns when
+// the unit results are complete and visible.
+__global__ void __launch_bounds__(256) k_decode_y(const __grid_constant__ DecodeArgs a) {
+  __shared__ Route R;
+  build_route(a.ids, a.P, a.E, R);  // ends with __syncthreads
+  pdl_wait();
+  const int RT = a.H / 16;
+  const float* ures = a.ures;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < a.T * a.H; idx += gridDim.x * blockDim.x) {
+    const int tok = idx / a.H, row = idx - tok * a.H, r = row >> 4, m = row & 15;
+    const int ln = (m & 7) * 4, el = (m >= 8) ? 2 : 0;
+    float d[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      d[s] = 0.f;
+      if (s < a.k) {
+        const int p = tok * a.k + s;
+        const int pv = R.pair_v[p];
+        if (pv >= 0) {
+          const int j = R.pair_j[p];
+          d[s] = __ldcg(ures + (((size_t)pv * RT + r) * 32 + ln + (j >> 1)) * 4 + el + (j & 1));
+        }
+      }
+    }
+    float yv = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (s < a.k) yv = fmaf(__ldg(a.w + tok * a.k + s), d[s], yv);
+    if (!finite_bits(yv)) set_status(QK_ERR_NONFINITE);
+    if (a.y_bf16) reinterpret_cast<__nv_bfloat16*>(a.y)[idx] = __float2bfloat16_rn(yv);
+    else reinterpret_cast<float*>(a.y)[idx] = yv;
+  }
 }
 
 // ================================================================= host ==
@@ -967,12 +921,15 @@ qk_status decode_forward(DecodeArgs args, cudaStream_t st) {
   else if (fu == MX) rc = go<NV, MX, true>(P1, st, true);
   else rc = go<NV, NV, true>(P1, st, true);
   if (rc != QK_OK) return rc;
-  return fd == MX ? go<MX, MX, false>(P2, st, true) : go<NV, NV, false>(P2, st, true);
+  rc = fd == MX ? go<MX, MX, false>(P2, st, true) : go<NV, NV, false>(P2, st, true);
+  if (rc != QK_OK) return rc;
+  const int grid = std::max(1, std::min(2 * num_sms(), (args.T * args.H + 255) / 256));
+  return launch_ex(k_decode_y, dim3(grid), dim3(256), 0, st, true, args);
 }
 
-// Workspace: h [P][I] f32 | hmax [P][I/8] | ures [P*H/16][32] float4 | cnt [H/16].
+// Workspace: h [P][I] f32 | hmax [P][I/8] | ures [P*H/16][32] float4.
 struct WsLayout {
-  size_t h, hmax, ures, cnt, total;
+  size_t h, hmax, ures, total;
 };
 
 static WsLayout ws_layout(int T, int k, int H, int I) {
@@ -982,7 +939,6 @@ static WsLayout ws_layout(int T, int k, int H, int I) {
   L.h = o; o += align256(P * I * 4);
   L.hmax = o; o += align256(P * (I / 8) * 4);
   L.ures = o; o += align256(P * (H / 16) * 512);
-  L.cnt = o; o += align256((size_t)(H / 16) * 4);
   L.total = o;
   return L;
 }
@@ -995,7 +951,6 @@ void decode_carve(DecodeArgs& a, void* ws) {
   a.h = reinterpret_cast<float*>(p + L.h);
   a.hmax = reinterpret_cast<float*>(p + L.hmax);
   a.ures = reinterpret_cast<float*>(p + L.ures);
-  a.cnt = reinterpret_cast<uint32_t*>(p + L.cnt);
 }
 
 }  // namespace qk

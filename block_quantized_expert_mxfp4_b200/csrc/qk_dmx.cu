@@ -20,9 +20,10 @@
 //                   pg, no reduction across units.
 //   k_dmx<down>     (programmatic dependent launch) A = h terms, built from
 //                   the gate/up partials summed in chunk order, SwiGLU, and
-//                   the split; partial sums to pd; the last unit to finish an
-//                   output block of 128 rows (a per-block counter) forms y
-//                   for those rows in slot order (deterministic).
+//                   the split; partial sums to pd.
+//   k_dmx_y         (programmatic dependent launch) one warp per (token,
+//                   128 output rows): y in slot order from pd
+//                   (deterministic).
 //
 // Warp roles (8 warps): weight TMA (16 x 4-bit -> 16-byte slots, box 128
 // codes x 128 rows, 3 stages), MMA issuer, weight-scale formatter (16 bytes
@@ -61,7 +62,6 @@ struct DmxArgs {
   void* y;               // [T][H] fp32 or bf16
   float* pg;             // [P sorted][2 I / 128][H / 1024][128] gate/up partial sums
   float* pd;             // [P sorted][H / 128][I / 1024][128] down partial sums
-  uint32_t* cnt;         // [H / 128] down units finished per output block
   int T, k, E, H, I, P, y_bf16;
   alignas(64) CUtensorMap ta, tb;  // packed weights, 16 x 4-bit -> 16-byte slots, box {128, 128}, 128B swizzle
 };
@@ -245,25 +245,14 @@ __global__ void __launch_bounds__(kDThreads, 2) k_dmx(const __grid_constant__ Dm
   if (warp == 1) tmem_alloc(&S.tmem, kDTmemCols);
   // The ids may come from the kernel launched just before (router); the down
   // kernel's ids were complete before the gate/up kernel it follows started.
-  if (GATEUP) {
-    pdl_wait();
-    if (blockIdx.x == 0)  // the down kernel's per-block counters (it starts after this kernel completes)
-      for (int i = threadIdx.x; i < G.H / kDN; i += blockDim.x) G.cnt[i] = 0u;
-  }
+  if (GATEUP) pdl_wait();
   build_route(G.ids, G.P, G.E, R);  // ends with __syncthreads
-  if (GATEUP) pdl_launch_dependents();
+  pdl_launch_dependents();  // the next kernel (down, then k_dmx_y) may start its prologue
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem;
   const int U = R.n_v * NB * CH;
-  if (!GATEUP && U == 0 && blockIdx.x == 0)  // every id invalid: no unit writes y
-    for (int i = threadIdx.x; i < G.T * G.H; i += blockDim.x) {
-      if (G.y_bf16)
-        reinterpret_cast<__nv_bfloat16*>(G.y)[i] = __float2bfloat16_rn(0.f);
-      else
-        reinterpret_cast<float*>(G.y)[i] = 0.f;
-    }
   const int u0 = (int)((long long)blockIdx.x * U / gridDim.x), u1 = (int)((long long)(blockIdx.x + 1) * U / gridDim.x);
   auto unit = [&](int u, int& v, int& nb, int& c) {
     c = u % CH;
@@ -451,48 +440,6 @@ __global__ void __launch_bounds__(kDThreads, 2) k_dmx(const __grid_constant__ Dm
                                __uint_as_float(r[4 * q + 3]));
         }
       }
-      if (!GATEUP) {
-        // Output block nb is complete when all n_v x CH of its units are in.
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) last = atomicAdd(&G.cnt[nb], 1u) == (unsigned)(R.n_v * CH - 1);
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          // y[t][rows] = sum over slots in order of w * (sum over chunks in order of d)
-          for (int t = 0; t < G.T; ++t) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int s = 0; s < G.k; ++s) {
-              const int p = t * G.k + s, pv = R.pair_v[p];
-              if (pv < 0) continue;
-              const int sp = R.v_p0[pv] + R.pair_j[p];
-              const float wt = G.w[p];
-              float d[4] = {0.f, 0.f, 0.f, 0.f};
-              for (int cc = 0; cc < CH; ++cc) {
-                const float4 x4 =
-                    __ldcg(reinterpret_cast<const float4*>(G.pd + (((size_t)sp * NB + nb) * CH + cc) * kDN) + lane);
-                d[0] += x4.x;
-                d[1] += x4.y;
-                d[2] += x4.z;
-                d[3] += x4.w;
-              }
-#pragma unroll
-              for (int q = 0; q < 4; ++q) acc[q] = fmaf(wt, d[q], acc[q]);
-            }
-            if (!(finite_bits(acc[0]) && finite_bits(acc[1]) && finite_bits(acc[2]) && finite_bits(acc[3])))
-              set_status(QK_ERR_NONFINITE);
-            const size_t o = (size_t)t * G.H + nb * kDN + lane * 4;
-            if (G.y_bf16) {
-              __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(G.y) + o;
-#pragma unroll
-              for (int q = 0; q < 4; ++q) yb[q] = __float2bfloat16_rn(acc[q]);
-            } else {
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(G.y) + o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            }
-          }
-        }
-      }
     }
   }
   if (warp == 4) {  // the epilogue's TMEM reads are done (also on an early exit)
@@ -506,6 +453,87 @@ __global__ void __launch_bounds__(kDThreads, 2) k_dmx(const __grid_constant__ Dm
     mbar_wait_bounded(&S.epi_done, 0, kDrainLimitNs);
     tc_fence_after();
     tmem_free(tmem, kDTmemCols);
+  }
+}
+
+// y[t][block nb] = sum over slots s in order of w[t][s] * (sum over K chunks
+// in order of the down partial sums): one warp per (token, 128-row output
+// block), 32 lanes x 4 rows; all the (slot, chunk) loads in flight at once.
+// Launched after the down kernel (programmatic dependent launch): the
+// routing table is built while the down kernel runs; griddepcontrol.wait
+// returns when its partial sums are complete and visible.
+constexpr int kDyWarps = 8;
+__global__ void __launch_bounds__(kDyWarps * 32) k_dmx_y(const __grid_constant__ DmxArgs G) {
+  __shared__ Route R;
+  build_route(G.ids, G.P, G.E, R);  // ends with __syncthreads
+  pdl_wait();
+  const int lane = threadIdx.x & 31, nb = blockIdx.x, t = blockIdx.y * kDyWarps + (threadIdx.x >> 5);
+  if (t >= G.T) return;
+  const int NB = G.H / kDN, CH = G.I / kDKc;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (CH <= 4) {
+    float4 x4[8][4];
+    float wt[8];
+    bool on[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      on[s] = false;
+      if (s < G.k) {
+        const int p = t * G.k + s, pv = R.pair_v[p];
+        if (pv >= 0) {
+          on[s] = true;
+          wt[s] = __ldg(G.w + p);
+          const float4* src =
+              reinterpret_cast<const float4*>(G.pd + (size_t)(R.v_p0[pv] + R.pair_j[p]) * NB * CH * kDN) +
+              (size_t)nb * CH * (kDN / 4) + lane;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+            if (cc < CH) x4[s][cc] = __ldcg(src + cc * (kDN / 4));
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (on[s]) {
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          if (cc < CH) {
+            d[0] += x4[s][cc].x;
+            d[1] += x4[s][cc].y;
+            d[2] += x4[s][cc].z;
+            d[3] += x4[s][cc].w;
+          }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = fmaf(wt[s], d[q], acc[q]);
+      }
+  } else {
+    for (int s = 0; s < G.k; ++s) {
+      const int p = t * G.k + s, pv = R.pair_v[p];
+      if (pv < 0) continue;
+      const int sp = R.v_p0[pv] + R.pair_j[p];
+      const float wt = G.w[p];
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int cc = 0; cc < CH; ++cc) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(G.pd + (((size_t)sp * NB + nb) * CH + cc) * kDN) + lane);
+        d[0] += v.x;
+        d[1] += v.y;
+        d[2] += v.z;
+        d[3] += v.w;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[q] = fmaf(wt, d[q], acc[q]);
+    }
+  }
+  if (!(finite_bits(acc[0]) && finite_bits(acc[1]) && finite_bits(acc[2]) && finite_bits(acc[3])))
+    set_status(QK_ERR_NONFINITE);
+  const size_t o = (size_t)t * G.H + nb * kDN + lane * 4;
+  if (G.y_bf16) {
+    __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(G.y) + o;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) yb[q] = __float2bfloat16_rn(acc[q]);
+  } else {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(G.y) + o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
   }
 }
 
@@ -523,7 +551,7 @@ bool dmx_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight& d
 }
 
 struct DmxWs {
-  size_t pg, pd, cnt, total;
+  size_t pg, pd, total;
 };
 static DmxWs dmx_layout(int T, int k, int H, int I) {
   const size_t P = (size_t)T * k;
@@ -531,7 +559,6 @@ static DmxWs dmx_layout(int T, int k, int H, int I) {
   size_t o = 0;
   L.pg = o; o += align256(P * (2 * I / kDN) * (H / kDKc) * kDN * 4);
   L.pd = o; o += align256(P * (H / kDN) * (I / kDKc) * kDN * 4);
-  L.cnt = o; o += align256((size_t)(H / kDN) * 4);
   L.total = o;
   return L;
 }
@@ -561,7 +588,6 @@ qk_status dmx_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
   g.y = a.y;
   g.pg = reinterpret_cast<float*>(p + L.pg);
   g.pd = reinterpret_cast<float*>(p + L.pd);
-  g.cnt = reinterpret_cast<uint32_t*>(p + L.cnt);
   g.T = a.T;
   g.k = a.k;
   g.E = a.E;
@@ -580,7 +606,9 @@ qk_status dmx_forward(const DecodeArgs& a, void* workspace, cudaStream_t st) {
   g.B = a.down;
   if (!d_map_weights(&g.ta, a.down.q, (int64_t)a.E * a.H, a.I)) return QK_ERR_CUDA;
   g.tb = g.ta;
-  return d_launch<false>(g, st);
+  rc = d_launch<false>(g, st);
+  if (rc != QK_OK) return rc;
+  return launch_ex(k_dmx_y, dim3(a.H / kDN, (a.T + kDyWarps - 1) / kDyWarps), dim3(kDyWarps * 32), 0, st, true, g);
 }
 
 }  // namespace qk

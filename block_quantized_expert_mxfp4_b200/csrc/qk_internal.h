@@ -34,7 +34,6 @@ struct DecodeArgs {
   float* h;           // [P][I] fp32 SwiGLU output
   float* hmax;        // [P][I/8] absmax of h per 8-row tile
   float* ures;        // [units][32] float4: k_down result of each (virtual expert, row tile)
-  uint32_t* cnt;      // [H/16] k_down units finished per row tile (zeroed by k_gateup)
 };
 
 qk_status decode_forward(DecodeArgs args, cudaStream_t st);
