@@ -342,6 +342,14 @@ struct GmxArgs {
   const float* s2a;      // NVFP4 weights: scale_2 [E] of the gate (or down) projection
   const float* s2b;      //    and of the up projection
   const float* fac;      // NVFP4 weights: per sorted row, the factor of its token scales
+  // Fused gate/up (fuse = 1): a tile is 128 gate rows and the same 128 up
+  // rows (two 128-row boxes per step), and the epilogue writes h = silu(gate)
+  // * up straight into the down tiles in the mode's split (no gu, no h split
+  // kernel).
+  int fuse, act_quant, I;
+  const int* rtile2;     // [P] per sorted row: (down tile << 8) | row within it
+  uint8_t* ht;           // down token blocks
+  uint8_t* sfh;          // their scale atoms
   alignas(64) CUtensorMap ta, tb;  // MXFP4: 16 x 4-bit -> 16-byte slots; FP8: bytes; box {128, 256}, 128B swizzle
 };
 
@@ -448,6 +456,11 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
       auto coords = [&](int t, const void*& map, int& wrow) {
         int f, mb;
         gmx_tile(L, MB, t, f, mb);
+        if (GATEUP && G.fuse) {  // gate rows, then the same up rows (map tb)
+          map = &G.ta;
+          wrow = L.tile_e[f] * G.rows_per_e + mb * (kWN / 2);
+          return;
+        }
         const bool b = mb >= G.MBA;
         map = b ? &G.tb : &G.ta;
         wrow = L.tile_e[f] * G.rows_per_e + (b ? mb - G.MBA : mb) * kWN;
@@ -462,7 +475,12 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
           if (n >= kXWS && !wait(&S.wempty[s], (uint32_t)((n / kXWS - 1) & 1))) break;
           // counted in global bytes: packed (4-bit) codes, or one byte per FP8 code
           mbar_arrive_expect_tx(&S.wfull[s], (uint32_t)(G.wfp8 || FP4 ? kXStageW : kXStageW / 2));
-          tma_load_2d(sW + s * kXStageW, map, ks * kXK, wrow, &S.wfull[s], pw);
+          if (GATEUP && G.fuse) {
+            tma_load_2d(sW + s * kXStageW, &G.ta, ks * kXK, wrow, &S.wfull[s], pw);
+            tma_load_2d(sW + s * kXStageW + kXStageW / 2, &G.tb, ks * kXK, wrow, &S.wfull[s], pw);
+          } else {
+            tma_load_2d(sW + s * kXStageW, map, ks * kXK, wrow, &S.wfull[s], pw);
+          }
         }
       }
       for (int q = n > kXWS ? n - kXWS : 0; q < n; ++q)  // nothing may still be landing at exit
@@ -482,25 +500,42 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
     auto fetch = [&](int t, int chunk, uint4 (&r)[8]) {
       int f, mb;
       gmx_tile(L, MB, t, f, mb);
-      const bool b = mb >= G.MBA;
-      const uint8_t* sf = b ? G.sf_b : G.sf_a;
-      const int base = L.tile_e[f] * G.rows_per_e + (b ? mb - G.MBA : mb) * kWN;
+      const bool fz = GATEUP && G.fuse;  // rows 0-127 gate, 128-255 the same up rows
+      const bool b = !fz && mb >= G.MBA;
+      const int base = L.tile_e[f] * G.rows_per_e + (fz ? mb * (kWN / 2) : (b ? mb - G.MBA : mb) * kWN);
+      // row lane + 32 j of the tile: its projection's scales and row index
+      auto src = [&](int j, int& row) -> const uint8_t* {
+        if (fz) {
+          row = base + lane + 32 * (j & 3);
+          return j < 4 ? G.sf_a : G.sf_b;
+        }
+        row = base + lane + 32 * j;
+        return b ? G.sf_b : G.sf_a;
+      };
       if (!G.wfp8) {
-        const uint8_t* rp = sf + (size_t)(base + lane) * srow + chunk * 16;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) r[j] = __ldg(reinterpret_cast<const uint4*>(rp + (size_t)32 * j * srow));
+        for (int j = 0; j < 8; ++j) {
+          int row;
+          const uint8_t* sf = src(j, row);
+          r[j] = __ldg(reinterpret_cast<const uint4*>(sf + (size_t)row * srow + chunk * 16));
+        }
       } else if (G.sblk == 128) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
+          int row;
+          const uint8_t* sf = src(j, row);
           const uint32_t c4 = __ldg(reinterpret_cast<const uint32_t*>(
-              sf + (size_t)((base + 32 * j) / 128) * (G.K / 128) + 4 * chunk));
+              sf + (size_t)((row - lane) / 128) * (G.K / 128) + 4 * chunk));
           r[j] = make_uint4((c4 & 0xFFu) * 0x01010101u, ((c4 >> 8) & 0xFFu) * 0x01010101u,
                             ((c4 >> 16) & 0xFFu) * 0x01010101u, (c4 >> 24) * 0x01010101u);
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          r[j] = __ldg(reinterpret_cast<const uint4*>(sf + (size_t)((base + 32 * j) / 32) * (G.K / 32) + 16 * chunk));
+        for (int j = 0; j < 8; ++j) {
+          int row;
+          const uint8_t* sf = src(j, row);
+          r[j] = __ldg(reinterpret_cast<const uint4*>(sf + (size_t)((row - lane) / 32) * (G.K / 32) + 16 * chunk));
+        }
       }
     };
     uint4 cur[8], nxt[8];
@@ -659,6 +694,65 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
       tc_fence_after();
       const int tok = NPQ * quad + lane;
       const bool st = lane < NPQ && tok < nrow;
+      if (GATEUP && G.fuse) {
+        // Columns c (gate) and 128 + c (up) are intermediate index 128 mb + c
+        // of the same token: warp half h takes the 32-column chunks 2 h and
+        // 2 h + 1, forms h = silu(gate) * up (the h split kernel's
+        // arithmetic) and writes its 32-blocks into the down tiles.
+        const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
+        float hv[2][32];
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int cc = 2 * half + k2;
+          uint32_t g[32], u[32];
+          tmem_ld32(tq + (uint32_t)(cc * 32), g);
+          tmem_ld32(tq + (uint32_t)(kWN / 2 + cc * 32), u);
+          if (k2 == 1) {  // the accumulator is read: the next tile's MMAs may start
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_one(&S.acc_empty);
+          }
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            float a = __uint_as_float(g[jj]), b = __uint_as_float(u[jj]);
+            if (NT > 1) {
+              a += __shfl_down_sync(0xffffffffu, a, NPQ);
+              b += __shfl_down_sync(0xffffffffu, b, NPQ);
+              if (NT == 3) {
+                a += __shfl_down_sync(0xffffffffu, __uint_as_float(g[jj]), 2 * NPQ);
+                b += __shfl_down_sync(0xffffffffu, __uint_as_float(u[jj]), 2 * NPQ);
+              }
+            }
+            hv[k2][jj] = __fdividef(a, 1.0f + __expf(-a)) * b;
+          }
+        }
+        if (st) {
+          const int tj = __ldg(G.rtile2 + row0 + tok), f2 = tj >> 8, j2 = tj & 255;
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            float (&v)[32] = hv[k2];
+            const int b = mb * 4 + 2 * half + k2;  // 32-block of the h row
+            if (!all_finite32(v)) set_status(QK_ERR_NONFINITE);
+            if (G.act_quant == QK_ACT_NONE) {
+#pragma unroll
+              for (int term = 0; term < 3; ++term) {
+                uint32_t q[8];
+                const int c = split_term(v, q);
+                put_term(G.ht, G.sfh, f2, G.I / kXK, kXTok2 / 4, j2, term, b, q, c);
+              }
+            } else if (G.act_quant == QK_ACT_MXFP4) {
+              uint32_t q4[4];
+              const int c = actq_block_fp4(v, q4);
+              put_fp4(G.ht, G.sfh, f2, G.I / 256, j2, b, q4, c);
+            } else {
+              uint32_t q[8];
+              const int c = actq_block(v, q, 0);
+              put_term(G.ht, G.sfh, f2, G.I / kXK, 32, j2, 0, b, q, c);
+            }
+          }
+        }
+        continue;
+      }
       float* out = G.out + (size_t)(row0 + (st ? tok : 0)) * G.out_ld + mb * kWN + half * 128;
       float mul = 1.f;  // NVFP4: scale_2 of the tile's expert and projection, times the row's factor
       if (NV && st) mul = __ldg((mb >= G.MBA ? G.s2b : G.s2a) + L.tile_e[f]) * __ldg(G.fac + row0 + tok);
@@ -728,20 +822,20 @@ bool gmx_nv_eligible(const qk_weight& gate, const qk_weight& up, const qk_weight
 // shared memory, boxes {128 codes, 256 rows}, 128-byte swizzle.  A box reads
 // 64 bytes of each row; 256-byte L2 promotion brings the row's next three
 // steps into L2 with the first.
-static bool x_map_weights(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
+static bool x_map_weights(CUtensorMap* m, const uint8_t* q, int64_t rows, int K, int box_rows = kWN) {
   const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
   const uint64_t strides[1] = {(uint64_t)K / 2};
-  const uint32_t box[2] = {(uint32_t)kXK, (uint32_t)kWN};
+  const uint32_t box[2] = {(uint32_t)kXK, (uint32_t)box_rows};
   return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 // FP8 E4M3 rows [rows][K] bytes, boxes {128, 256}, 128-byte swizzle: the same
 // shared-memory layout as the expanded e2m1 slots (one code per byte).
-static bool x_map_fp8(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
+static bool x_map_fp8(CUtensorMap* m, const uint8_t* q, int64_t rows, int K, int box_rows = kWN) {
   const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
   const uint64_t strides[1] = {(uint64_t)K};
-  const uint32_t box[2] = {(uint32_t)kXK, (uint32_t)kWN};
+  const uint32_t box[2] = {(uint32_t)kXK, (uint32_t)box_rows};
   return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
@@ -755,10 +849,10 @@ static qk_status x_launch(const GmxArgs& A, cudaStream_t st) {
 
 // Packed e2m1 rows [rows][K / 2] as bytes, boxes {128 bytes (256 codes), 256
 // rows}, 128-byte swizzle: the fp4 x fp4 path reads the weights as stored.
-static bool x_map_packed(CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
+static bool x_map_packed(CUtensorMap* m, const uint8_t* q, int64_t rows, int K, int box_rows = kWN) {
   const uint64_t dims[2] = {(uint64_t)K / 2, (uint64_t)rows};
   const uint64_t strides[1] = {(uint64_t)K / 2};
-  const uint32_t box[2] = {(uint32_t)kXK, (uint32_t)kWN};
+  const uint32_t box[2] = {(uint32_t)kXK, (uint32_t)box_rows};
   return tmap_get(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
@@ -773,9 +867,13 @@ qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, 
   const bool nv = fp4 && a.gate.fmt == QK_FMT_NVFP4;  // an all-NVFP4 layer (gmx_nv_eligible): kind::mxf4nvf4
   k_gmx_xsplit<<<T, kRowThreads, 0, st>>>(W, a.x, a.ids, k, E, H, act_quant, nv ? 1 : 0);
   if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
-  auto wmap = [&](CUtensorMap* m, const uint8_t* q, int64_t rows, int K) {
-    return fp4 ? x_map_packed(m, q, rows, K) : x_map_weights(m, q, rows, K);
+  auto wmap = [&](CUtensorMap* m, const uint8_t* q, int64_t rows, int K, int box_rows = kWN) {
+    return fp4 ? x_map_packed(m, q, rows, K, box_rows) : x_map_weights(m, q, rows, K, box_rows);
   };
+  // MXFP4 layers: the gate/up epilogue forms h and writes the down tiles
+  // itself (NVFP4 layers keep the h split kernel: their h scales are
+  // anchored at the row's largest, known only once the whole row is in).
+  const bool fuse = !nv;
 
   GmxArgs g1 = {};
   g1.L = W.L1;
@@ -792,15 +890,29 @@ qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, 
   g1.s2a = a.gate.scale_2;
   g1.s2b = a.up.scale_2;
   g1.fac = W.fac1;
-  if (!wmap(&g1.ta, a.gate.q, (int64_t)E * I, H) || !wmap(&g1.tb, a.up.q, (int64_t)E * I, H)) return QK_ERR_CUDA;
+  if (fuse) {
+    g1.fuse = 1;
+    g1.MB = I / (kWN / 2);  // 128 gate rows and the same 128 up rows per tile
+    g1.MBA = g1.MB;
+    g1.act_quant = act_quant;
+    g1.I = I;
+    g1.rtile2 = W.rtile2;
+    g1.ht = W.ht;
+    g1.sfh = W.sfh;
+  }
+  const int br = fuse ? kWN / 2 : kWN;
+  if (!wmap(&g1.ta, a.gate.q, (int64_t)E * I, H, br) || !wmap(&g1.tb, a.up.q, (int64_t)E * I, H, br))
+    return QK_ERR_CUDA;
   qk_status rc = nv    ? x_launch<true, 1, true, true>(g1, st)
                  : fp4 ? x_launch<true, 1, true>(g1, st)
                  : one ? x_launch<true, 1>(g1, st)
                        : x_launch<true, 2>(g1, st);
   if (rc != QK_OK) return rc;
 
-  k_gmx_hsplit<<<a.P, kRowThreads, 0, st>>>(W, E, I, act_quant, nv ? 1 : 0);
-  if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
+  if (!fuse) {
+    k_gmx_hsplit<<<a.P, kRowThreads, 0, st>>>(W, E, I, act_quant, nv ? 1 : 0);
+    if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
+  }
 
   GmxArgs g2 = {};
   g2.L = W.L2;
@@ -849,11 +961,17 @@ qk_status gmx_fp8_ffn(const GroupWs& W, const uint16_t* x, const int32_t* ids, i
   g1.out_ld = 2 * I;
   g1.wfp8 = 1;
   g1.sblk = blk;
-  if (!x_map_fp8(&g1.ta, wg, I, H) || !x_map_fp8(&g1.tb, wu, I, H)) return QK_ERR_CUDA;
+  g1.fuse = 1;  // h formed and split in the gate/up epilogue
+  g1.MB = I / (kWN / 2);
+  g1.MBA = g1.MB;
+  g1.act_quant = QK_ACT_NONE;
+  g1.I = I;
+  g1.rtile2 = W.rtile2;
+  g1.ht = W.ht;
+  g1.sfh = W.sfh;
+  if (!x_map_fp8(&g1.ta, wg, I, H, kWN / 2) || !x_map_fp8(&g1.tb, wu, I, H, kWN / 2)) return QK_ERR_CUDA;
   qk_status rc = x_launch<true, 2>(g1, st);
   if (rc != QK_OK) return rc;
-  k_gmx_hsplit<<<M, kRowThreads, 0, st>>>(W, 1, I, QK_ACT_NONE, 0);
-  if (cudaGetLastError() != cudaSuccess) return QK_ERR_CUDA;
   GmxArgs g2 = {};
   g2.L = W.L2;
   g2.blocks = W.ht;
