@@ -380,7 +380,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.empty_cache()
     if args.prefill_steps > 0:
         out["prefill"] = run_prefill(args, rank, world, dev)
-        # count, two tile-list scans, x split, gate/up GEMM, h split, down GEMM, combine
+        # count, two tile-list scans, x split, gate/up GEMM (+ SwiGLU and the h split), down GEMM, combine
         out["gpu_launches"] += out["prefill"]["gpu_launches"]
     if args.extra == "all":
         # the other configurations, each timed in its own region (not part of `value`)
@@ -450,7 +450,8 @@ def run_shared_fp8(args, rank, world, dev):
     res = {"workload": "FP8 E4M3 shared expert, hidden 4096, intermediate 2048, UE8M0 per 128x128 tile, "
                        "bf16 N(0,1) activations, result added into y",
            "path": "one group of M tokens on the block-scaled grouped GEMMs: x as 2 exact e4m3 terms, "
-                   "e4m3 weights as stored (kind::mxf8f6f4), SwiGLU + 3-term h split, add into y",
+                   "e4m3 weights as stored (kind::mxf8f6f4), SwiGLU + 3-term h split in the gate/up epilogue, "
+                   "add into y",
            "tensor_peak_tflops": 2 * bf16,
            "tensor_peak_kind": f"{src} bf16 x 2 (nominal fp8/bf16 ratio): kind::mxf8f6f4",
            "by_rows": {}}
@@ -471,7 +472,7 @@ def run_shared_fp8(args, rank, world, dev):
                                   "achieved_tflops": round(flops / t / 1e12, 1),
                                   "tensor_frac": round(flops / t / 1e12 / (2 * bf16), 4),
                                   "weight_bytes": sh.nbytes(), "hbm_frac": round(sh.nbytes() / t / 1e9 / peak, 4)}
-        launches += K * 9  # route fill, count, two scans, x split, gate/up, h split, down, combine
+        launches += K * 8  # route fill, count, two scans, x split, gate/up (+ h split), down, combine
         del x, y, ws
     res["gpu_launches"] = launches
     return res
@@ -673,7 +674,8 @@ def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0, nv=False):
                    "peak_tflops": tpeak, "peak_kind": tkind, "frac": round(flops / t / 1e12 / tpeak, 4),
                    "frac_of_fp4_peak": round(flops / t / 1e12 / (4 * bf16), 4)},
         "path": ("counting sort by expert; x as 2 exact e4m3 terms; block-scaled tcgen05 grouped GEMMs "
-                 "(e2m1 weights + e8m0 scales as stored): gate/up, SwiGLU + 3-term h split, down; combine")
+                 "(e2m1 weights + e8m0 scales as stored): gate/up with SwiGLU + 3-term h split in its epilogue, "
+                 "down; combine")
         if aq == qk.QK_ACT_NONE else
         (f"counting sort by expert; x and h quantized to {act_name} (one term per token, 128-token tiles); "
          + ("both operands packed e2m1, block-scaled tcgen05 kind::mxf4nvf4 grouped GEMMs (e2m1 + e4m3 per 16 "
@@ -681,7 +683,7 @@ def run_prefill(args, rank, world, dev, tokens=0, act=None, steps=0, nv=False):
             "both operands packed e2m1, block-scaled tcgen05 kind::mxf4 grouped GEMMs (weights as stored)"
             if aq == qk.QK_ACT_MXFP4 else "block-scaled tcgen05 kind::mxf8f6f4 grouped GEMMs")
          + "; combine"),
-        "gpu_launches": 8 * K,
+        "gpu_launches": (8 if nv else 7) * K,  # the NVFP4 fp4 mode keeps the h split kernel
     }
 
 

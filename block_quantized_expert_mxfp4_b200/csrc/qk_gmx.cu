@@ -40,11 +40,14 @@
 //   k_gmx_xsplit  per token: x -> 2 e4m3 terms (1 term, or packed e2m1, in
 //                 the quantized modes), written into the tile blocks of each
 //                 of its pairs (gate/up tiles of 64 tokens, 128 quantized).
-//   k_gmx<gate/up>  per (expert, 256 gate or up rows, token tile): gate and up
-//                 outputs (fp32) to gu.
-//   k_gmx_hsplit  per sorted row: h = silu(gate) * up -> 3 e4m3 terms in the
-//                 down tile blocks (40 tokens per tile; 1 term or packed
-//                 e2m1 and 128 tokens in the quantized modes).
+//   k_gmx<gate/up>  per (expert, 128 gate rows + the same 128 up rows, token
+//                 tile): the epilogue forms h = silu(gate) * up and writes
+//                 its 3 e4m3 terms into the down tile blocks (40 tokens per
+//                 tile; 1 term or packed e2m1 and 128 tokens in the quantized
+//                 modes).  NVFP4 layers in the fp4 mode instead write gate and
+//                 up (fp32) to gu, and
+//   k_gmx_hsplit  per sorted row forms and splits h (its scales anchor at the
+//                 row's largest, known once the whole row is in).
 //   k_gmx<down>   per (expert, 256 down rows, token tile): d (fp32).
 //
 // Token block (one reduction step of a tile, the MMA's A operand as it sits
