@@ -402,6 +402,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
   constexpr int NPQ = NT == 1 ? 32 : NT == 2 ? kXTok1 / 4 : kXTok2 / 4;  // tokens per TMEM lane quadrant
   constexpr int AT = NV ? 4 : FP4 ? 2 : 1;   // token scale atoms per step
   constexpr int SPC = NV ? 1 : FP4 ? 2 : 4;  // steps per weight-scale chunk (16 bytes of each row)
+  constexpr bool FUSE = GATEUP && !NV;       // instantiations that may run the fused gate/up (G.fuse)
   extern __shared__ __align__(16) uint8_t smem_raw[];  // rounded up to 1024 below, at run time
   uint8_t* base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sW = base;                                  // kXWS weight stages
@@ -459,7 +460,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
       auto coords = [&](int t, const void*& map, int& wrow) {
         int f, mb;
         gmx_tile(L, MB, t, f, mb);
-        if (GATEUP && G.fuse) {  // gate rows, then the same up rows (map tb)
+        if (FUSE && G.fuse) {  // gate rows, then the same up rows (map tb)
           map = &G.ta;
           wrow = L.tile_e[f] * G.rows_per_e + mb * (kWN / 2);
           return;
@@ -478,7 +479,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
           if (n >= kXWS && !wait(&S.wempty[s], (uint32_t)((n / kXWS - 1) & 1))) break;
           // counted in global bytes: packed (4-bit) codes, or one byte per FP8 code
           mbar_arrive_expect_tx(&S.wfull[s], (uint32_t)(G.wfp8 || FP4 ? kXStageW : kXStageW / 2));
-          if (GATEUP && G.fuse) {
+          if (FUSE && G.fuse) {
             tma_load_2d(sW + s * kXStageW, &G.ta, ks * kXK, wrow, &S.wfull[s], pw);
             tma_load_2d(sW + s * kXStageW + kXStageW / 2, &G.tb, ks * kXK, wrow, &S.wfull[s], pw);
           } else {
@@ -503,42 +504,52 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
     auto fetch = [&](int t, int chunk, uint4 (&r)[8]) {
       int f, mb;
       gmx_tile(L, MB, t, f, mb);
-      const bool fz = GATEUP && G.fuse;  // rows 0-127 gate, 128-255 the same up rows
-      const bool b = !fz && mb >= G.MBA;
-      const int base = L.tile_e[f] * G.rows_per_e + (fz ? mb * (kWN / 2) : (b ? mb - G.MBA : mb) * kWN);
-      // row lane + 32 j of the tile: its projection's scales and row index
-      auto src = [&](int j, int& row) -> const uint8_t* {
-        if (fz) {
-          row = base + lane + 32 * (j & 3);
-          return j < 4 ? G.sf_a : G.sf_b;
-        }
-        row = base + lane + 32 * j;
-        return b ? G.sf_b : G.sf_a;
-      };
-      if (!G.wfp8) {
+      if (FUSE && G.fuse) {  // rows 0-127 gate, 128-255 the same up rows
+        const int base = L.tile_e[f] * G.rows_per_e + mb * (kWN / 2);
+        if (!G.wfp8) {
+          const uint8_t* ra = G.sf_a + (size_t)(base + lane) * srow + chunk * 16;
+          const uint8_t* rb = G.sf_b + (size_t)(base + lane) * srow + chunk * 16;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          int row;
-          const uint8_t* sf = src(j, row);
-          r[j] = __ldg(reinterpret_cast<const uint4*>(sf + (size_t)row * srow + chunk * 16));
+          for (int j = 0; j < 4; ++j) {
+            r[j] = __ldg(reinterpret_cast<const uint4*>(ra + (size_t)32 * j * srow));
+            r[4 + j] = __ldg(reinterpret_cast<const uint4*>(rb + (size_t)32 * j * srow));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint8_t* sf = j < 4 ? G.sf_a : G.sf_b;
+            const int r0 = base + 32 * (j & 3);  // first of the 32 rows
+            if (G.sblk == 128) {
+              const uint32_t c4 =
+                  __ldg(reinterpret_cast<const uint32_t*>(sf + (size_t)(r0 / 128) * (G.K / 128) + 4 * chunk));
+              r[j] = make_uint4((c4 & 0xFFu) * 0x01010101u, ((c4 >> 8) & 0xFFu) * 0x01010101u,
+                                ((c4 >> 16) & 0xFFu) * 0x01010101u, (c4 >> 24) * 0x01010101u);
+            } else {
+              r[j] = __ldg(reinterpret_cast<const uint4*>(sf + (size_t)(r0 / 32) * (G.K / 32) + 16 * chunk));
+            }
+          }
         }
+        return;
+      }
+      const bool b = mb >= G.MBA;
+      const uint8_t* sf = b ? G.sf_b : G.sf_a;
+      const int base = L.tile_e[f] * G.rows_per_e + (b ? mb - G.MBA : mb) * kWN;
+      if (!G.wfp8) {
+        const uint8_t* rp = sf + (size_t)(base + lane) * srow + chunk * 16;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[j] = __ldg(reinterpret_cast<const uint4*>(rp + (size_t)32 * j * srow));
       } else if (G.sblk == 128) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          int row;
-          const uint8_t* sf = src(j, row);
           const uint32_t c4 = __ldg(reinterpret_cast<const uint32_t*>(
-              sf + (size_t)((row - lane) / 128) * (G.K / 128) + 4 * chunk));
+              sf + (size_t)((base + 32 * j) / 128) * (G.K / 128) + 4 * chunk));
           r[j] = make_uint4((c4 & 0xFFu) * 0x01010101u, ((c4 >> 8) & 0xFFu) * 0x01010101u,
                             ((c4 >> 16) & 0xFFu) * 0x01010101u, (c4 >> 24) * 0x01010101u);
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          int row;
-          const uint8_t* sf = src(j, row);
-          r[j] = __ldg(reinterpret_cast<const uint4*>(sf + (size_t)((row - lane) / 32) * (G.K / 32) + 16 * chunk));
-        }
+        for (int j = 0; j < 8; ++j)
+          r[j] = __ldg(reinterpret_cast<const uint4*>(sf + (size_t)((base + 32 * j) / 32) * (G.K / 32) + 16 * chunk));
       }
     };
     uint4 cur[8], nxt[8];
@@ -697,7 +708,7 @@ __global__ void __launch_bounds__(kXThreads, 1) k_gmx(const __grid_constant__ Gm
       tc_fence_after();
       const int tok = NPQ * quad + lane;
       const bool st = lane < NPQ && tok < nrow;
-      if (GATEUP && G.fuse) {
+      if (FUSE && G.fuse) {
         // Columns c (gate) and 128 + c (up) are intermediate index 128 mb + c
         // of the same token: warp half h takes the 32-column chunks 2 h and
         // 2 h + 1, forms h = silu(gate) * up (the h split kernel's
