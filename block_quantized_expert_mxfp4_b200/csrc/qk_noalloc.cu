@@ -14,8 +14,7 @@
 //
 // The kernels are the decode kernels of moe_expert_forward, unchanged; only
 // the origin of the workspace differs.  Nothing in the scratch has to start at
-// zero: the one counter array that must be zero is cleared by the first kernel
-// of every call.
+// zero: every buffer in it is written before it is read within a call.
 #include <cuda_runtime.h>
 
 #include "qk_internal.h"

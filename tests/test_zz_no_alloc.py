@@ -21,7 +21,11 @@ def _inputs(wl, T, seed):
     return layer, x, ids, w
 
 
-@pytest.mark.parametrize("name,T", [("decode_mx", 1), ("decode_mx", 4), ("tiny", 4)])
+# decode_mx: the block-scaled decode kernels; decode_nv: the f16 decode
+# kernels (NVFP4 layer); tiny at 100 tokens x top-2: the grouped path (200
+# pairs, within the array for this small layer)
+@pytest.mark.parametrize("name,T", [("decode_mx", 1), ("decode_mx", 4), ("tiny", 4), ("decode_nv", 4),
+                                    ("tiny", 100)])
 def test_noalloc_matches_workspace_entry(name, T):
     wl = synth.WORKLOADS[name]
     layer, x, ids, w = _inputs(wl, T, 3)
