@@ -365,9 +365,11 @@ def run_ours(args, rank, world, local_rank):
                    "bytes_per_step": bytes_per_step,
                    "l2": "inputs larger than L2: steps rotate over the resident layers",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "moe_expert_forward (k_dmx gate/up -> k_dmx down, block-scaled tcgen05, PDL-chained)",
+        "roofline": {"kernel": "moe_expert_forward (k_dmx gate/up -> k_dmx down -> k_dmx_y combine, "
+                               "block-scaled tcgen05, PDL-chained)",
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "frac_of_nominal_8tbs": round(achieved / 8000.0, 4),
                      "ffn_us": round(ffn_s * 1e6, 3), "ffn_calls_timed": len(ffn_ms),
                      "traffic": recorded_traffic()},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
