@@ -133,6 +133,21 @@ QK_HD int actq_block_fp4(const float (&v)[32], uint32_t (&q)[4]) {
   return c;
 }
 
+// NVFP4 layers in QK_ACT_MXFP4 (kind::mxf4nvf4 takes ue4m3 scales per 16):
+// a row's 32-block code c becomes the ue4m3 code of 2^(c - cmax + 8), cmax
+// the row's largest, and the row's factor is 2^(cmax - 135), so that code x
+// factor = 2^(c - 127) exactly while c >= cmax - 17.
+// ue4m3 code of 2^d (d <= 8); 0 below 2^-9, the smallest subnormal.
+QK_HD uint32_t actq_nv_code(int d) {
+  if (d >= -6) return (uint32_t)(d + 7) << 3;
+  return d >= -9 ? 1u << (d + 9) : 0u;
+}
+
+// 2^e as fp32 for -149 <= e <= 127 (subnormal below -126): the row factor.
+QK_HD float actq_pow2(int e) {
+  return e >= -126 ? actq_float((uint32_t)(e + 127) << 23) : actq_float(1u << (e + 149));
+}
+
 }  // namespace qk
 
 #if defined(__CUDACC__) && !defined(QK_ACTQ_ARITHMETIC_ONLY)

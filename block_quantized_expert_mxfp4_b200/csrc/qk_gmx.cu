@@ -133,17 +133,6 @@ __device__ __forceinline__ void put_nv(uint8_t* blocks, uint8_t* atoms, int f, i
                                (j >> 5) * 4 + 2 * (c8 & 1)) = (uint16_t)(code * 0x0101u);
 }
 
-// ue4m3 code of 2^d (d <= 8); 0 below 2^-9, the smallest subnormal.
-__device__ __forceinline__ uint32_t nv_pow2_code(int d) {
-  if (d >= -6) return (uint32_t)(d + 7) << 3;
-  return d >= -9 ? 1u << (d + 9) : 0u;
-}
-
-// 2^e as fp32 for -149 <= e <= 127 (subnormal below -126).
-__device__ __forceinline__ float pow2f_sub(int e) {
-  return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
-}
-
 // NVFP4 layers in QK_ACT_MXFP4: the row's 32-block scale codes c (the OCP
 // rule, as for MXFP4 layers) become ue4m3 codes of 2^(c - cmax + 8), cmax the
 // row's largest, and the row's factor 2^(cmax - 135) goes to the epilogue:
@@ -216,11 +205,11 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_xsplit(GroupWs W, const uin
       float v[32];
       uint32_t q4[4];
       load(b, v);
-      const uint32_t code = nv_pow2_code(actq_block_fp4(v, q4) - cm + 8);
+      const uint32_t code = actq_nv_code(actq_block_fp4(v, q4) - cm + 8);
       for (int s = 0; s < k; ++s)
         if (fj[s] >= 0) put_nv(W.xt, W.sfx, fj[s] >> 8, H / 256, fj[s] & 255, b, q4, code);
     }
-    if (threadIdx.x < k && fj[threadIdx.x] >= 0) W.fac1[W.inv[t * k + threadIdx.x]] = pow2f_sub(cm - 135);
+    if (threadIdx.x < k && fj[threadIdx.x] >= 0) W.fac1[W.inv[t * k + threadIdx.x]] = actq_pow2(cm - 135);
     return;
   }
   for (int b = threadIdx.x; b < nb; b += kRowThreads) {
@@ -286,10 +275,10 @@ __global__ void __launch_bounds__(kRowThreads) k_gmx_hsplit(GroupWs W, int E, in
       float v[32];
       uint32_t q4[4];
       swiglu(b, v);
-      const uint32_t code = nv_pow2_code(actq_block_fp4(v, q4) - cm + 8);
+      const uint32_t code = actq_nv_code(actq_block_fp4(v, q4) - cm + 8);
       put_nv(W.ht, W.sfh, f, I / 256, j, b, q4, code);
     }
-    if (threadIdx.x == 0) W.fac2[r] = pow2f_sub(cm - 135);
+    if (threadIdx.x == 0) W.fac2[r] = actq_pow2(cm - 135);
     return;
   }
   for (int b = threadIdx.x; b < nb; b += kRowThreads) {

@@ -27,3 +27,33 @@ extern "C" void actq_host_fp4packed(const float* v, int n, uint8_t* packed, uint
     memcpy(packed + b * 16, q, 16);
   }
 }
+
+// The NVFP4 form of the same tiles (kind::mxf4nvf4): per row of n values
+// (n % 32 == 0) the packed codes, one ue4m3 code per 32-block (both 16-halves
+// take it) re-anchored at the row's largest 32-block code, and the row's
+// factor; the split kernels' two passes, in order.
+extern "C" void actq_host_nv_rows(const float* v, int rows, int n, uint8_t* packed, uint8_t* codes, float* fac) {
+  for (int r = 0; r < rows; ++r) {
+    const float* row = v + (size_t)r * n;
+    int cm = 0;
+    for (int b = 0; b < n / 32; ++b) {
+      float blk[32];
+      uint32_t q[4];
+      for (int i = 0; i < 32; ++i) blk[i] = row[b * 32 + i];
+      const int c = qk::actq_block_fp4(blk, q);
+      cm = cm > c ? cm : c;
+    }
+    for (int b = 0; b < n / 32; ++b) {
+      float blk[32];
+      uint32_t q[4];
+      for (int i = 0; i < 32; ++i) blk[i] = row[b * 32 + i];
+      const int c = qk::actq_block_fp4(blk, q);
+      codes[(size_t)r * (n / 32) + b] = (uint8_t)qk::actq_nv_code(c - cm + 8);
+      memcpy(packed + (size_t)r * (n / 2) + b * 16, q, 16);
+    }
+    fac[r] = qk::actq_pow2(cm - 135);
+  }
+}
+
+extern "C" unsigned actq_host_nv_code(int d) { return qk::actq_nv_code(d); }
+extern "C" float actq_host_pow2(int e) { return qk::actq_pow2(e); }

@@ -31,6 +31,12 @@ def host():
     L = ctypes.CDLL(OUT)
     L.actq_host.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
     L.actq_host_fp4packed.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    L.actq_host_nv_rows.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_void_p]
+    L.actq_host_nv_code.argtypes = [ctypes.c_int]
+    L.actq_host_nv_code.restype = ctypes.c_uint
+    L.actq_host_pow2.argtypes = [ctypes.c_int]
+    L.actq_host_pow2.restype = ctypes.c_float
 
     def run(v, fp4):
         v = np.ascontiguousarray(v, np.float32)
@@ -45,7 +51,17 @@ def host():
         scales = np.empty(v.size // 32, np.uint8)
         L.actq_host_fp4packed(v.ctypes.data, v.size, p.ctypes.data, scales.ctypes.data)
         return p, scales
+    def nv_rows(v):
+        v = np.ascontiguousarray(v, np.float32)
+        rows, n = v.shape
+        p = np.empty((rows, n // 2), np.uint8)
+        codes = np.empty((rows, n // 32), np.uint8)
+        fac = np.empty(rows, np.float32)
+        L.actq_host_nv_rows(v.ctypes.data, rows, n, p.ctypes.data, codes.ctypes.data, fac.ctypes.data)
+        return p, codes, fac
     run.packed = packed
+    run.nv_rows = nv_rows
+    run.lib = L
     return run
 
 
@@ -120,3 +136,47 @@ def test_packed_e2m1_matches_oracle_codes(host, kind):
     assert np.array_equal(scales, os_)
     assert np.array_equal(nib, oc)
 
+
+
+def test_nv_scale_code_is_the_e4m3_power_of_two(host):
+    """The ue4m3 code of 2^d that the NVFP4 fp4-mode tiles carry, for every d
+    the rule produces, against the ml_dtypes e4m3 decoder: exact for
+    -9 <= d <= 8 (subnormals 2^-9 .. 2^-7 included), 0 below."""
+    for d in range(-20, 9):
+        code = host.lib.actq_host_nv_code(d)
+        if d >= -9:
+            assert E4M3[code] == 2.0 ** d, (d, code)
+        else:
+            assert code == 0, (d, code)
+    for e in range(-149, 128):
+        assert float(host.lib.actq_host_pow2(e)) == 2.0 ** e, e
+
+
+def test_nv_rows_restore_the_mxfp4_scales(host):
+    """Per row: the packed codes are the MXFP4 mode's (the oracle's), and
+    every 32-block within 17 binades of the row's largest scale gets an
+    e4m3 code whose value times the row factor is 2^(c - 127) exactly (c the
+    oracle's e8m0 code); blocks further below get code 0 (dropped)."""
+    rng = np.random.default_rng(7)
+    rows = []
+    for r in range(24):
+        v = rng.standard_normal(512) * 2.0 ** rng.integers(-30, 30)
+        # blocks scaled down by up to 2^-40 (some far below the row's largest)
+        v *= np.repeat(2.0 ** -rng.integers(0, 41, 16), 32)
+        if r % 5 == 0:
+            v[32:64] = 0.0  # an all-zero block
+        rows.append(v)
+    v = np.asarray(rows, np.float32)
+    p, codes, fac = host.nv_rows(v)
+    for r in range(v.shape[0]):
+        oc, osc, _ = oracle.act_quant(v[r].astype(np.float64), oracle.ACT_MXFP4)
+        pm, sm = host.packed(v[r])
+        assert np.array_equal(p[r], pm)
+        assert np.array_equal(np.asarray(osc, np.uint8), sm)
+        cmax = int(np.max(sm))
+        assert float(fac[r]) == 2.0 ** (cmax - 135)
+        for b, c in enumerate(sm.astype(int)):
+            if c >= cmax - 17:
+                assert E4M3[codes[r, b]] * float(fac[r]) == 2.0 ** (c - 127), (r, b, c, cmax)
+            else:
+                assert codes[r, b] == 0, (r, b, c, cmax)
