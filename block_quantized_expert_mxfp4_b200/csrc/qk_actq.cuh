@@ -156,7 +156,9 @@ QK_HD float actq_pow2(int e) {
 
 namespace qk {
 // The grouped path with an activation mode (QK_ACT_*): group_forward is
-// group_forward_act(a, QK_ACT_NONE, ...), gmx_forward likewise.
+// group_forward_act(a, QK_ACT_NONE, ...); gmx_forward_act runs the x split
+// and the two block-scaled GEMMs (the sort and both tile lists are done, the
+// combine follows).
 qk_status group_forward_act(const DecodeArgs& a, int act_quant, void* workspace, cudaStream_t st);
 qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, cudaStream_t st);
 // Token tile heights of the grouped block-scaled path: 64 (gate/up, x as 2

@@ -860,10 +860,6 @@ static bool x_map_packed(CUtensorMap* m, const uint8_t* q, int64_t rows, int K, 
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
-qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st) {
-  return gmx_forward_act(a, W, QK_ACT_NONE, st);
-}
-
 qk_status gmx_forward_act(const DecodeArgs& a, const GroupWs& W, int act_quant, cudaStream_t st) {
   const int T = a.T, k = a.k, E = a.E, H = a.H, I = a.I;
   const bool fp4 = act_quant == QK_ACT_MXFP4, one = act_quant != QK_ACT_NONE;

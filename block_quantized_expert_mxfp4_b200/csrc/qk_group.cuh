@@ -73,10 +73,6 @@ qk_status gmx_fp8_ffn(const GroupWs& W, const uint16_t* x, const int32_t* ids, i
                       const uint8_t* wg, const uint8_t* sg, const uint8_t* wu, const uint8_t* su,
                       const uint8_t* wd, const uint8_t* sd, int blk, cudaStream_t st);
 
-// x split, gate/up GEMM, h split, down GEMM of the MXFP4 path (the counting
-// sort and both tile lists are done; the combine follows).
-qk_status gmx_forward(const DecodeArgs& a, const GroupWs& W, cudaStream_t st);
-
 inline int g_max_tiles(int P, int E, int tn) { return P / tn + E + 1; }
 
 }  // namespace qk
