@@ -396,8 +396,12 @@ def run_ours(args, rank, world, local_rank):
         out["prefill_w4a4_nvfp4_16k"] = run_prefill(args, rank, world, dev, tokens=16384, act="mxfp4", steps=3,
                                                     nv=True)
         out["shared_fp8_prefill"] = run_shared_fp8(args, rank, world, dev)
+        try:  # reported, never fatal to the line
+            out["convert"] = run_convert(args, rank, world, dev)
+        except Exception as e:  # noqa: BLE001
+            out["convert"] = {"error": f"{type(e).__name__}: {e}", "gpu_launches": 0}
         for key in ("decode_nvfp4", "stack43", "prefill_16k", "prefill_w4a8", "prefill_w4a4", "prefill_w4a4_16k",
-                    "prefill_w4a4_nvfp4", "prefill_w4a4_nvfp4_16k", "shared_fp8_prefill"):
+                    "prefill_w4a4_nvfp4", "prefill_w4a4_nvfp4_16k", "shared_fp8_prefill", "convert"):
             out["gpu_launches"] += out[key]["gpu_launches"]
     return out
 
@@ -430,6 +434,55 @@ def _graph_time(fn, K, world, dev, reps_warm=3):
     t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / K, world, dev)
     del g
     return t
+
+
+def run_convert(args, rank, world, dev):
+    """The scale-only conversions on the decode layer's three projections
+    (256 experts; gate and up 2048 x 4096, down 4096 x 2048): MXFP4 -> NVFP4
+    (e8m0 per 32 in, e4m3 per 16 and scale_2 out) and back; GB/s on the
+    bytes read and written, against the measured HBM rate."""
+    import torch
+
+    import block_quantized_expert_mxfp4_b200 as qk
+    from block_quantized_expert_mxfp4_b200 import synth, workload
+
+    wl = synth.WORKLOADS["decode_mx"]
+    layer = workload.make_layer(wl, rank, 0)
+    projs = (layer.gate, layer.up, layer.down)
+    e4 = [torch.empty((p.scales.shape[0], p.scales.shape[1], 2 * p.scales.shape[2]), dtype=torch.uint8,
+                      device=dev) for p in projs]
+    s2 = [torch.empty(p.scales.shape[0], dtype=torch.float32, device=dev) for p in projs]
+    back = [torch.empty_like(p.scales) for p in projs]
+    bad = torch.zeros(1, dtype=torch.int64, device=dev)
+    peak, peak_kind = peaks()
+    res = {"workload": "scale-only conversions of the decode layer's three projections (256 experts, "
+                       "hidden 4096, intermediate 2048; e8m0 codes uniform in 118..127)",
+           "peak_gbs": peak, "peak_kind": peak_kind}
+    K = 10
+    for name, fn, nbytes in (
+            ("mxfp4_to_nvfp4", lambda i: qk.quant_convert_mxfp4_to_nvfp4(projs[i].scales, e4[i], s2[i], bad),
+             sum(p.scales.numel() * 3 + p.scales.shape[0] * 4 for p in projs)),
+            ("nvfp4_to_mxfp4", lambda i: qk.quant_convert_nvfp4_to_mxfp4(e4[i], s2[i], back[i], bad),
+             sum(p.scales.numel() * 3 + p.scales.shape[0] * 4 for p in projs))):
+        for _ in range(2):
+            for i in range(3):
+                fn(i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            for i in range(3):
+                fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / K, world, dev)
+        res[name] = {"us_per_layer": round(t * 1e6, 2), "bytes_per_layer": int(nbytes),
+                     "achieved_gbs": round(nbytes / t / 1e9, 1), "frac": round(nbytes / t / 1e9 / peak, 4)}
+    if qk.qk_last_device_status() != qk.QK_OK:
+        raise RuntimeError("device status after the conversions")
+    res["round_trip_identity"] = bool(all(torch.equal(b, p.scales) for b, p in zip(back, projs)))
+    res["gpu_launches"] = 2 * (2 + K) * 3
+    return res
 
 
 def run_shared_fp8(args, rank, world, dev):
