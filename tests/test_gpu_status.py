@@ -155,3 +155,21 @@ def test_nan_scale_reported_block_scaled(T):
     ids, w = _bs_routing(T, 7 + T)
     _fwd_wl(BS, layer, x, torch.from_numpy(ids).cuda(), torch.from_numpy(w).float().cuda())
     assert qk.qk_last_device_status() == qk.QK_ERR_NAN_SCALE
+
+
+@pytest.mark.parametrize("code", [0x7F, 0xFF])
+def test_nan_e4m3_scale_reported_nvfp4_fp4_mode(code):
+    """An NVFP4 layer in QK_ACT_MXFP4 (the kind::mxf4nvf4 grouped kernels,
+    whose weight-scale warp checks e4m3 NaN codes 0x7F and 0xFF): one NaN
+    block scale in expert 3's up projection, 4 tokens."""
+    layer = workload.make_layer(BS, 8, 0, (2, 2, 2), nv_codes=(0x60, 0x7E))
+    layer.up.scales[3, 7, 2] = code
+    x = synth.activations(8, 4, BS.H)
+    ids, w = _bs_routing(4, 15)
+    lay = layer.c()
+    y = torch.zeros((4, BS.H), device="cuda")
+    ws = torch.empty(qk.moe_expert_workspace_size(lay, 4, BS.k, qk.QK_ACT_MXFP4), dtype=torch.uint8,
+                     device="cuda")
+    qk.moe_expert_forward(lay, x.cuda(), torch.from_numpy(ids).cuda(), torch.from_numpy(w).float().cuda(), y, ws,
+                          act_quant=qk.QK_ACT_MXFP4)
+    assert qk.qk_last_device_status() == qk.QK_ERR_NAN_SCALE
